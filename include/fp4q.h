@@ -1,0 +1,150 @@
+/*
+ * fp4q.h — C ABI of the fused block-Hadamard rotation + microscaling FP4 quantizer.
+ *
+ * What it computes.  The online activation path of MR-GPTQ-style FP4 inference
+ * ("Bridging the Gap Between Promise and Performance for Microscaling FP4 Quantization",
+ * gist.science/de/paper/2509.23202, Technische Zusammenfassung, 2. Methodik,
+ * GPU-Kernel-Unterstützung: the activation's block Hadamard rotation is fused into a
+ * lightweight quantization kernel computed online).  For a bf16 activation matrix X
+ * (M rows x K columns, row-major):
+ *
+ *   1. rotate every contiguous b-block of each row:  y = x_blk * H_b / sqrt(b), with the
+ *      Sylvester Hadamard matrix H_b in natural order (b = 1 means no rotation);
+ *   2. split each row into groups of g consecutive rotated values (g = 32 for MXFP4,
+ *      16 for NVFP4 — same page, 1. Problemstellung) and take the group amax A;
+ *   3. pick the group scale:
+ *        MXFP4: X = 2^e stored as the E8M0 byte e + 127 ("Unveiling the Potential of
+ *               Quantization with MXFP4", gist.science/nl/paper/2603.08713, Technische
+ *               samenvatting, Probleemstelling: E8M0, powers of two), with e by rule
+ *                 FP4Q_SCALE_FLOOR_OCP    e = floor(log2 A) - 2
+ *                 FP4Q_SCALE_CEIL_NOCLIP  e = ceil(log2(A / 6))   (A/X in (3, 6])
+ *                 FP4Q_SCALE_OAS          the ceil rule, then e - 1 when A/X is in
+ *                                         [3, 3.5] (same page, Methodologie 1,
+ *                                         Overflow-Aware Scaling)
+ *               e clamped to [-127, 127]; A = 0 gives byte 0;
+ *        NVFP4: an fp32 tensor scale s_g and E4M3 block scales
+ *               s_b = E4M3_RNE_satfinite(A / fp32(6 s_g)), element divisor
+ *               S = fp32(E4M3(s_b) s_g) (same page, Probleemstelling: E4M3 scales;
+ *               gist.science/es/paper/2509.23202, Resumen técnico 2.B: group and
+ *               tensor scales).  s_g = fp32(A_t / 2688) from the amax A_t of the whole
+ *               rotated tensor (1 when A_t = 0);
+ *   4. divide by the scale and round to E2M1 (magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6),
+ *      nearest with ties to the even code, saturating at 6, sign bit = sign of y;
+ *      a zero NV block scale gives all-zero codes;
+ *   5. pack two codes per byte, element 2j in the low nibble.
+ *
+ * Layout (all row-major, contiguous):
+ *   x        bf16  [M][K]          device memory, 16-byte aligned
+ *   codes    uint8 [M][K/2]        device memory, 16-byte aligned
+ *   scales   uint8 [M][K/g]        device memory, 16-byte aligned when K/g*M >= 16
+ *                                  (E8M0 bytes for MXFP4, E4M3 bytes for NVFP4)
+ *   tensor_scale  one fp32 in device memory (NVFP4 only; NULL for MXFP4)
+ *
+ * Shape rules: M >= 0, K >= 0, K a multiple of lcm(g, b), M*K < 2^40.  M*K = 0 is a valid
+ * empty call that launches nothing.
+ *
+ * Ownership.  The caller owns every buffer passed in.  A plan owns nothing on the device
+ * except, for FP4Q_SCALE_NV_DYNAMIC and for fp4q_amax, a small device array of per-CTA
+ * partial maxima that fp4q_plan_create allocates and fp4q_plan_destroy frees.  Calls
+ * allocate nothing.
+ *
+ * Streams.  Every call is asynchronous and stream-ordered on the given stream (a
+ * cudaStream_t passed as void*; NULL is the legacy default stream).  A plan is immutable
+ * after creation; two calls that share a DYNAMIC plan must be ordered on one stream
+ * (they share the plan's partial-maximum array).
+ *
+ * Errors.  Argument problems are found on the host before anything is launched and
+ * return FP4Q_ERR_ARG / _SHAPE / _ALIGN / _UNSUPPORTED.  A CUDA launch failure returns
+ * FP4Q_ERR_CUDA (fp4q_last_cuda_error gives the message).  No C++ exception crosses the
+ * ABI.  Every wait inside a kernel is bounded in time; a wait that runs out records a
+ * code that fp4q_device_status reads back (and clears) instead of hanging.
+ */
+#ifndef FP4Q_H_
+#define FP4Q_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FP4Q_OK = 0,
+  FP4Q_ERR_ARG = 1,          /* null pointer where one is required, bad plan handle  */
+  FP4Q_ERR_SHAPE = 2,        /* M, K outside the shape rules                          */
+  FP4Q_ERR_ALIGN = 3,        /* a pointer is not 16-byte aligned                      */
+  FP4Q_ERR_UNSUPPORTED = 4,  /* format / group / block / rule combination not offered */
+  FP4Q_ERR_CUDA = 5,         /* a CUDA runtime call failed                            */
+  FP4Q_ERR_TIMEOUT = 6       /* a bounded wait inside a kernel ran out                */
+} fp4q_status;
+
+typedef enum { FP4Q_MXFP4 = 0, FP4Q_NVFP4 = 1 } fp4q_format;
+
+typedef enum {
+  FP4Q_SCALE_FLOOR_OCP = 0,   /* MX: e = floor(log2 A) - 2; values above 6 X saturate  */
+  FP4Q_SCALE_CEIL_NOCLIP = 1, /* MX: e = ceil(log2(A/6)); overflow-aware, never clips  */
+  FP4Q_SCALE_OAS = 2,         /* MX: ceil rule, A/X in [3, 3.5] pushed to [6, 7]        */
+  FP4Q_SCALE_NV_STATIC = 3,   /* NV: caller supplies s_g in *tensor_scale (read only)  */
+  FP4Q_SCALE_NV_DYNAMIC = 4   /* NV: the call computes s_g from X and writes it        */
+} fp4q_scale_rule;
+
+typedef struct fp4q_plan_s* fp4q_plan;
+
+/* Create a plan.  format: fp4q_format; group: 32 (MXFP4) or 16 (NVFP4); hadamard_block:
+ * 1, 2, 4, ..., 128 (1 = no rotation); scale_rule: an fp4q_scale_rule valid for the
+ * format.  Writes the plan to *out.  FP4Q_SCALE_NV_DYNAMIC plans allocate their partial-
+ * maximum array on the current CUDA device, which every later call must also use. */
+fp4q_status fp4q_plan_create(fp4q_plan* out, int format, int group, int hadamard_block,
+                             int scale_rule);
+
+/* Free a plan (NULL is accepted).  Synchronizes nothing: the caller must make sure no
+ * call using the plan is still running on the device. */
+fp4q_status fp4q_plan_destroy(fp4q_plan plan);
+
+/* Rotate and quantize X in one pass over HBM (steps 1-5 above).
+ * x_bf16: device bf16 [M][K]; codes_out: device uint8 [M][K/2]; scales_out: device
+ * uint8 [M][K/g]; tensor_scale: device fp32 — NV static: read; NV dynamic: written with
+ * the s_g the call used; MX: ignored (may be NULL). */
+fp4q_status fp4q_rotate_quantize(fp4q_plan plan, const void* x_bf16, int64_t M, int64_t K,
+                                 void* codes_out, void* scales_out, float* tensor_scale,
+                                 void* stream);
+
+/* Same as fp4q_rotate_quantize, and also stores the fp32 rotated values y (before any
+ * scaling) to y_out (device fp32 [M][K]).  A debugging and testing aid: the same kernel
+ * body with one extra store. */
+fp4q_status fp4q_rotate_quantize_dump(fp4q_plan plan, const void* x_bf16, int64_t M, int64_t K,
+                                      void* codes_out, void* scales_out, float* tensor_scale,
+                                      float* y_out, void* stream);
+
+/* NVFP4 per-tensor scale: s_g = fp32(max|y| / 2688) over the rotated X (1 for an all-zero
+ * X), written to *tensor_scale_out (device fp32).  Uses the plan's block size; needs a
+ * plan made with an NV rule. */
+fp4q_status fp4q_amax(fp4q_plan plan, const void* x_bf16, int64_t M, int64_t K,
+                      float* tensor_scale_out, void* stream);
+
+/* Decode: out[r][k] = E2M1(code) * scale (MX: 2^(byte-127); NV: fp32(E4M3(byte) * s_g)),
+ * then, when unrotate != 0, the inverse rotation (H_b / sqrt(b) again, it is its own
+ * inverse).  codes, scales: device, layout as produced above; tensor_scale: device fp32
+ * (NV only); out_f32: device fp32 [M][K]. */
+fp4q_status fp4q_dequantize(fp4q_plan plan, const void* codes, const void* scales,
+                            const float* tensor_scale, int64_t M, int64_t K, int unrotate,
+                            float* out_f32, void* stream);
+
+/* Read and clear the device-side status word (FP4Q_OK, or FP4Q_ERR_TIMEOUT when a bounded
+ * wait ran out in a kernel since the last read).  Synchronizes the current device. */
+fp4q_status fp4q_device_status(void);
+
+/* Static string for a status code. */
+const char* fp4q_status_string(fp4q_status status);
+
+/* Message of the last CUDA error seen by this library on the calling thread (or ""). */
+const char* fp4q_last_cuda_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int fp4q_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP4Q_H_ */

@@ -1,0 +1,152 @@
+"""Plant plausible mistakes in the CPU oracle and check that its pins catch each one.
+
+Each mutation replaces one oracle function with a subtly wrong variant (a transposed or
+permuted operand, a dropped normalisation, a wrong tie direction, an off-by-one exponent,
+a swapped nibble order ...).  The pins in test_oracle_pins.py must then fail."""
+
+import math
+
+import numpy as np
+import pytest
+
+import oracle as o
+import oracle.fp4q_oracle as core
+import test_oracle_pins as pins
+
+
+def patch(monkeypatch, name, fn):
+    monkeypatch.setattr(core, name, fn)
+    monkeypatch.setattr(o, name, fn)
+
+
+def fails(fn, *args):
+    try:
+        fn(*args)
+    except AssertionError:
+        return True
+    return False
+
+
+_orig_H = core.sylvester_hadamard
+_orig_rotate = core.rotate
+_orig_e2m1 = core.e2m1_encode
+_orig_mx = core.mx_scale_exponent
+_orig_e4m3 = core.e4m3_encode
+_orig_pack = core.pack_nibbles
+
+
+def h_columns_swapped(b):
+    H = _orig_H(b).copy()
+    if b >= 2:
+        H[:, [b - 2, b - 1]] = H[:, [b - 1, b - 2]]
+    return H
+
+
+def h_wrong_sign(b):
+    H = _orig_H(b).copy()
+    if b >= 4:
+        H[1, 1] = -H[1, 1]
+    return H
+
+
+def rotate_unnormalised(x_bits, b):
+    return _orig_rotate(x_bits, b) * math.sqrt(b)
+
+
+def rotate_along_rows(x_bits, b):
+    """Rotates across M instead of along K when the shape allows it."""
+    x = np.asarray(x_bits)
+    if x.shape[0] % b == 0 and x.shape[0] >= b:
+        return _orig_rotate(np.ascontiguousarray(x.T), b).T
+    return _orig_rotate(np.roll(x, 1, axis=1), b)
+
+
+def e2m1_ties_away(v):
+    """Ties round away from zero instead of to the even code."""
+    v = np.asarray(v, np.float32)
+    c = _orig_e2m1(v)
+    a = np.abs(v.astype(np.float64))
+    for mid, up in ((0.25, 1), (0.75, 2), (1.25, 3), (1.75, 4), (2.5, 5), (3.5, 6), (5.0, 7)):
+        c = np.where(a == mid, (c & 8) | up, c)
+    return c.astype(np.uint8)
+
+
+def e2m1_no_sign(v):
+    return (_orig_e2m1(v) & 7).astype(np.uint8)
+
+
+def mx_floor_off_by_one(A32, rule):
+    e = _orig_mx(A32, rule)
+    if rule == o.SCALE_FLOOR_OCP:
+        e = np.where(np.asarray(A32) > 0, np.clip(e + 1, -127, 127), e)
+    return e
+
+
+def mx_ceil_wrong_threshold(A32, rule):
+    """ceil rule that bumps at m >= 1.5 instead of m > 1.5."""
+    e = _orig_mx(A32, rule)
+    if rule == o.SCALE_CEIL_NOCLIP:
+        A = np.asarray(A32, np.float64)
+        m = np.frexp(A)[0] * 2
+        e = np.where((A > 0) & (m == 1.5), e + 1, e)
+    return e
+
+
+def e4m3_ties_up(s):
+    s32 = np.asarray(s, np.float32)
+    c = _orig_e4m3(s32)
+    T = o.e4m3_table()
+    mids = (T[1:] + T[:-1]) / 2
+    a = s32.astype(np.float64)
+    hit = np.isin(a, mids)
+    idx = np.searchsorted(mids, a)
+    return np.where(hit, np.minimum(idx + 1, 126), c).astype(np.uint8)
+
+
+def pack_swapped(codes):
+    c = np.asarray(codes, np.uint8)
+    return (c[..., 1::2] | (c[..., 0::2] << 4)).astype(np.uint8)
+
+
+MUTATIONS = [
+    ("sylvester_hadamard", h_columns_swapped,
+     [(pins.test_sylvester_closed_form, 32), (pins.test_rotation_matches_fast_butterfly, 32)]),
+    ("sylvester_hadamard", h_wrong_sign,
+     [(pins.test_sylvester_closed_form, 16), (pins.test_rotation_of_basis_vectors_gives_rows, 16)]),
+    ("rotate", rotate_unnormalised,
+     [(pins.test_rotation_norm_inverse_and_gemm_identity, 32), (pins.test_rotation_matches_fast_butterfly, 16)]),
+    ("rotate", rotate_along_rows,
+     [(pins.test_rotation_matches_fast_butterfly, 16), (pins.test_rotation_of_basis_vectors_gives_rows, 32)]),
+    ("e2m1_encode", e2m1_ties_away,
+     [(pins.test_e2m1_dense_sweep_against_ml_dtypes_cast,), (pins.test_mx_worked_groups,)]),
+    ("e2m1_encode", e2m1_no_sign,
+     [(pins.test_e2m1_dense_sweep_against_ml_dtypes_cast,), (pins.test_mx_worked_groups,)]),
+    ("mx_scale_exponent", mx_floor_off_by_one,
+     [(pins.test_mx_exponent_brute_force, o.SCALE_FLOOR_OCP), (pins.test_mx_worked_groups,)]),
+    ("mx_scale_exponent", mx_ceil_wrong_threshold,
+     [(pins.test_mx_exponent_brute_force, o.SCALE_CEIL_NOCLIP), (pins.test_mx_worked_groups,)]),
+    ("e4m3_encode", e4m3_ties_up,
+     [(pins.test_e4m3_encode_against_torch_cast,)]),
+    ("pack_nibbles", pack_swapped,
+     [(pins.test_pack_nibbles_order,), (pins.test_mx_worked_groups,)]),
+]
+
+
+@pytest.mark.parametrize("name,fn,catchers", MUTATIONS, ids=[m[1].__name__ for m in MUTATIONS])
+def test_pins_catch_planted_mistake(monkeypatch, name, fn, catchers):
+    patch(monkeypatch, name, fn)
+    for catcher in catchers:
+        assert fails(catcher[0], *catcher[1:]), f"{catcher[0].__name__} missed {fn.__name__}"
+
+
+def test_nv_divisor_mistake_is_caught(monkeypatch):
+    """s_b computed with A / (448 s_g) instead of A / (6 s_g)."""
+    orig = core.rotate_quantize
+
+    def wrong(x_bits, fmt, group, block, rule, tensor_scale=None):
+        if fmt == o.NVFP4 and tensor_scale is not None:
+            tensor_scale = np.float32(tensor_scale) * np.float32(448.0 / 6.0)
+        return orig(x_bits, fmt, group, block, rule, tensor_scale)
+
+    patch(monkeypatch, "rotate_quantize", wrong)
+    assert fails(pins.test_nv_worked_groups)
