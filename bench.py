@@ -1,0 +1,525 @@
+#!/usr/bin/env python
+"""Benchmark of the fused block-Hadamard rotate + FP4 quantize path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step is one fp4q_rotate_quantize call over the whole workload (rotation, amax, scale,
+round, pack and store of every element).  The default workload is NVFP4 (group 16,
+Hadamard block 16, static per-tensor scale) on a 4096 x 4096 bf16 activation matrix.
+Inputs are resident in HBM when timing starts; successive steps cycle through enough
+distinct input/output buffers that every step reads from HBM, not L2.  Steps are replayed
+from CUDA graphs and timed with CUDA events on the launching stream.  Rank 0 prints one
+JSON line.
+
+Under torchrun (N > 1) every rank runs the same workload on its own GPU (rows are
+independent: no collective on the data path); the elapsed time is the max over ranks.
+
+--impl reference times the CPU oracle (as it stands) on a bounded sample of the same
+workload on the host cores and prints the same line with "impl": "reference".
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from microscaling_fp4_quantization_b200 import workloads as W  # noqa: E402
+
+METRIC = "fused rotate+FP4-quantize GB/s (bf16 in + packed out), % of B200 HBM peak"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "rotate_quantize_nvfp4_b16_4096x4096.md")
+KERNEL_SOURCES = ["fp4q.cu", "fp4q_kernels.cuh", "fp4q_device.cuh"]
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "microscaling_fp4_quantization_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, when
+    it was taken on the current kernel sources; else None."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    vals = {}
+    for line in text.splitlines():
+        line = line.strip().lstrip("-* ")
+        if ":" in line:
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    try:
+        return int(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons of one GPU while running (NVML, every 5 ms)."""
+
+    REASONS = {
+        "sw_power_cap": 0x4, "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80, "applications_clocks_setting": 0x2,
+    }
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": [k for k, v in self.REASONS.items() if self.reasons & v],
+                "samples": len(self.samples)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def time_graph_steps(torch, launch, n_buf: int, steps: int, warmup: int, stream):
+    """Capture `launch(i)` for i in 0..G-1 into a CUDA graph (i cycles the buffers) and time
+    `steps` steps.  Returns (ms total, n_graph_launches)."""
+    G = min(max(steps, 1), 256)
+    G = max(n_buf, (G // n_buf) * n_buf) if G >= n_buf else G
+    for i in range(max(warmup, 3)):
+        launch(i % n_buf)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(G):
+            launch(i % n_buf)
+    rem = steps % G
+    g_rem = None
+    if rem:
+        g_rem = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_rem, stream=stream):
+            for i in range(rem):
+                launch(i % n_buf)
+    reps = steps // G
+    # a short untimed soak so that the clocks settle under this load
+    g.replay()
+    torch.cuda.synchronize()
+    return g, g_rem, reps
+
+
+def run_gpu(args):
+    import torch
+    from microscaling_fp4_quantization_b200 import fp4q as F
+
+    world, rank, local = dist_setup()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = workload_for(args)
+    M, K = w.M, w.K
+    plan = F.fp4q_plan_create(w.fmt, w.group, w.block, w.rule)
+    x_np = w.generate()
+    bytes_call = w.bytes_per_call()
+    n_buf = max(1, math.ceil(3 * L2_BYTES / bytes_call)) if bytes_call < 2 * L2_BYTES else 1
+    n_buf = min(n_buf, 16)
+    x_host = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
+    xs = [x_host.to(dev, non_blocking=True) for _ in range(n_buf)]
+    codes = [torch.empty((M, K // 2), dtype=torch.uint8, device=dev) for _ in range(n_buf)]
+    scales = [torch.empty((M, K // w.group), dtype=torch.uint8, device=dev) for _ in range(n_buf)]
+    ts = torch.ones(1, dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+
+    extra = {}
+    is_nv = w.fmt == W.NVFP4
+    if is_nv:
+        # static per-tensor scale from the library's own amax pass, before timing
+        F.fp4q_amax(plan, xs[0], M, K, ts, stream=torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        extra["tensor_scale"] = float(ts.item())
+
+    def launch(i):
+        F.fp4q_rotate_quantize(plan, xs[i], M, K, codes[i], scales[i], ts if is_nv else None,
+                               stream=torch.cuda.current_stream())
+
+    with torch.cuda.stream(stream):
+        g, g_rem, reps = time_graph_steps(torch, launch, n_buf, args.steps, args.warmup, stream)
+    sampler = ClockSampler(dev.index if world == 1 else local)
+    sampler.start()
+    # soak: about half a second of the same replays, untimed, so the clock samples mean something
+    with torch.cuda.stream(stream):
+        t_end = time.time() + 0.5
+        while time.time() < t_end:
+            g.replay()
+            stream.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    sampler.stop()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    value = world * bytes_call * args.steps / (ms * 1e-3) / 1e9
+    kernel_us = ms_step * 1e3
+    peak, peak_kind = measured_peak()
+
+    # NVFP4: the amax pass and the dynamic mode (amax pass + quantize), timed on their own
+    if is_nv and rank == 0:
+        dyn = F.fp4q_plan_create(W.NVFP4, w.group, w.block, W.SCALE_NV_DYNAMIC)
+        ts_d = torch.empty(1, dtype=torch.float32, device=dev)
+
+        def launch_amax(i):
+            F.fp4q_amax(plan, xs[i], M, K, ts_d, stream=torch.cuda.current_stream())
+
+        def launch_dyn(i):
+            F.fp4q_rotate_quantize(dyn, xs[i], M, K, codes[i], scales[i], ts_d, stream=torch.cuda.current_stream())
+
+        for name, fn, nbytes in (("amax_pass", launch_amax, 2 * M * K), ("dynamic_mode", launch_dyn, bytes_call)):
+            steps2 = max(50, min(args.steps, 400))
+            with torch.cuda.stream(stream):
+                g2, g2r, reps2 = time_graph_steps(torch, fn, n_buf, steps2, 3, stream)
+                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a0.record(stream)
+                for _ in range(reps2):
+                    g2.replay()
+                if g2r is not None:
+                    g2r.replay()
+                a1.record(stream)
+            torch.cuda.synchronize()
+            us = a0.elapsed_time(a1) * 1e3 / steps2
+            extra[name] = {"us_per_call": round(us, 3), "GBps_algorithmic": round(nbytes / us / 1e3, 1),
+                           "bytes_per_call": nbytes}
+        extra["dynamic_mode"]["note"] = "reads X twice (amax pass, then quantize); bytes are the algorithmic ones"
+
+    # e2e: the public API with host buffers, H2D of X and D2H of codes + scales inside the region
+    e2e = None
+    if rank == 0 or world > 1:
+        codes_h = torch.empty((M, K // 2), dtype=torch.uint8).pin_memory()
+        scales_h = torch.empty((M, K // w.group), dtype=torch.uint8).pin_memory()
+        xd = xs[0]
+        n_e2e = max(3, min(20, args.steps))
+        cur = torch.cuda.current_stream()
+
+        def e2e_step():
+            xd.copy_(x_host, non_blocking=True)
+            F.fp4q_rotate_quantize(plan, xd, M, K, codes[0], scales[0], ts if is_nv else None, stream=cur)
+            codes_h.copy_(codes[0], non_blocking=True)
+            scales_h.copy_(scales[0], non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(cur)
+        for _ in range(n_e2e):
+            e2e_step()
+        b1.record(cur)
+        torch.cuda.synchronize()
+        e_ms = b0.elapsed_time(b1)
+        if world > 1:
+            import torch.distributed as dist
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": round(world * bytes_call * n_e2e / (e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": int(x_host.numel() * 2),
+               "d2h_bytes_per_step": int(codes_h.numel() + scales_h.numel()), "steps": n_e2e}
+
+    # the other workloads' throughput, each timed the same way (rank 0, when asked)
+    others = {}
+    if args.all_workloads and rank == 0:
+        for ow in (W.MX_8K_FLOOR, W.MX_8K_CEIL, W.PREFILL_NV, W.PREFILL_MX) + W.DECODE:
+            others[ow.name] = time_other(torch, F, ow, dev, stream, peak)
+
+    if rank == 0:
+        cpu = cpu_baseline(w, args) if world == 1 and not args.no_cpu_baseline else None
+        traffic = profiled_traffic()
+        line = {
+            "metric": METRIC,
+            "value": round(value, 2),
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_step, 6),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32",
+            "data": "synthetic (seeded; N(0,1) rows with 0.5% outlier channels x50, bf16)",
+            "config": {
+                "workload": w.name, "M": M, "K": K,
+                "format": "NVFP4" if is_nv else "MXFP4", "group": w.group, "hadamard_block": w.block,
+                "scale_rule": W.RULE_NAMES[w.rule], "bytes_per_step": bytes_call,
+                "l2": f"inputs larger than L2 per step: {n_buf} rotating buffer sets "
+                      f"({n_buf * bytes_call / 1e6:.0f} MB in total)" if n_buf > 1 else "input larger than L2",
+                "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            },
+            "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+            "pct_of_spec_8TBps": round(100 * value / world / SPEC_HBM_GBS, 2),
+            "elements_per_s": round(world * M * K / (ms_step * 1e-3), 1),
+            "roofline": {
+                "bound": "hbm",
+                "achieved": round(bytes_call / (kernel_us * 1e-6) / 1e9, 2),
+                "peak": peak,
+                "unit": "GB/s",
+                "frac": round(bytes_call / (kernel_us * 1e-6) / 1e9 / peak, 4),
+                "traffic": traffic,
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                else "fallback 6650 GB/s",
+                "kernel": "rotate_quantize_kernel", "us_per_launch": round(kernel_us, 3),
+            },
+            "gpu_launches": args.steps,
+            "clocks": sampler.summary(),
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "extra": extra,
+        }
+        if others:
+            line["workloads"] = others
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def workload_for(args):
+    w = W.BY_NAME[args.workload]
+    return w.with_rows(args.rows) if args.rows else w
+
+
+def run_kernel_only(args):
+    """W + K back-to-back launches of the workload's kernel on cuda:0, nothing else timed."""
+    import torch
+    from microscaling_fp4_quantization_b200 import fp4q as F
+    torch.cuda.set_device(0)
+    w = workload_for(args)
+    plan = F.fp4q_plan_create(w.fmt, w.group, w.block, w.rule)
+    x = torch.from_numpy(w.generate().view(np.int16)).view(torch.bfloat16).cuda()
+    codes = torch.empty((w.M, w.K // 2), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((w.M, w.K // w.group), dtype=torch.uint8, device="cuda")
+    ts = torch.ones(1, dtype=torch.float32, device="cuda")
+    if w.fmt == W.NVFP4:
+        F.fp4q_amax(plan, x, w.M, w.K, ts)
+    for _ in range(args.warmup + args.steps):
+        F.fp4q_rotate_quantize(plan, x, w.M, w.K, codes, scales, ts if w.fmt == W.NVFP4 else None)
+    torch.cuda.synchronize()
+    assert F.fp4q_device_status() == F.FP4Q_OK
+    print(f"kernel-only: {w.name} M={w.M} K={w.K} launches={args.warmup + args.steps}", flush=True)
+
+
+def time_other(torch, F, w, dev, stream, peak):
+    M, K = w.M, w.K
+    plan = F.fp4q_plan_create(w.fmt, w.group, w.block, w.rule)
+    x_np = w.generate()
+    bytes_call = w.bytes_per_call()
+    n_buf = max(1, math.ceil(3 * L2_BYTES / bytes_call)) if bytes_call < 2 * L2_BYTES else 1
+    n_buf = min(n_buf, 64)
+    xh = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16)
+    xs = [xh.to(dev) for _ in range(n_buf)]
+    del x_np, xh
+    codes = [torch.empty((M, K // 2), dtype=torch.uint8, device=dev) for _ in range(n_buf)]
+    scales = [torch.empty((M, K // w.group), dtype=torch.uint8, device=dev) for _ in range(n_buf)]
+    ts = torch.ones(1, dtype=torch.float32, device=dev)
+    if w.fmt == W.NVFP4:
+        F.fp4q_amax(plan, xs[0], M, K, ts, stream=torch.cuda.current_stream())
+
+    def launch(i):
+        F.fp4q_rotate_quantize(plan, xs[i], M, K, codes[i], scales[i], ts if w.fmt == W.NVFP4 else None,
+                               stream=torch.cuda.current_stream())
+
+    steps = 200 if bytes_call > 1e8 else 2000
+    with torch.cuda.stream(stream):
+        g, g_rem, reps = time_graph_steps(torch, launch, n_buf, steps, 5, stream)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        a1.record(stream)
+    torch.cuda.synchronize()
+    us = a0.elapsed_time(a1) * 1e3 / steps
+    gbs = bytes_call / us / 1e3
+    out = {"GBps": round(gbs, 1), "pct_of_hbm_peak": round(100 * gbs / peak, 2), "us_per_call": round(us, 3),
+           "bytes_per_call": bytes_call, "buffers": n_buf}
+    del xs, codes, scales
+    torch.cuda.empty_cache()
+    return out
+
+
+def cpu_baseline(w, args, seconds: float = 10.0):
+    """The oracle, as it stands, on a bounded sample of the workload's rows, on one host
+    thread; GB/s on the sample's algorithmic bytes."""
+    import oracle
+    from threadpoolctl import threadpool_limits
+
+    rows_per_batch = max(1, (1 << 20) // w.K)
+    x = None
+    for ch in w.row_chunks(chunk_rows=rows_per_batch):
+        x = ch
+        break
+    ts = None
+    if w.fmt == W.NVFP4:
+        ts = oracle.nv_tensor_scale(oracle.rotated_amax(x, w.block))
+    done_rows = 0
+    t0 = time.perf_counter()
+    with threadpool_limits(limits=1):
+        while True:
+            oracle.rotate_quantize(x, w.fmt, w.group, w.block, w.rule, tensor_scale=ts)
+            done_rows += x.shape[0]
+            if time.perf_counter() - t0 >= seconds:
+                break
+    dt = time.perf_counter() - t0
+    sample_bytes = w.with_rows(done_rows).bytes_per_call()
+    return {"value": round(sample_bytes / dt / 1e9, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{done_rows} rows x {w.K} ({x.shape[0]}-row batches of the same workload), "
+                      f"{dt:.1f} s wall on 1 host thread"}
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return
+    import oracle
+    from threadpoolctl import threadpool_limits
+    w = W.BY_NAME[args.workload]
+    rows = max(1, (1 << 18) // w.K)          # a bounded sample per step
+    x = next(iter(w.row_chunks(chunk_rows=rows)))
+    ts = oracle.nv_tensor_scale(oracle.rotated_amax(x, w.block)) if w.fmt == W.NVFP4 else None
+    cores = 1
+    with threadpool_limits(limits=cores):
+        for _ in range(args.warmup):
+            oracle.rotate_quantize(x, w.fmt, w.group, w.block, w.rule, tensor_scale=ts)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            oracle.rotate_quantize(x, w.fmt, w.group, w.block, w.rule, tensor_scale=ts)
+        dt = time.perf_counter() - t0
+    sb = w.with_rows(x.shape[0]).bytes_per_call()
+    value = sb * args.steps / dt / 1e9
+    line = {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 5), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": w.name, "M": w.M, "K": w.K, "sample_rows_per_step": x.shape[0]},
+        "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{x.shape[0]} rows x {w.K} per step"},
+        "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=W.NV_4K.name, choices=sorted(W.BY_NAME))
+    ap.add_argument("--impl", default="fp4q", choices=["fp4q", "reference"])
+    ap.add_argument("--all-workloads", action="store_true", help="also time the other workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rows", type=int, default=0, help="override the workload's row count M")
+    ap.add_argument("--kernel-only", action="store_true",
+                    help="only W + K plain launches of the workload (a case for profilers), no JSON line")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    elif args.kernel_only:
+        run_kernel_only(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,332 @@
+// C ABI of the fused rotate + FP4 quantizer (declared in include/fp4q.h): plan objects,
+// host-side validation, kernel selection and launch on the caller's stream.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <unordered_map>
+
+#include "fp4q.h"
+#include "fp4q_kernels.cuh"
+
+using namespace fp4q;
+
+struct fp4q_plan_s {
+  uint32_t magic;
+  int format, group, block, rule;
+  int unit;        // E = max(block, group)
+  int device;
+  float* partials; // NV plans: per-CTA rotated amaxima (device)
+  int n_partials;
+};
+
+namespace {
+
+constexpr uint32_t kPlanMagic = 0xF4F4A11Cu;
+thread_local char g_last_cuda_error[512] = "";
+
+fp4q_status cuda_fail(cudaError_t e, const char* what) {
+  std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s (%s)", what, cudaGetErrorString(e),
+                cudaGetErrorName(e));
+  return FP4Q_ERR_CUDA;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool valid_plan(fp4q_plan p) { return p != nullptr && p->magic == kPlanMagic; }
+
+// Per (kernel, device) one-time set-up: opt in to the dynamic shared memory the kernel
+// needs and record how many CTAs fit on one SM.
+struct KernelInfo {
+  int ctas_per_sm = 0;
+  int sm_count = 0;
+};
+
+std::mutex g_info_mu;
+std::unordered_map<uint64_t, KernelInfo> g_info;
+
+template <class K>
+fp4q_status kernel_info(K kernel, int smem_bytes, int threads, KernelInfo* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  const uint64_t key = (reinterpret_cast<uint64_t>(reinterpret_cast<const void*>(kernel)) << 8) ^ static_cast<uint64_t>(dev);
+  std::lock_guard<std::mutex> lk(g_info_mu);
+  auto it = g_info.find(key);
+  if (it != g_info.end()) {
+    *out = it->second;
+    return FP4Q_OK;
+  }
+  KernelInfo ki;
+  e = cudaDeviceGetAttribute(&ki.sm_count, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ki.ctas_per_sm, kernel, threads, smem_bytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+  if (ki.ctas_per_sm < 1) ki.ctas_per_sm = 1;
+  g_info[key] = ki;
+  *out = ki;
+  return FP4Q_OK;
+}
+
+// Call f.template operator()<B>() for the runtime Hadamard block b.
+template <class F>
+fp4q_status with_block(int b, F&& f) {
+  switch (b) {
+    case 1: return f.template operator()<1>();
+    case 2: return f.template operator()<2>();
+    case 4: return f.template operator()<4>();
+    case 8: return f.template operator()<8>();
+    case 16: return f.template operator()<16>();
+    case 32: return f.template operator()<32>();
+    case 64: return f.template operator()<64>();
+    case 128: return f.template operator()<128>();
+    default: return FP4Q_ERR_UNSUPPORTED;
+  }
+}
+
+template <class Cfg>
+fp4q_status launch_rq(const RQArgs& a, cudaStream_t stream) {
+  auto kernel = rotate_quantize_kernel<Cfg>;
+  KernelInfo ki;
+  fp4q_status st = kernel_info(kernel, Cfg::kSmemBytes, Cfg::kThreads, &ki);
+  if (st != FP4Q_OK) return st;
+  const int64_t warps_needed = (a.n_units + Cfg::kUnitsPerStage - 1) / Cfg::kUnitsPerStage;
+  int64_t ctas = (warps_needed + Cfg::kWarps - 1) / Cfg::kWarps;
+  const int64_t max_ctas = static_cast<int64_t>(ki.sm_count) * ki.ctas_per_sm;
+  if (ctas > max_ctas) ctas = max_ctas;
+  kernel<<<static_cast<unsigned>(ctas), Cfg::kThreads, Cfg::kSmemBytes, stream>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "rotate_quantize launch");
+  return FP4Q_OK;
+}
+
+template <int B>
+using AmaxCfg = RQConfig<kNV, B, kRuleNvStatic, false>;
+
+// Number of CTAs the amax pass always launches (and of partial maxima a plan holds).
+fp4q_status amax_grid(int b, int* n) {
+  return with_block(b, [&]<int B>() -> fp4q_status {
+    KernelInfo ki;
+    fp4q_status st = kernel_info(rotated_amax_kernel<AmaxCfg<B>>, AmaxCfg<B>::kSmemBytes, AmaxCfg<B>::kThreads, &ki);
+    if (st != FP4Q_OK) return st;
+    *n = ki.sm_count * ki.ctas_per_sm;
+    return FP4Q_OK;
+  });
+}
+
+fp4q_status launch_amax(fp4q_plan p, const uint16_t* x, int64_t n_units, cudaStream_t stream) {
+  return with_block(p->block, [&]<int B>() -> fp4q_status {
+    using Cfg = AmaxCfg<B>;
+    rotated_amax_kernel<Cfg><<<p->n_partials, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(x, n_units, p->partials);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "amax launch");
+    return FP4Q_OK;
+  });
+}
+
+fp4q_status check_shape(fp4q_plan p, int64_t M, int64_t K) {
+  if (M < 0 || K < 0) return FP4Q_ERR_SHAPE;
+  if (K % p->unit != 0) return FP4Q_ERR_SHAPE;  // unit = lcm(group, block) for powers of two
+  if (M > 0 && K > 0 && M > (int64_t(1) << 40) / K) return FP4Q_ERR_SHAPE;
+  return FP4Q_OK;
+}
+
+fp4q_status rotate_quantize_impl(fp4q_plan p, const void* x, int64_t M, int64_t K, void* codes, void* scales,
+                                 float* tensor_scale, float* y_out, bool dump, void* stream) {
+  if (!valid_plan(p)) return FP4Q_ERR_ARG;
+  fp4q_status st = check_shape(p, M, K);
+  if (st != FP4Q_OK) return st;
+  if (M * K == 0) return FP4Q_OK;
+  if (!x || !codes || !scales || (dump && !y_out)) return FP4Q_ERR_ARG;
+  if (p->format == FP4Q_NVFP4 && !tensor_scale) return FP4Q_ERR_ARG;
+  if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, 16) || (dump && !aligned(y_out, 16)) ||
+      (tensor_scale && !aligned(tensor_scale, 4)))
+    return FP4Q_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  RQArgs a;
+  a.x = static_cast<const uint16_t*>(x);
+  a.n_units = (M * K) / p->unit;
+  a.codes = static_cast<uint8_t*>(codes);
+  a.scales = static_cast<uint8_t*>(scales);
+  a.tensor_scale = tensor_scale;
+  a.partials = p->partials;
+  a.n_partials = p->n_partials;
+  a.y_dump = y_out;
+  if (p->format == FP4Q_NVFP4 && p->rule == FP4Q_SCALE_NV_DYNAMIC) {
+    st = launch_amax(p, a.x, a.n_units, s);
+    if (st != FP4Q_OK) return st;
+  }
+  return with_block(p->block, [&]<int B>() -> fp4q_status {
+    if (p->format == FP4Q_MXFP4) {
+      switch (p->rule) {
+        case FP4Q_SCALE_FLOOR_OCP:
+          return dump ? launch_rq<RQConfig<kMX, B, kRuleFloor, true>>(a, s)
+                      : launch_rq<RQConfig<kMX, B, kRuleFloor, false>>(a, s);
+        case FP4Q_SCALE_CEIL_NOCLIP:
+          return dump ? launch_rq<RQConfig<kMX, B, kRuleCeil, true>>(a, s)
+                      : launch_rq<RQConfig<kMX, B, kRuleCeil, false>>(a, s);
+        case FP4Q_SCALE_OAS:
+          return dump ? launch_rq<RQConfig<kMX, B, kRuleOas, true>>(a, s)
+                      : launch_rq<RQConfig<kMX, B, kRuleOas, false>>(a, s);
+        default: return FP4Q_ERR_UNSUPPORTED;
+      }
+    }
+    if (p->rule == FP4Q_SCALE_NV_DYNAMIC)
+      return dump ? launch_rq<RQConfig<kNV, B, kRuleNvDynamic, true>>(a, s)
+                  : launch_rq<RQConfig<kNV, B, kRuleNvDynamic, false>>(a, s);
+    return dump ? launch_rq<RQConfig<kNV, B, kRuleNvStatic, true>>(a, s)
+                : launch_rq<RQConfig<kNV, B, kRuleNvStatic, false>>(a, s);
+  });
+}
+
+}  // namespace
+
+extern "C" {
+
+fp4q_status fp4q_plan_create(fp4q_plan* out, int format, int group, int hadamard_block, int scale_rule) {
+  if (!out) return FP4Q_ERR_ARG;
+  *out = nullptr;
+  if (format == FP4Q_MXFP4) {
+    if (group != 32) return FP4Q_ERR_UNSUPPORTED;
+    if (scale_rule != FP4Q_SCALE_FLOOR_OCP && scale_rule != FP4Q_SCALE_CEIL_NOCLIP && scale_rule != FP4Q_SCALE_OAS)
+      return FP4Q_ERR_UNSUPPORTED;
+  } else if (format == FP4Q_NVFP4) {
+    if (group != 16) return FP4Q_ERR_UNSUPPORTED;
+    if (scale_rule != FP4Q_SCALE_NV_STATIC && scale_rule != FP4Q_SCALE_NV_DYNAMIC) return FP4Q_ERR_UNSUPPORTED;
+  } else {
+    return FP4Q_ERR_UNSUPPORTED;
+  }
+  if (hadamard_block < 1 || hadamard_block > 128 || (hadamard_block & (hadamard_block - 1)) != 0)
+    return FP4Q_ERR_UNSUPPORTED;
+  fp4q_plan p = new (std::nothrow) fp4q_plan_s();
+  if (!p) return FP4Q_ERR_ARG;
+  p->magic = kPlanMagic;
+  p->format = format;
+  p->group = group;
+  p->block = hadamard_block;
+  p->rule = scale_rule;
+  p->unit = group > hadamard_block ? group : hadamard_block;
+  p->device = -1;
+  p->partials = nullptr;
+  p->n_partials = 0;
+  if (format == FP4Q_NVFP4) {
+    cudaError_t e = cudaGetDevice(&p->device);
+    fp4q_status st = e == cudaSuccess ? amax_grid(hadamard_block, &p->n_partials) : cuda_fail(e, "cudaGetDevice");
+    if (st == FP4Q_OK) {
+      e = cudaMalloc(&p->partials, sizeof(float) * static_cast<size_t>(p->n_partials));
+      if (e != cudaSuccess) st = cuda_fail(e, "cudaMalloc partials");
+    }
+    if (st != FP4Q_OK) {
+      p->magic = 0;
+      delete p;
+      return st;
+    }
+  }
+  *out = p;
+  return FP4Q_OK;
+}
+
+fp4q_status fp4q_plan_destroy(fp4q_plan plan) {
+  if (!plan) return FP4Q_OK;
+  if (!valid_plan(plan)) return FP4Q_ERR_ARG;
+  fp4q_status st = FP4Q_OK;
+  if (plan->partials) {
+    cudaError_t e = cudaFree(plan->partials);
+    if (e != cudaSuccess) st = cuda_fail(e, "cudaFree partials");
+  }
+  plan->magic = 0;
+  delete plan;
+  return st;
+}
+
+fp4q_status fp4q_rotate_quantize(fp4q_plan plan, const void* x_bf16, int64_t M, int64_t K, void* codes_out,
+                                 void* scales_out, float* tensor_scale, void* stream) {
+  return rotate_quantize_impl(plan, x_bf16, M, K, codes_out, scales_out, tensor_scale, nullptr, false, stream);
+}
+
+fp4q_status fp4q_rotate_quantize_dump(fp4q_plan plan, const void* x_bf16, int64_t M, int64_t K, void* codes_out,
+                                      void* scales_out, float* tensor_scale, float* y_out, void* stream) {
+  return rotate_quantize_impl(plan, x_bf16, M, K, codes_out, scales_out, tensor_scale, y_out, true, stream);
+}
+
+fp4q_status fp4q_amax(fp4q_plan plan, const void* x_bf16, int64_t M, int64_t K, float* tensor_scale_out,
+                      void* stream) {
+  if (!valid_plan(plan)) return FP4Q_ERR_ARG;
+  if (plan->format != FP4Q_NVFP4) return FP4Q_ERR_UNSUPPORTED;
+  fp4q_status st = check_shape(plan, M, K);
+  if (st != FP4Q_OK) return st;
+  if (!tensor_scale_out) return FP4Q_ERR_ARG;
+  if (M * K > 0 && !x_bf16) return FP4Q_ERR_ARG;
+  if ((x_bf16 && !aligned(x_bf16, 16)) || !aligned(tensor_scale_out, 4)) return FP4Q_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = launch_amax(plan, static_cast<const uint16_t*>(x_bf16), (M * K) / plan->unit, s);
+  if (st != FP4Q_OK) return st;
+  tensor_scale_finalize_kernel<<<1, 32, 0, s>>>(plan->partials, plan->n_partials, tensor_scale_out);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "finalize launch");
+  return FP4Q_OK;
+}
+
+fp4q_status fp4q_dequantize(fp4q_plan plan, const void* codes, const void* scales, const float* tensor_scale,
+                            int64_t M, int64_t K, int unrotate, float* out_f32, void* stream) {
+  if (!valid_plan(plan)) return FP4Q_ERR_ARG;
+  fp4q_status st = check_shape(plan, M, K);
+  if (st != FP4Q_OK) return st;
+  if (M * K == 0) return FP4Q_OK;
+  if (!codes || !scales || !out_f32 || (plan->format == FP4Q_NVFP4 && !tensor_scale)) return FP4Q_ERR_ARG;
+  if (!aligned(codes, 16) || !aligned(scales, 16) || !aligned(out_f32, 16) ||
+      (tensor_scale && !aligned(tensor_scale, 4)))
+    return FP4Q_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t n_units = (M * K) / plan->unit;
+  const unsigned grid = static_cast<unsigned>((n_units + 127) / 128);
+  const uint8_t* c = static_cast<const uint8_t*>(codes);
+  const uint8_t* sc = static_cast<const uint8_t*>(scales);
+  st = with_block(plan->block, [&]<int B>() -> fp4q_status {
+    if (plan->format == FP4Q_MXFP4) {
+      if (unrotate) dequantize_kernel<kMX, B, true><<<grid, 128, 0, s>>>(c, sc, tensor_scale, n_units, out_f32);
+      else dequantize_kernel<kMX, B, false><<<grid, 128, 0, s>>>(c, sc, tensor_scale, n_units, out_f32);
+    } else {
+      if (unrotate) dequantize_kernel<kNV, B, true><<<grid, 128, 0, s>>>(c, sc, tensor_scale, n_units, out_f32);
+      else dequantize_kernel<kNV, B, false><<<grid, 128, 0, s>>>(c, sc, tensor_scale, n_units, out_f32);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");
+    return FP4Q_OK;
+  });
+  return st;
+}
+
+fp4q_status fp4q_device_status(void) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  unsigned int v = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyFromSymbol");
+  e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol");
+  return (v & kStatusTimeout) ? FP4Q_ERR_TIMEOUT : FP4Q_OK;
+}
+
+const char* fp4q_status_string(fp4q_status status) {
+  switch (status) {
+    case FP4Q_OK: return "ok";
+    case FP4Q_ERR_ARG: return "invalid argument";
+    case FP4Q_ERR_SHAPE: return "invalid shape (K must be a multiple of max(group, hadamard_block))";
+    case FP4Q_ERR_ALIGN: return "pointer not aligned (16 bytes for arrays, 4 for the tensor scale)";
+    case FP4Q_ERR_UNSUPPORTED: return "unsupported format / group / block / rule";
+    case FP4Q_ERR_CUDA: return "CUDA error";
+    case FP4Q_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
+  }
+  return "unknown status";
+}
+
+const char* fp4q_last_cuda_error(void) { return g_last_cuda_error; }
+
+int fp4q_version(void) { return 100; }
+
+}  // extern "C"

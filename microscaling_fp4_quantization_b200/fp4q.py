@@ -1,0 +1,179 @@
+"""Python binding of the fp4q C ABI (include/fp4q.h), through ctypes.
+
+The functions carry the C names and do argument marshalling only: every step of the
+rotate + quantize path runs in the library's CUDA kernels.  PyTorch tensors are used as
+device allocations and streams.  Importing this module loads lib/libfp4q.so and raises
+ImportError when it is missing; there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libfp4q.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"fp4q native library not built: {LIB_PATH} (run python -m "
+                      "microscaling_fp4_quantization_b200.build)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+FP4Q_OK, FP4Q_ERR_ARG, FP4Q_ERR_SHAPE, FP4Q_ERR_ALIGN, FP4Q_ERR_UNSUPPORTED, FP4Q_ERR_CUDA, FP4Q_ERR_TIMEOUT = range(7)
+FP4Q_MXFP4, FP4Q_NVFP4 = 0, 1
+(FP4Q_SCALE_FLOOR_OCP, FP4Q_SCALE_CEIL_NOCLIP, FP4Q_SCALE_OAS,
+ FP4Q_SCALE_NV_STATIC, FP4Q_SCALE_NV_DYNAMIC) = range(5)
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+
+_SIGS = {
+    "fp4q_plan_create": (_int, [ctypes.POINTER(_vp), _int, _int, _int, _int]),
+    "fp4q_plan_destroy": (_int, [_vp]),
+    "fp4q_rotate_quantize": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "fp4q_rotate_quantize_dump": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
+    "fp4q_amax": (_int, [_vp, _vp, _i64, _i64, _vp, _vp]),
+    "fp4q_dequantize": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _int, _vp, _vp]),
+    "fp4q_device_status": (_int, []),
+    "fp4q_status_string": (ctypes.c_char_p, [_int]),
+    "fp4q_last_cuda_error": (ctypes.c_char_p, []),
+    "fp4q_version": (_int, []),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+EXPORTED = tuple(_SIGS)
+
+
+class Fp4qError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = _lib.fp4q_status_string(status).decode()
+        if status == FP4Q_ERR_CUDA:
+            msg += ": " + _lib.fp4q_last_cuda_error().decode()
+        super().__init__(f"{where}: {msg} (status {status})")
+        self.status = status
+
+
+def _check(status: int, where: str) -> None:
+    if status != FP4Q_OK:
+        raise Fp4qError(status, where)
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+class Plan:
+    """An fp4q plan handle (format, group, Hadamard block, scale rule)."""
+
+    def __init__(self, handle: int, fmt: int, group: int, block: int, rule: int):
+        self.handle = handle
+        self.fmt, self.group, self.block, self.rule = fmt, group, block, rule
+
+    def __del__(self):
+        h, self.handle = getattr(self, "handle", None), None
+        if h:
+            try:
+                _lib.fp4q_plan_destroy(h)
+            except Exception:
+                pass
+
+    @property
+    def unit(self) -> int:
+        return max(self.group, self.block)
+
+
+# ---------------------------------------------------------------- the C names
+
+def fp4q_plan_create(fmt: int, group: int, hadamard_block: int, scale_rule: int) -> Plan:
+    h = _vp()
+    _check(_lib.fp4q_plan_create(ctypes.byref(h), fmt, group, hadamard_block, scale_rule), "fp4q_plan_create")
+    return Plan(h.value, fmt, group, hadamard_block, scale_rule)
+
+
+def fp4q_plan_destroy(plan: Plan) -> None:
+    h, plan.handle = plan.handle, None
+    _check(_lib.fp4q_plan_destroy(h), "fp4q_plan_destroy")
+
+
+def fp4q_rotate_quantize(plan: Plan, x, M: int, K: int, codes_out, scales_out, tensor_scale=None,
+                         stream=None) -> None:
+    _check(_lib.fp4q_rotate_quantize(plan.handle, _ptr(x), M, K, _ptr(codes_out), _ptr(scales_out),
+                                     _ptr(tensor_scale), _stream(stream)), "fp4q_rotate_quantize")
+
+
+def fp4q_rotate_quantize_dump(plan: Plan, x, M: int, K: int, codes_out, scales_out, tensor_scale, y_out,
+                              stream=None) -> None:
+    _check(_lib.fp4q_rotate_quantize_dump(plan.handle, _ptr(x), M, K, _ptr(codes_out), _ptr(scales_out),
+                                          _ptr(tensor_scale), _ptr(y_out), _stream(stream)),
+           "fp4q_rotate_quantize_dump")
+
+
+def fp4q_amax(plan: Plan, x, M: int, K: int, tensor_scale_out, stream=None) -> None:
+    _check(_lib.fp4q_amax(plan.handle, _ptr(x), M, K, _ptr(tensor_scale_out), _stream(stream)), "fp4q_amax")
+
+
+def fp4q_dequantize(plan: Plan, codes, scales, tensor_scale, M: int, K: int, unrotate: bool, out_f32,
+                    stream=None) -> None:
+    _check(_lib.fp4q_dequantize(plan.handle, _ptr(codes), _ptr(scales), _ptr(tensor_scale), M, K,
+                                int(bool(unrotate)), _ptr(out_f32), _stream(stream)), "fp4q_dequantize")
+
+
+def fp4q_device_status() -> int:
+    return _lib.fp4q_device_status()
+
+
+def fp4q_status_string(status: int) -> str:
+    return _lib.fp4q_status_string(status).decode()
+
+
+def fp4q_version() -> int:
+    return _lib.fp4q_version()
+
+
+def raw_call(name: str, *args) -> int:
+    """Call a C entry point with raw arguments and return its status (for tests of the
+    host-side argument checks)."""
+    return getattr(_lib, name)(*args)
+
+
+# ---------------------------------------------------------------- tensor conveniences
+
+def empty_outputs(plan: Plan, M: int, K: int, device="cuda"):
+    """Allocate codes (uint8 [M, K/2]), scales (uint8 [M, K/g]) and the fp32 tensor scale."""
+    import torch
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
+    scales = torch.empty((M, K // plan.group), dtype=torch.uint8, device=device)
+    ts = torch.empty((1,), dtype=torch.float32, device=device)
+    return codes, scales, ts
+
+
+def rotate_quantize(plan: Plan, x, tensor_scale=None, stream=None) -> Tuple[object, object, object]:
+    """x: bf16 CUDA tensor [M, K] -> (codes, scales, tensor_scale)."""
+    import torch
+    if x.dtype != torch.bfloat16 or not x.is_cuda or x.dim() != 2 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous 2-D bf16 CUDA tensor")
+    M, K = x.shape
+    codes, scales, ts = empty_outputs(plan, M, K, x.device)
+    if tensor_scale is not None:
+        ts = tensor_scale
+    fp4q_rotate_quantize(plan, x, M, K, codes, scales, ts if plan.fmt == FP4Q_NVFP4 else None, stream)
+    return codes, scales, ts

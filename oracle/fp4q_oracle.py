@@ -256,10 +256,15 @@ def check_plan(fmt: int, group: int, block: int, rule: int) -> None:
     sylvester_hadamard(block)
 
 
-def rotated_amax(x_bits: np.ndarray, block: int) -> np.float32:
-    """max |y| over the whole tensor, taken on the fp32 rotated values."""
-    y32 = rotate(x_bits, block).astype(np.float32)
-    return np.float32(np.max(np.abs(y32))) if y32.size else np.float32(0)
+def rotated_amax(x_bits: np.ndarray, block: int, chunk_rows: int = 512) -> np.float32:
+    """max |y| over the whole tensor, taken on the fp32 rotated values (row chunks keep the
+    fp64 intermediate small)."""
+    m = np.float32(0)
+    for r in range(0, x_bits.shape[0], chunk_rows):
+        y32 = rotate(x_bits[r:r + chunk_rows], block).astype(np.float32)
+        if y32.size:
+            m = max(m, np.float32(np.max(np.abs(y32))))
+    return np.float32(m)
 
 
 def rotate_quantize(x_bits: np.ndarray, fmt: int, group: int, block: int, rule: int,

@@ -1,0 +1,87 @@
+"""The C ABI library, without a GPU: it loads, it exports every function include/*.h
+declares, and argument errors come back as status codes before any CUDA call."""
+
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def F():
+    from microscaling_fp4_quantization_b200 import build
+    build.build()
+    from microscaling_fp4_quantization_b200 import fp4q
+    return fp4q
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names |= set(re.findall(r"\b(fp4q_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported(F):
+    names = declared_functions()
+    assert "fp4q_rotate_quantize" in names and "fp4q_plan_create" in names
+    lib = ctypes.CDLL(F.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(F.EXPORTED) | {n for n in names if hasattr(lib, n)}
+
+
+def test_version_and_strings(F):
+    assert F.fp4q_version() >= 100
+    for s in range(7):
+        assert F.fp4q_status_string(s)
+
+
+def test_plan_validation_without_gpu(F):
+    for args in [(0, 16, 32, 0), (1, 32, 16, 3), (0, 32, 3, 0), (0, 32, 256, 0), (0, 32, 32, 3), (1, 16, 16, 0),
+                 (2, 32, 32, 0), (0, 32, 0, 0)]:
+        with pytest.raises(F.Fp4qError) as e:
+            F.fp4q_plan_create(*args)
+        assert e.value.status == F.FP4Q_ERR_UNSUPPORTED, args
+    assert F.raw_call("fp4q_plan_create", None, 0, 32, 32, 0) == F.FP4Q_ERR_ARG
+    # MX plans allocate nothing on the device, so they can be made on a CPU-only machine
+    p = F.fp4q_plan_create(F.FP4Q_MXFP4, 32, 32, F.FP4Q_SCALE_FLOOR_OCP)
+    F.fp4q_plan_destroy(p)
+    assert F.raw_call("fp4q_plan_destroy", None) == F.FP4Q_OK
+
+
+def test_call_validation_without_gpu(F):
+    p = F.fp4q_plan_create(F.FP4Q_MXFP4, 32, 128, F.FP4Q_SCALE_FLOOR_OCP)
+    rq = lambda *a: F.raw_call("fp4q_rotate_quantize", *a)
+    A = 1 << 20            # an aligned fake address: never dereferenced, validation fails first
+    assert rq(None, A, 4, 128, A, A, None, None) == F.FP4Q_ERR_ARG
+    assert rq(p.handle, A, 4, 96, A, A, None, None) == F.FP4Q_ERR_SHAPE        # K % 128
+    assert rq(p.handle, A, -1, 128, A, A, None, None) == F.FP4Q_ERR_SHAPE
+    assert rq(p.handle, A, 1 << 34, 1 << 7, A, A, None, None) == F.FP4Q_ERR_SHAPE   # > 2^40 elements
+    assert rq(p.handle, None, 4, 128, A, A, None, None) == F.FP4Q_ERR_ARG
+    assert rq(p.handle, A, 4, 128, None, A, None, None) == F.FP4Q_ERR_ARG
+    assert rq(p.handle, A + 8, 4, 128, A, A, None, None) == F.FP4Q_ERR_ALIGN
+    assert rq(p.handle, A, 4, 128, A + 4, A, None, None) == F.FP4Q_ERR_ALIGN
+    assert rq(p.handle, A, 4, 128, A, A + 2, None, None) == F.FP4Q_ERR_ALIGN
+    assert rq(p.handle, A, 0, 128, None, None, None, None) == F.FP4Q_OK          # empty call
+    dq = lambda *a: F.raw_call("fp4q_dequantize", *a)
+    assert dq(p.handle, A, A, None, 4, 100, 0, A, None) == F.FP4Q_ERR_SHAPE
+    assert dq(p.handle, A, None, None, 4, 128, 0, A, None) == F.FP4Q_ERR_ARG
+    assert dq(p.handle, A, A, None, 4, 128, 0, A + 4, None) == F.FP4Q_ERR_ALIGN
+    am = lambda *a: F.raw_call("fp4q_amax", *a)
+    assert am(p.handle, A, 4, 128, A, None) == F.FP4Q_ERR_UNSUPPORTED            # MX plan
+    F.fp4q_plan_destroy(p)
+
+
+def test_product_path_does_not_reference_the_oracle():
+    pkg = os.path.join(ROOT, "microscaling_fp4_quantization_b200")
+    for path in glob.glob(os.path.join(pkg, "**", "*"), recursive=True):
+        if os.path.isfile(path) and path.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+            text = open(path, encoding="utf-8").read()
+            assert "import oracle" not in text and "from oracle" not in text, path
