@@ -101,6 +101,47 @@ __device__ __forceinline__ void stg64(void* p, uint32_t a, uint32_t b) {
   asm volatile("st.global.v2.b32 [%0], {%1,%2};" ::"l"(p), "r"(a), "r"(b) : "memory");
 }
 
+// ---- packed fp32 pairs (f32x2 arithmetic on sm_100); the low half is the even element
+using f32x2 = unsigned long long;
+
+__device__ __forceinline__ f32x2 f2_pack(float lo, float hi) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(f32x2 p, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(p));
+}
+__device__ __forceinline__ f32x2 f2_add(f32x2 a, f32x2 b) {
+  f32x2 r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f32x2 f2_sub(f32x2 a, f32x2 b) {
+  f32x2 r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f32x2 f2_mul(f32x2 a, f32x2 b) {
+  f32x2 r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// First butterfly stage straight from a bf16 pair word (element 2k in the low half):
+// (x[2k] + x[2k+1], x[2k] - x[2k+1]), each rounded once to fp32, as a packed pair.
+__device__ __forceinline__ f32x2 bf16_pair_butterfly(uint32_t w) {
+  float s, d;
+  asm("{\n .reg .b16 lo16, hi16;\n .reg .b32 hi32;\n"
+      " mov.b32 {lo16, hi16}, %2;\n"
+      " and.b32 hi32, %2, 0xFFFF0000;\n"
+      " add.rn.f32.bf16 %0, lo16, hi32;\n"
+      " sub.rn.f32.bf16 %1, lo16, hi32;\n}"
+      : "=f"(s), "=f"(d)
+      : "r"(w));
+  return f2_pack(s, d);
+}
+
 // bf16 pair (element 2k in the low half) -> two exact fp32 values.
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }

@@ -55,46 +55,6 @@ __host__ __device__ constexpr float inv_sqrt_block(int b) {
                     : 0.0f;
 }
 
-// Compile-time shape of one kernel instance.
-template <int FMT, int B, int RULE, bool DUMP>
-struct RQConfig {
-  static constexpr int kFmt = FMT;
-  static constexpr int kBlock = B;
-  static constexpr int kRule = RULE;
-  static constexpr bool kDump = DUMP;
-  static constexpr int kGroup = FMT == kMX ? 32 : 16;
-  static constexpr int kE = cmax(B, kGroup);              // elements per unit
-  static constexpr int kChunks = kE / 8;                  // 16-byte chunks per unit
-  static constexpr int kGroupsPerUnit = kE / kGroup;
-  // Units per lane per stage: a stage of about 4 KB (8 KB for E = 128).
-  static constexpr int kR = cmax(1, 64 / kE);
-  static constexpr int kUnitsPerStage = 32 * kR;
-  static constexpr int kStageBytes = kUnitsPerStage * kE * 2;
-  static constexpr int kStages = kE >= 128 ? 3 : 4;
-  static constexpr int kWarps = 4;                       // warps per CTA
-  static constexpr int kThreads = kWarps * 32;
-  // Chunk-index XOR (see the file comment): as many low chunk bits as make a quarter-warp
-  // conflict-free, but never more than the chunk bits inside one Hadamard block.
-  static constexpr int kTauMaxChunks = cmin(kChunks, 8);
-  static constexpr int kTauShift = 3 - ilog2(kTauMaxChunks);
-  static constexpr int kTauMask = B >= 16 ? cmin(kTauMaxChunks, B / 8) - 1 : 0;
-  static constexpr int kBarBytes = 8 * kStages;
-  static constexpr int kWarpSmem = kStages * kStageBytes + 128;  // stages + barriers (padded)
-  static constexpr int kSmemBytes = kWarps * kWarpSmem;
-  static constexpr float kC = inv_sqrt_block(B);
-};
-
-struct RQArgs {
-  const uint16_t* x;       // bf16 [n_units * E]
-  int64_t n_units;
-  uint8_t* codes;          // [n_units * E / 2]
-  uint8_t* scales;         // [n_units * E / g]
-  float* tensor_scale;     // NV: static -> read; dynamic -> written by CTA 0
-  const float* partials;   // NV dynamic: per-CTA rotated amaxima from the amax pass
-  int n_partials;
-  float* y_dump;           // [n_units * E] when dumping
-};
-
 // Butterflies of H_B on every B-block of v[0..E) (unnormalised, in place).
 template <int B, int E>
 __device__ __forceinline__ void fwht_inplace(float (&v)[E]) {
@@ -111,24 +71,115 @@ __device__ __forceinline__ void fwht_inplace(float (&v)[E]) {
   }
 }
 
-// Load one unit from shared memory with the chunk XOR, widening bf16 -> fp32.
-template <int E>
-__device__ __forceinline__ void load_unit(uint32_t saddr, int tau, float (&v)[E]) {
+// Compile-time shape of one kernel instance.
+template <int FMT, int B, int RULE, bool DUMP>
+struct RQConfig {
+  static constexpr int kFmt = FMT;
+  static constexpr int kBlock = B;
+  static constexpr int kRule = RULE;
+  static constexpr bool kDump = DUMP;
+  static constexpr int kGroup = FMT == kMX ? 32 : 16;
+  static constexpr int kE = cmax(B, kGroup);              // elements per unit
+  static constexpr int kPairs = kE / 2;                   // packed fp32 pairs per unit
+  static constexpr int kChunks = kE / 8;                  // 16-byte chunks per unit
+  static constexpr int kGroupsPerUnit = kE / kGroup;
+  // Units per lane per stage: a stage of 2 KB (E <= 32), 4 KB (E = 64) or 8 KB (E = 128).
+  static constexpr int kR = cmax(1, 32 / kE);
+  static constexpr int kUnitsPerStage = 32 * kR;
+  static constexpr int kStageBytes = kUnitsPerStage * kE * 2;
+  static constexpr int kStages = kE >= 64 ? 3 : 4;
+  static constexpr int kWarps = kE >= 128 ? 2 : 4;        // warps per CTA
+  static constexpr int kThreads = kWarps * 32;
+  // Chunk-index XOR (see the file comment): as many low chunk bits as make a quarter-warp
+  // conflict-free, but never more than the chunk bits inside one Hadamard block.
+  static constexpr int kTauMaxChunks = cmin(kChunks, 8);
+  static constexpr int kTauShift = 3 - ilog2(kTauMaxChunks);
+  static constexpr int kTauMask = B >= 16 ? cmin(kTauMaxChunks, B / 8) - 1 : 0;
+  static constexpr int kWarpSmem = kStages * kStageBytes + 128;  // stages + barriers (padded)
+  static constexpr int kSmemBytes = kWarps * kWarpSmem;
+  static constexpr float kC = inv_sqrt_block(B);
+};
+
+struct RQArgs {
+  const uint16_t* x;       // bf16 [n_units * E]
+  int64_t n_units;
+  uint8_t* codes;          // [n_units * E / 2]
+  uint8_t* scales;         // [n_units * E / g]
+  float* tensor_scale;     // NV: static -> read; dynamic -> written by CTA 0
+  const float* partials;   // NV dynamic: per-CTA rotated amaxima from the amax pass
+  int n_partials;
+  float* y_dump;           // [n_units * E] when dumping
+};
+
+// Per-lane constants of the chunk XOR: tau, and bit j of `flips` set when output chunk j
+// comes out of the butterfly with its sign flipped (popcount(tau & j) odd).
+struct LaneXor {
+  int tau;
+  uint32_t flips;
+};
+
+template <class Cfg>
+__device__ __forceinline__ LaneXor lane_xor(int lane) {
+  LaneXor lx;
+  lx.tau = (lane >> Cfg::kTauShift) & Cfg::kTauMask;
+  lx.flips = 0;
+#pragma unroll
+  for (int j = 0; j < Cfg::kChunks; ++j) lx.flips |= static_cast<uint32_t>(__popc(lx.tau & j) & 1) << j;
+  return lx;
+}
+
+// Load one unit from shared memory (chunk j read from position j ^ tau), widen bf16 to
+// fp32 and run the butterfly of H_B on every B-block (unnormalised sums).  p[k] holds the
+// pair (element 2k, element 2k + 1).  The first stage (distance 1) is taken straight from
+// the bf16 pair; the others run on packed pairs, pair k against pair k + h/2.  Every element
+// sees the same additions, in the same order, as in the scalar butterfly.
+template <int B, int E>
+__device__ __forceinline__ void load_rotate_unit(uint32_t saddr, int tau, f32x2 (&p)[E / 2]) {
 #pragma unroll
   for (int j = 0; j < E / 8; ++j) {
     const uint4 w = lds128(saddr + 16u * static_cast<uint32_t>(j ^ tau));
-    v[8 * j + 0] = bf16_lo(w.x);
-    v[8 * j + 1] = bf16_hi(w.x);
-    v[8 * j + 2] = bf16_lo(w.y);
-    v[8 * j + 3] = bf16_hi(w.y);
-    v[8 * j + 4] = bf16_lo(w.z);
-    v[8 * j + 5] = bf16_hi(w.z);
-    v[8 * j + 6] = bf16_lo(w.w);
-    v[8 * j + 7] = bf16_hi(w.w);
+    if constexpr (B >= 2) {
+      p[4 * j + 0] = bf16_pair_butterfly(w.x);
+      p[4 * j + 1] = bf16_pair_butterfly(w.y);
+      p[4 * j + 2] = bf16_pair_butterfly(w.z);
+      p[4 * j + 3] = bf16_pair_butterfly(w.w);
+    } else {
+      p[4 * j + 0] = f2_pack(bf16_lo(w.x), bf16_hi(w.x));
+      p[4 * j + 1] = f2_pack(bf16_lo(w.y), bf16_hi(w.y));
+      p[4 * j + 2] = f2_pack(bf16_lo(w.z), bf16_hi(w.z));
+      p[4 * j + 3] = f2_pack(bf16_lo(w.w), bf16_hi(w.w));
+    }
+  }
+#pragma unroll
+  for (int h = 2; h < B; h <<= 1) {
+    const int hp = h / 2;
+#pragma unroll
+    for (int k = 0; k < E / 2; ++k) {
+      if ((k & hp) == 0) {
+        const f32x2 a = p[k], b = p[k + hp];
+        p[k] = f2_add(a, b);
+        p[k + hp] = f2_sub(a, b);
+      }
+    }
   }
 }
 
-__device__ __forceinline__ uint32_t parity32(uint32_t v) { return __popc(v) & 1u; }
+// max |value| over N pairs, as a tree for instruction-level parallelism.
+template <int N>
+__device__ __forceinline__ float pairs_amax(const f32x2* p) {
+  float t[N];
+#pragma unroll
+  for (int k = 0; k < N; ++k) {
+    float lo, hi;
+    f2_unpack(p[k], lo, hi);
+    t[k] = fmaxf(fabsf(lo), fabsf(hi));
+  }
+#pragma unroll
+  for (int s = N / 2; s >= 1; s /= 2)
+#pragma unroll
+    for (int k = 0; k < s; ++k) t[k] = fmaxf(t[k], t[k + s]);
+  return t[0];
+}
 
 // MX scale byte from the fp32 group amax A >= 0 (see fp4q.h for the rules).
 template <int RULE>
@@ -139,8 +190,8 @@ __device__ __forceinline__ int mx_scale_byte(float A) {
   int bump = 0;
   if (RULE == kRuleCeil) bump = man > 0x400000u;       // mantissa above 1.5
   if (RULE == kRuleOas) bump = man > 0x600000u;        // mantissa above 1.75
-  int byte = eb - 2 + bump;                            // e + 127 with e = floor(log2 A) - 2 + bump
-  return byte < 0 ? 0 : (byte > 254 ? 254 : byte);
+  const int byte = eb - 2 + bump;                      // e + 127 with e = floor(log2 A) - 2 + bump
+  return byte < 0 ? 0 : byte;                          // finite A keeps byte <= 253
 }
 
 // 2^(127 - byte) as fp32 (byte in [0, 253]).
@@ -148,28 +199,36 @@ __device__ __forceinline__ float mx_inv_scale(int byte) {
   return __uint_as_float(static_cast<uint32_t>(254 - byte) << 23);
 }
 
-// Quantize one rotated unit v (unnormalised butterfly sums) and store its codes / scales.
+// Correctly rounded a / d from rd = RN(1/d): one Markstein correction step of the product
+// a * rd (P. Markstein, "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990).  Valid while the quotient and the residual
+// stay in the normal range; a quotient below that range rounds to a zero E4M3 scale anyway.
+__device__ __forceinline__ float div_rn_markstein(float a, float d, float rd) {
+  const float q0 = a * rd;
+  const float r = fmaf(-q0, d, a);
+  return fmaf(r, rd, q0);
+}
+
+// Quantize one rotated unit (pairs p, unnormalised butterfly sums) and store its codes and
+// scales.  `lx` undoes the chunk XOR's sign flips.
 template <class Cfg>
-__device__ __forceinline__ void quantize_store_unit(float (&v)[Cfg::kE], int64_t unit, int tau, float s_g,
-                                                    float nv_den, const RQArgs& a) {
+__device__ __forceinline__ void quantize_store_unit(const f32x2 (&p)[Cfg::kPairs], int64_t unit, const LaneXor& lx,
+                                                    float s_g, float nv_den, float nv_rden, const RQArgs& a) {
   constexpr int E = Cfg::kE, G = Cfg::kGroup, NG = Cfg::kGroupsPerUnit;
   constexpr float c = Cfg::kC;
   uint32_t words[E / 8];
   uint32_t sbytes[NG];
 #pragma unroll
   for (int q = 0; q < NG; ++q) {
-    float m = 0.0f;
-#pragma unroll
-    for (int i = 0; i < G; ++i) m = fmaxf(m, fabsf(v[q * G + i]));
-    const float A = m * c;                 // = max |fl(v * c)|: rounding is monotonic
+    const float A = pairs_amax<G / 2>(&p[q * G / 2]) * c;   // = max |fl(v c)|: rounding is monotonic
     float mult;
     uint32_t keep = 0xFFFFFFFFu;
-    if (Cfg::kFmt == kMX) {
+    if constexpr (Cfg::kFmt == kMX) {
       const int byte = mx_scale_byte<Cfg::kRule>(A);
       sbytes[q] = static_cast<uint32_t>(byte);
       mult = c * mx_inv_scale(byte);      // exact: a power-of-two multiple of c
     } else {
-      const float s_b = __fdiv_rn(A, nv_den);
+      const float s_b = div_rn_markstein(A, nv_den, nv_rden);
       const uint32_t byte = e4m3_encode(s_b);
       sbytes[q] = byte;
       const float S = e4m3_decode(byte) * s_g;
@@ -178,23 +237,25 @@ __device__ __forceinline__ void quantize_store_unit(float (&v)[Cfg::kE], int64_t
     }
 #pragma unroll
     for (int j = 0; j < G / 8; ++j) {
-      const int i = q * G + 8 * j;
-      uint32_t w = e2m1x8(v[i] * mult, v[i + 1] * mult, v[i + 2] * mult, v[i + 3] * mult, v[i + 4] * mult,
-                          v[i + 5] * mult, v[i + 6] * mult, v[i + 7] * mult);
-      const int chunk = i / 8;
-      if (parity32(static_cast<uint32_t>(tau & chunk))) w ^= 0x88888888u;
-      words[chunk] = w & keep;
+      const int chunk = q * (G / 8) + j;
+      float m = mult;
+      if constexpr (Cfg::kTauMask != 0)
+        m = __uint_as_float(__float_as_uint(mult) ^ ((lx.flips << (31 - chunk)) & 0x80000000u));
+      const f32x2 mm = f2_pack(m, m);
+      float v[8];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) f2_unpack(f2_mul(p[4 * chunk + t], mm), v[2 * t], v[2 * t + 1]);
+      words[chunk] = e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]) & keep;
     }
   }
   // codes: E/2 bytes per unit
   uint8_t* cp = a.codes + unit * (E / 2);
   if constexpr (E == 16) {
     stg64(cp, words[0], words[1]);
-  } else if constexpr (E == 32) {
-    stg128(cp, words[0], words[1], words[2], words[3]);
   } else {
 #pragma unroll
-    for (int k = 0; k < E / 32; ++k) stg128(cp + 16 * k, words[4 * k], words[4 * k + 1], words[4 * k + 2], words[4 * k + 3]);
+    for (int k = 0; k < E / 32; ++k)
+      stg128(cp + 16 * k, words[4 * k], words[4 * k + 1], words[4 * k + 2], words[4 * k + 3]);
   }
   // scales: E/g bytes per unit
   uint8_t* sp = a.scales + unit * NG;
@@ -213,21 +274,22 @@ __device__ __forceinline__ void quantize_store_unit(float (&v)[Cfg::kE], int64_t
     float* yp = a.y_dump + unit * E;
 #pragma unroll
     for (int j = 0; j < E / 8; ++j) {
-      const float sg = parity32(static_cast<uint32_t>(tau & j)) ? -c : c;
-      float4 lo = make_float4(v[8 * j] * sg, v[8 * j + 1] * sg, v[8 * j + 2] * sg, v[8 * j + 3] * sg);
-      float4 hi = make_float4(v[8 * j + 4] * sg, v[8 * j + 5] * sg, v[8 * j + 6] * sg, v[8 * j + 7] * sg);
-      reinterpret_cast<float4*>(yp)[2 * j] = lo;
-      reinterpret_cast<float4*>(yp)[2 * j + 1] = hi;
+      const float sg = ((lx.flips >> j) & 1u) ? -c : c;
+      float v[8];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) f2_unpack(p[4 * j + t], v[2 * t], v[2 * t + 1]);
+      reinterpret_cast<float4*>(yp)[2 * j] = make_float4(v[0] * sg, v[1] * sg, v[2] * sg, v[3] * sg);
+      reinterpret_cast<float4*>(yp)[2 * j + 1] = make_float4(v[4] * sg, v[5] * sg, v[6] * sg, v[7] * sg);
     }
   }
 }
 
-// Per-warp streaming skeleton shared by the quantize and the amax kernels.  `body(v, unit,
-// tau)` is called once per unit with the rotated (unnormalised) values.  Returns false when
-// a bounded wait ran out.
+// Per-warp streaming skeleton shared by the quantize and the amax kernels.  `body(p, unit)`
+// is called once per unit with the rotated (unnormalised) pairs.  Returns false when a
+// bounded wait ran out.
 template <class Cfg, class Body>
 __device__ __forceinline__ bool stream_units(const uint16_t* __restrict__ x, int64_t n_units, uint8_t* warp_smem,
-                                             Body&& body) {
+                                             int tau, Body&& body) {
   constexpr int S = Cfg::kStages, SU = Cfg::kUnitsPerStage, E = Cfg::kE;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -238,7 +300,6 @@ __device__ __forceinline__ bool stream_units(const uint16_t* __restrict__ x, int
   const int64_t n_stages = (u1 - u0 + SU - 1) / SU;
   const uint32_t bar0 = smem_addr(warp_smem);
   const uint32_t buf0 = smem_addr(warp_smem + 128);
-  const int tau = (lane >> Cfg::kTauShift) & Cfg::kTauMask;
 
   auto issue = [&](int64_t t) {
     const int st = static_cast<int>(t % S);
@@ -275,14 +336,24 @@ __device__ __forceinline__ bool stream_units(const uint16_t* __restrict__ x, int
     const int64_t us = u0 + t * SU;
     const int64_t cnt = (u1 - us) < SU ? (u1 - us) : SU;
     const uint32_t sbase = buf0 + static_cast<uint32_t>(st) * Cfg::kStageBytes;
+    if (cnt == SU) {
+      // full stage: no per-unit bounds test, so the R units interleave freely
 #pragma unroll
-    for (int r = 0; r < Cfg::kR; ++r) {
-      const int lu = r * 32 + lane;
-      if (lu < cnt) {
-        float v[E];
-        load_unit<E>(sbase + static_cast<uint32_t>(lu) * (E * 2), tau, v);
-        fwht_inplace<Cfg::kBlock, E>(v);
-        body(v, us + lu, tau);
+      for (int r = 0; r < Cfg::kR; ++r) {
+        const int lu = r * 32 + lane;
+        f32x2 p[Cfg::kPairs];
+        load_rotate_unit<Cfg::kBlock, E>(sbase + static_cast<uint32_t>(lu) * (E * 2), tau, p);
+        body(p, us + lu);
+      }
+    } else {
+#pragma unroll
+      for (int r = 0; r < Cfg::kR; ++r) {
+        const int lu = r * 32 + lane;
+        if (lu < cnt) {
+          f32x2 p[Cfg::kPairs];
+          load_rotate_unit<Cfg::kBlock, E>(sbase + static_cast<uint32_t>(lu) * (E * 2), tau, p);
+          body(p, us + lu);
+        }
       }
     }
     __syncwarp();
@@ -299,6 +370,7 @@ __global__ void __launch_bounds__(Cfg::kThreads) rotate_quantize_kernel(RQArgs a
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float s_tensor_scale;
   const int warp = threadIdx.x >> 5;
+  const LaneXor lx = lane_xor<Cfg>(threadIdx.x & 31);
   float s_g = 1.0f;
   if constexpr (Cfg::kFmt == kNV) {
     if constexpr (Cfg::kRule == kRuleNvDynamic) {
@@ -320,9 +392,10 @@ __global__ void __launch_bounds__(Cfg::kThreads) rotate_quantize_kernel(RQArgs a
     s_g = s_tensor_scale;
   }
   const float nv_den = 6.0f * s_g;
-  stream_units<Cfg>(a.x, a.n_units, smem + warp * Cfg::kWarpSmem,
-                    [&](float (&v)[Cfg::kE], int64_t unit, int tau) {
-                      quantize_store_unit<Cfg>(v, unit, tau, s_g, nv_den, a);
+  const float nv_rden = __frcp_rn(nv_den);
+  stream_units<Cfg>(a.x, a.n_units, smem + warp * Cfg::kWarpSmem, lx.tau,
+                    [&](const f32x2 (&p)[Cfg::kPairs], int64_t unit) {
+                      quantize_store_unit<Cfg>(p, unit, lx, s_g, nv_den, nv_rden, a);
                     });
 }
 
@@ -333,11 +406,10 @@ __global__ void __launch_bounds__(Cfg::kThreads) rotated_amax_kernel(const uint1
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float s_max[Cfg::kWarps];
   const int warp = threadIdx.x >> 5;
+  const LaneXor lx = lane_xor<Cfg>(threadIdx.x & 31);
   float m = 0.0f;
-  stream_units<Cfg>(x, n_units, smem + warp * Cfg::kWarpSmem, [&](float (&v)[Cfg::kE], int64_t, int) {
-#pragma unroll
-    for (int i = 0; i < Cfg::kE; ++i) m = fmaxf(m, fabsf(v[i]));
-  });
+  stream_units<Cfg>(x, n_units, smem + warp * Cfg::kWarpSmem, lx.tau,
+                    [&](const f32x2 (&p)[Cfg::kPairs], int64_t) { m = fmaxf(m, pairs_amax<Cfg::kPairs>(p)); });
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
   if ((threadIdx.x & 31) == 0) s_max[warp] = m;

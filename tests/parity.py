@@ -5,7 +5,8 @@
     whose exact amax (or NV block-scale quotient) lies within 1e-5 of the scale rule's
     boundary;
   * at most 1e-4 of the elements may differ (a group whose scale differs counts whole);
-  * a rotated value that is exactly zero may carry either sign bit (both codes encode 0);
+  * two codes of magnitude zero are equal whatever their sign bits (+0 and -0 encode the
+    same value; the sign of a cancelled fp32 butterfly sum is not the sign of the exact sum);
   * rotated values: |y_gpu - y_exact| <= 1e-5 * ||x_block||_2 for every element.
 """
 
@@ -32,9 +33,11 @@ class ParityReport:
     flagged_groups: int
     mismatch_elements: int
 
-    def ok(self) -> bool:
-        return (self.unflagged_code_mismatch == 0 and self.unflagged_scale_mismatch == 0
-                and self.mismatch_elements <= MAX_MISMATCH_FRACTION * max(self.n, 1))
+    def ok(self, count_bound: bool = True) -> bool:
+        subset = self.unflagged_code_mismatch == 0 and self.unflagged_scale_mismatch == 0
+        if not count_bound:
+            return subset
+        return subset and self.mismatch_elements <= MAX_MISMATCH_FRACTION * max(self.n, 1)
 
 
 def compare(res: dict, codes_gpu: np.ndarray, scales_gpu: np.ndarray, tol: float = REL_TOL) -> ParityReport:
@@ -46,8 +49,8 @@ def compare(res: dict, codes_gpu: np.ndarray, scales_gpu: np.ndarray, tol: float
     qo = o.unpack_nibbles(res["codes"])
     qg = o.unpack_nibbles(codes_gpu)
     M, K = qo.shape
-    zero = res["y64"] == 0.0
-    diff = np.where(zero, (qo & 7) != (qg & 7), qo != qg)
+    both_zero = ((qo & 7) == 0) & ((qg & 7) == 0)
+    diff = (qo != qg) & ~both_zero
     sdiff = res["scales"] != scales_gpu
     el, gr = o.flags(res, tol)
     gr_el = np.repeat(gr, g, axis=1)
@@ -67,9 +70,11 @@ def compare(res: dict, codes_gpu: np.ndarray, scales_gpu: np.ndarray, tol: float
     )
 
 
-def assert_parity(res: dict, codes_gpu, scales_gpu, label: str = "") -> ParityReport:
+def assert_parity(res: dict, codes_gpu, scales_gpu, label: str = "", count_bound: bool = True) -> ParityReport:
+    """count_bound=False keeps only "every mismatch is flagged": for inputs built to sit on
+    ties (exact midpoints, powers of two), where near-ties are dense by construction."""
     rep = compare(res, codes_gpu, scales_gpu)
-    assert rep.ok(), f"{label}: {rep}"
+    assert rep.ok(count_bound), f"{label}: {rep}"
     return rep
 
 

@@ -57,6 +57,7 @@ def test_rotate_quantize_matches_oracle(F, combo):
     unit = max(g, b)
     for i, (M, K) in enumerate(shapes_for(unit)):
         x = make_input(M, K, seed=100 * b + 10 * rule + i)
+        adversarial = M >= 8
         if fmt == o.NVFP4 and rule == o.SCALE_NV_STATIC:
             s_g = o.nv_tensor_scale(o.rotated_amax(x, b))
             res = o.rotate_quantize(x, fmt, g, b, rule, tensor_scale=s_g)
@@ -67,7 +68,14 @@ def test_rotate_quantize_matches_oracle(F, combo):
         if fmt == o.NVFP4 and rule == o.SCALE_NV_DYNAMIC:
             rel = abs(float(out["tensor_scale"]) - float(res["tensor_scale"])) / float(res["tensor_scale"])
             assert rel <= 2.5e-7, (M, K, out["tensor_scale"], res["tensor_scale"])
-        assert_parity(res, out["codes"], out["scales"], f"{combo_id(combo)} {M}x{K}")
+        # rows built on ties (midpoints, powers of two) make near-ties dense: there only the
+        # "every mismatch is flagged" part of the rule applies; realistic rows get the count bound too
+        assert_parity(res, out["codes"], out["scales"], f"{combo_id(combo)} {M}x{K}", count_bound=not adversarial)
+        if adversarial:
+            real = slice(8, M)
+            res_r = {k: (v[real] if isinstance(v, np.ndarray) and v.ndim == 2 and v.shape[0] == M else v)
+                     for k, v in res.items()}
+            assert_parity(res_r, out["codes"][real], out["scales"][real], f"{combo_id(combo)} {M}x{K} rows 8+")
         assert rotated_value_error(out["y"], res) <= 1e-5, (M, K)
         # the non-dumping kernel gives the same bytes as the dumping one
         plain = gu.run_rotate_quantize(F, plan, x, tensor_scale=out["tensor_scale"] if fmt == o.NVFP4 and
