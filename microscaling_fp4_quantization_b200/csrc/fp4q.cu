@@ -89,7 +89,8 @@ fp4q_status with_block(int b, F&& f) {
 }
 
 template <class Cfg>
-fp4q_status launch_rq(const RQArgs& a, cudaStream_t stream) {
+fp4q_status launch_rq(RQArgs a, int64_t n_elems, cudaStream_t stream) {
+  a.n_units = n_elems / Cfg::kE;
   auto kernel = rotate_quantize_kernel<Cfg>;
   KernelInfo ki;
   fp4q_status st = kernel_info(kernel, Cfg::kSmemBytes, Cfg::kThreads, &ki);
@@ -104,27 +105,38 @@ fp4q_status launch_rq(const RQArgs& a, cudaStream_t stream) {
   return FP4Q_OK;
 }
 
-template <int B>
-using AmaxCfg = RQConfig<kNV, B, kRuleNvStatic, false>;
+template <int B, int MINU>
+using AmaxCfg = RQConfig<kNV, B, kRuleNvStatic, false, MINU>;
 
-// Number of CTAs the amax pass always launches (and of partial maxima a plan holds).
+// Number of CTAs the amax pass always launches (and of partial maxima a plan holds): one
+// full wave of the larger of its two instances.
 fp4q_status amax_grid(int b, int* n) {
   return with_block(b, [&]<int B>() -> fp4q_status {
-    KernelInfo ki;
-    fp4q_status st = kernel_info(rotated_amax_kernel<AmaxCfg<B>>, AmaxCfg<B>::kSmemBytes, AmaxCfg<B>::kThreads, &ki);
+    KernelInfo k16, k32;
+    fp4q_status st = kernel_info(rotated_amax_kernel<AmaxCfg<B, 16>>, AmaxCfg<B, 16>::kSmemBytes,
+                                 AmaxCfg<B, 16>::kThreads, &k16);
     if (st != FP4Q_OK) return st;
-    *n = ki.sm_count * ki.ctas_per_sm;
+    st = kernel_info(rotated_amax_kernel<AmaxCfg<B, 32>>, AmaxCfg<B, 32>::kSmemBytes, AmaxCfg<B, 32>::kThreads, &k32);
+    if (st != FP4Q_OK) return st;
+    const int a = k16.sm_count * k16.ctas_per_sm, c = k32.sm_count * k32.ctas_per_sm;
+    *n = a > c ? a : c;
     return FP4Q_OK;
   });
 }
 
-fp4q_status launch_amax(fp4q_plan p, const uint16_t* x, int64_t n_units, cudaStream_t stream) {
+template <class Cfg>
+fp4q_status launch_amax_cfg(fp4q_plan p, const uint16_t* x, int64_t n_elems, cudaStream_t stream) {
+  rotated_amax_kernel<Cfg><<<p->n_partials, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(x, n_elems / Cfg::kE,
+                                                                                        p->partials);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "amax launch");
+  return FP4Q_OK;
+}
+
+fp4q_status launch_amax(fp4q_plan p, const uint16_t* x, int64_t n_elems, cudaStream_t stream) {
   return with_block(p->block, [&]<int B>() -> fp4q_status {
-    using Cfg = AmaxCfg<B>;
-    rotated_amax_kernel<Cfg><<<p->n_partials, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(x, n_units, p->partials);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "amax launch");
-    return FP4Q_OK;
+    if (n_elems % AmaxCfg<B, 32>::kE == 0) return launch_amax_cfg<AmaxCfg<B, 32>>(p, x, n_elems, stream);
+    return launch_amax_cfg<AmaxCfg<B, 16>>(p, x, n_elems, stream);
   });
 }
 
@@ -148,8 +160,9 @@ fp4q_status rotate_quantize_impl(fp4q_plan p, const void* x, int64_t M, int64_t 
     return FP4Q_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   RQArgs a;
+  const int64_t n = M * K;
   a.x = static_cast<const uint16_t*>(x);
-  a.n_units = (M * K) / p->unit;
+  a.n_units = 0;  // set per instance from its unit size
   a.codes = static_cast<uint8_t*>(codes);
   a.scales = static_cast<uint8_t*>(scales);
   a.tensor_scale = tensor_scale;
@@ -157,29 +170,38 @@ fp4q_status rotate_quantize_impl(fp4q_plan p, const void* x, int64_t M, int64_t 
   a.n_partials = p->n_partials;
   a.y_dump = y_out;
   if (p->format == FP4Q_NVFP4 && p->rule == FP4Q_SCALE_NV_DYNAMIC) {
-    st = launch_amax(p, a.x, a.n_units, s);
+    st = launch_amax(p, a.x, n, s);
     if (st != FP4Q_OK) return st;
   }
   return with_block(p->block, [&]<int B>() -> fp4q_status {
     if (p->format == FP4Q_MXFP4) {
       switch (p->rule) {
         case FP4Q_SCALE_FLOOR_OCP:
-          return dump ? launch_rq<RQConfig<kMX, B, kRuleFloor, true>>(a, s)
-                      : launch_rq<RQConfig<kMX, B, kRuleFloor, false>>(a, s);
+          return dump ? launch_rq<RQConfig<kMX, B, kRuleFloor, true>>(a, n, s)
+                      : launch_rq<RQConfig<kMX, B, kRuleFloor, false>>(a, n, s);
         case FP4Q_SCALE_CEIL_NOCLIP:
-          return dump ? launch_rq<RQConfig<kMX, B, kRuleCeil, true>>(a, s)
-                      : launch_rq<RQConfig<kMX, B, kRuleCeil, false>>(a, s);
+          return dump ? launch_rq<RQConfig<kMX, B, kRuleCeil, true>>(a, n, s)
+                      : launch_rq<RQConfig<kMX, B, kRuleCeil, false>>(a, n, s);
         case FP4Q_SCALE_OAS:
-          return dump ? launch_rq<RQConfig<kMX, B, kRuleOas, true>>(a, s)
-                      : launch_rq<RQConfig<kMX, B, kRuleOas, false>>(a, s);
+          return dump ? launch_rq<RQConfig<kMX, B, kRuleOas, true>>(a, n, s)
+                      : launch_rq<RQConfig<kMX, B, kRuleOas, false>>(a, n, s);
         default: return FP4Q_ERR_UNSUPPORTED;
       }
     }
-    if (p->rule == FP4Q_SCALE_NV_DYNAMIC)
-      return dump ? launch_rq<RQConfig<kNV, B, kRuleNvDynamic, true>>(a, s)
-                  : launch_rq<RQConfig<kNV, B, kRuleNvDynamic, false>>(a, s);
-    return dump ? launch_rq<RQConfig<kNV, B, kRuleNvStatic, true>>(a, s)
-                : launch_rq<RQConfig<kNV, B, kRuleNvStatic, false>>(a, s);
+    // NVFP4: 32-element units when the element count allows, else 16
+    const bool u32 = n % 32 == 0;
+    if (p->rule == FP4Q_SCALE_NV_DYNAMIC) {
+      if (u32)
+        return dump ? launch_rq<RQConfig<kNV, B, kRuleNvDynamic, true, 32>>(a, n, s)
+                    : launch_rq<RQConfig<kNV, B, kRuleNvDynamic, false, 32>>(a, n, s);
+      return dump ? launch_rq<RQConfig<kNV, B, kRuleNvDynamic, true, 16>>(a, n, s)
+                  : launch_rq<RQConfig<kNV, B, kRuleNvDynamic, false, 16>>(a, n, s);
+    }
+    if (u32)
+      return dump ? launch_rq<RQConfig<kNV, B, kRuleNvStatic, true, 32>>(a, n, s)
+                  : launch_rq<RQConfig<kNV, B, kRuleNvStatic, false, 32>>(a, n, s);
+    return dump ? launch_rq<RQConfig<kNV, B, kRuleNvStatic, true, 16>>(a, n, s)
+                : launch_rq<RQConfig<kNV, B, kRuleNvStatic, false, 16>>(a, n, s);
   });
 }
 
@@ -263,7 +285,7 @@ fp4q_status fp4q_amax(fp4q_plan plan, const void* x_bf16, int64_t M, int64_t K, 
   if (M * K > 0 && !x_bf16) return FP4Q_ERR_ARG;
   if ((x_bf16 && !aligned(x_bf16, 16)) || !aligned(tensor_scale_out, 4)) return FP4Q_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = launch_amax(plan, static_cast<const uint16_t*>(x_bf16), (M * K) / plan->unit, s);
+  st = launch_amax(plan, static_cast<const uint16_t*>(x_bf16), M * K, s);
   if (st != FP4Q_OK) return st;
   tensor_scale_finalize_kernel<<<1, 32, 0, s>>>(plan->partials, plan->n_partials, tensor_scale_out);
   cudaError_t e = cudaGetLastError();

@@ -129,17 +129,28 @@ __device__ __forceinline__ f32x2 f2_mul(f32x2 a, f32x2 b) {
 }
 
 // First butterfly stage straight from a bf16 pair word (element 2k in the low half):
-// (x[2k] + x[2k+1], x[2k] - x[2k+1]), each rounded once to fp32, as a packed pair.
-__device__ __forceinline__ f32x2 bf16_pair_butterfly(uint32_t w) {
+// (x[2k] + x[2k+1], x[2k+1] - x[2k]), each rounded once to fp32, as a packed pair.  The
+// second entry is the negated difference: the mixed-precision add takes the high bf16 half
+// as its bf16 operand and the low half, widened by an integer multiply, as its fp32 operand.
+// Callers undo the negation of the odd elements (it commutes with every later stage, which
+// treats the two halves of a pair alike).
+__device__ __forceinline__ f32x2 bf16_pair_butterfly_oddneg(uint32_t w) {
   float s, d;
-  asm("{\n .reg .b16 lo16, hi16;\n .reg .b32 hi32;\n"
+  const float lo = __uint_as_float(w * 65536u);
+  asm("{\n .reg .b16 lo16, hi16;\n"
       " mov.b32 {lo16, hi16}, %2;\n"
-      " and.b32 hi32, %2, 0xFFFF0000;\n"
-      " add.rn.f32.bf16 %0, lo16, hi32;\n"
-      " sub.rn.f32.bf16 %1, lo16, hi32;\n}"
+      " add.rn.f32.bf16 %0, hi16, %3;\n"
+      " sub.rn.f32.bf16 %1, hi16, %3;\n}"
       : "=f"(s), "=f"(d)
-      : "r"(w));
+      : "r"(w), "f"(lo));
   return f2_pack(s, d);
+}
+
+// Approximate reciprocal (the hardware's rcp.approx: relative error below 2^-22).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
 }
 
 // bf16 pair (element 2k in the low half) -> two exact fp32 values.

@@ -71,15 +71,16 @@ __device__ __forceinline__ void fwht_inplace(float (&v)[E]) {
   }
 }
 
-// Compile-time shape of one kernel instance.
-template <int FMT, int B, int RULE, bool DUMP>
+// Compile-time shape of one kernel instance.  MINU is the smallest unit: 32 when the
+// tensor's element count allows it (fewer per-unit costs, 16-byte code stores), else 16.
+template <int FMT, int B, int RULE, bool DUMP, int MINU = 32>
 struct RQConfig {
   static constexpr int kFmt = FMT;
   static constexpr int kBlock = B;
   static constexpr int kRule = RULE;
   static constexpr bool kDump = DUMP;
   static constexpr int kGroup = FMT == kMX ? 32 : 16;
-  static constexpr int kE = cmax(B, kGroup);              // elements per unit
+  static constexpr int kE = cmax(cmax(B, kGroup), MINU);  // elements per unit
   static constexpr int kPairs = kE / 2;                   // packed fp32 pairs per unit
   static constexpr int kChunks = kE / 8;                  // 16-byte chunks per unit
   static constexpr int kGroupsPerUnit = kE / kGroup;
@@ -111,38 +112,51 @@ struct RQArgs {
   float* y_dump;           // [n_units * E] when dumping
 };
 
-// Per-lane constants of the chunk XOR: tau, and bit j of `flips` set when output chunk j
-// comes out of the butterfly with its sign flipped (popcount(tau & j) odd).
+// Per-lane constants of the chunk XOR: tau, and for each of tau's (at most three) bits the
+// code-word mask that flips the sign bits of a chunk (0x88888888) when that bit is set.
+// Output chunk j comes out of the butterfly with its sign flipped when popcount(tau & j) is
+// odd, i.e. its mask is the XOR of basis[b] over the bits b of j.
 struct LaneXor {
   int tau;
-  uint32_t flips;
+  uint32_t basis[3];
 };
 
 template <class Cfg>
 __device__ __forceinline__ LaneXor lane_xor(int lane) {
   LaneXor lx;
   lx.tau = (lane >> Cfg::kTauShift) & Cfg::kTauMask;
-  lx.flips = 0;
 #pragma unroll
-  for (int j = 0; j < Cfg::kChunks; ++j) lx.flips |= static_cast<uint32_t>(__popc(lx.tau & j) & 1) << j;
+  for (int b = 0; b < 3; ++b) lx.basis[b] = ((lx.tau >> b) & 1) ? 0x88888888u : 0u;
   return lx;
+}
+
+// Sign mask for the packed codes of output chunk j: the chunk XOR's flip, and (B >= 2) the
+// negated odd elements of the first butterfly stage (high nibbles, 0x80808080).
+template <int B>
+__device__ __forceinline__ uint32_t chunk_sign_mask(const LaneXor& lx, int j) {
+  uint32_t m = B >= 2 ? 0x80808080u : 0u;
+  if (j & 1) m ^= lx.basis[0];
+  if (j & 2) m ^= lx.basis[1];
+  if (j & 4) m ^= lx.basis[2];
+  return m;
 }
 
 // Load one unit from shared memory (chunk j read from position j ^ tau), widen bf16 to
 // fp32 and run the butterfly of H_B on every B-block (unnormalised sums).  p[k] holds the
 // pair (element 2k, element 2k + 1).  The first stage (distance 1) is taken straight from
 // the bf16 pair; the others run on packed pairs, pair k against pair k + h/2.  Every element
-// sees the same additions, in the same order, as in the scalar butterfly.
+// sees the same additions, in the same order, as in the scalar butterfly; for B >= 2 the odd
+// elements come out negated (see bf16_pair_butterfly_oddneg).
 template <int B, int E>
 __device__ __forceinline__ void load_rotate_unit(uint32_t saddr, int tau, f32x2 (&p)[E / 2]) {
 #pragma unroll
   for (int j = 0; j < E / 8; ++j) {
     const uint4 w = lds128(saddr + 16u * static_cast<uint32_t>(j ^ tau));
     if constexpr (B >= 2) {
-      p[4 * j + 0] = bf16_pair_butterfly(w.x);
-      p[4 * j + 1] = bf16_pair_butterfly(w.y);
-      p[4 * j + 2] = bf16_pair_butterfly(w.z);
-      p[4 * j + 3] = bf16_pair_butterfly(w.w);
+      p[4 * j + 0] = bf16_pair_butterfly_oddneg(w.x);
+      p[4 * j + 1] = bf16_pair_butterfly_oddneg(w.y);
+      p[4 * j + 2] = bf16_pair_butterfly_oddneg(w.z);
+      p[4 * j + 3] = bf16_pair_butterfly_oddneg(w.w);
     } else {
       p[4 * j + 0] = f2_pack(bf16_lo(w.x), bf16_hi(w.x));
       p[4 * j + 1] = f2_pack(bf16_lo(w.y), bf16_hi(w.y));
@@ -233,19 +247,16 @@ __device__ __forceinline__ void quantize_store_unit(const f32x2 (&p)[Cfg::kPairs
       sbytes[q] = byte;
       const float S = e4m3_decode(byte) * s_g;
       if (S == 0.0f) keep = 0u;           // a zero block scale gives zero codes
-      mult = S == 0.0f ? 0.0f : c * __frcp_rn(S);
+      mult = S == 0.0f ? 0.0f : c * rcp_approx(S);
     }
+    const f32x2 mm = f2_pack(mult, mult);
 #pragma unroll
     for (int j = 0; j < G / 8; ++j) {
       const int chunk = q * (G / 8) + j;
-      float m = mult;
-      if constexpr (Cfg::kTauMask != 0)
-        m = __uint_as_float(__float_as_uint(mult) ^ ((lx.flips << (31 - chunk)) & 0x80000000u));
-      const f32x2 mm = f2_pack(m, m);
       float v[8];
 #pragma unroll
       for (int t = 0; t < 4; ++t) f2_unpack(f2_mul(p[4 * chunk + t], mm), v[2 * t], v[2 * t + 1]);
-      words[chunk] = e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]) & keep;
+      words[chunk] = (e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]) ^ chunk_sign_mask<Cfg::kBlock>(lx, chunk)) & keep;
     }
   }
   // codes: E/2 bytes per unit
@@ -274,12 +285,14 @@ __device__ __forceinline__ void quantize_store_unit(const f32x2 (&p)[Cfg::kPairs
     float* yp = a.y_dump + unit * E;
 #pragma unroll
     for (int j = 0; j < E / 8; ++j) {
-      const float sg = ((lx.flips >> j) & 1u) ? -c : c;
+      const uint32_t msk = chunk_sign_mask<Cfg::kBlock>(lx, j);
+      const float se = (msk & 0x08u) ? -c : c;    // even elements: the chunk flip only
+      const float so = (msk & 0x80u) ? -c : c;    // odd elements: flip and first-stage negation
       float v[8];
 #pragma unroll
       for (int t = 0; t < 4; ++t) f2_unpack(p[4 * j + t], v[2 * t], v[2 * t + 1]);
-      reinterpret_cast<float4*>(yp)[2 * j] = make_float4(v[0] * sg, v[1] * sg, v[2] * sg, v[3] * sg);
-      reinterpret_cast<float4*>(yp)[2 * j + 1] = make_float4(v[4] * sg, v[5] * sg, v[6] * sg, v[7] * sg);
+      reinterpret_cast<float4*>(yp)[2 * j] = make_float4(v[0] * se, v[1] * so, v[2] * se, v[3] * so);
+      reinterpret_cast<float4*>(yp)[2 * j + 1] = make_float4(v[4] * se, v[5] * so, v[6] * se, v[7] * so);
     }
   }
 }
