@@ -128,6 +128,12 @@ __device__ __forceinline__ f32x2 f2_mul(f32x2 a, f32x2 b) {
   return r;
 }
 
+__device__ __forceinline__ f32x2 f2_fma(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
 // First butterfly stage straight from a bf16 pair word (element 2k in the low half):
 // (x[2k] + x[2k+1], x[2k+1] - x[2k]), each rounded once to fp32, as a packed pair.  The
 // second entry is the negated difference: the mixed-precision add takes the high bf16 half

@@ -71,6 +71,36 @@ __device__ __forceinline__ void fwht_inplace(float (&v)[E]) {
   }
 }
 
+// 1/sqrt(b) as an unevaluated sum hi + lo of two fp32 values (hi = RN(1/sqrt(b))).  Then
+// fma(s, hi, RN(s lo)) is the correctly rounded s/sqrt(b) except when s/sqrt(b) lies within
+// about 2^-48 (relative) of a rounding boundary.
+__host__ __device__ constexpr double inv_sqrt_block_f64(int b) {
+  return b == 1     ? 1.0
+         : b == 2   ? 0.70710678118654752440
+         : b == 4   ? 0.5
+         : b == 8   ? 0.35355339059327376220
+         : b == 16  ? 0.25
+         : b == 32  ? 0.17677669529663688110
+         : b == 64  ? 0.125
+         : b == 128 ? 0.08838834764831844055
+                    : 0.0;
+}
+__host__ __device__ constexpr float inv_sqrt_block_lo(int b) {
+  return static_cast<float>(inv_sqrt_block_f64(b) - static_cast<double>(inv_sqrt_block(b)));
+}
+// 1/sqrt(b) is a power of two for b = 1, 4, 16, 64 (even log2 b).
+__host__ __device__ constexpr bool inv_sqrt_block_is_pow2(int b) { return (ilog2(b) & 1) == 0; }
+
+// Correctly rounded m / sqrt(b) (see inv_sqrt_block_lo).
+template <int B>
+__device__ __forceinline__ float scale_by_inv_sqrt(float m) {
+  if constexpr (inv_sqrt_block_is_pow2(B)) {
+    return m * inv_sqrt_block(B);
+  } else {
+    return fmaf(m, inv_sqrt_block(B), m * inv_sqrt_block_lo(B));
+  }
+}
+
 // Compile-time shape of one kernel instance.  MINU is the smallest unit: 32 when the
 // tensor's element count allows it (fewer per-unit costs, 16-byte code stores), else 16.
 template <int FMT, int B, int RULE, bool DUMP, int MINU = 32>
@@ -234,29 +264,50 @@ __device__ __forceinline__ void quantize_store_unit(const f32x2 (&p)[Cfg::kPairs
   uint32_t sbytes[NG];
 #pragma unroll
   for (int q = 0; q < NG; ++q) {
-    const float A = pairs_amax<G / 2>(&p[q * G / 2]) * c;   // = max |fl(v c)|: rounding is monotonic
-    float mult;
-    uint32_t keep = 0xFFFFFFFFu;
+    // group amax of the fp32 rotated values: RN(max |s| / sqrt(b)) = max |RN(s / sqrt(b))|
+    const float A = scale_by_inv_sqrt<Cfg::kBlock>(pairs_amax<G / 2>(&p[q * G / 2]));
     if constexpr (Cfg::kFmt == kMX) {
       const int byte = mx_scale_byte<Cfg::kRule>(A);
       sbytes[q] = static_cast<uint32_t>(byte);
-      mult = c * mx_inv_scale(byte);      // exact: a power-of-two multiple of c
+      const float mult = c * mx_inv_scale(byte);   // a power-of-two multiple of c
+      const f32x2 mm = f2_pack(mult, mult);
+#pragma unroll
+      for (int j = 0; j < G / 8; ++j) {
+        const int chunk = q * (G / 8) + j;
+        float v[8];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) f2_unpack(f2_mul(p[4 * chunk + t], mm), v[2 * t], v[2 * t + 1]);
+        words[chunk] = e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]) ^ chunk_sign_mask<Cfg::kBlock>(lx, chunk);
+      }
     } else {
       const float s_b = div_rn_markstein(A, nv_den, nv_rden);
       const uint32_t byte = e4m3_encode(s_b);
       sbytes[q] = byte;
       const float S = e4m3_decode(byte) * s_g;
-      if (S == 0.0f) keep = 0u;           // a zero block scale gives zero codes
-      mult = S == 0.0f ? 0.0f : c * rcp_approx(S);
-    }
-    const f32x2 mm = f2_pack(mult, mult);
+      const uint32_t keep = S == 0.0f ? 0u : 0xFFFFFFFFu;   // a zero block scale gives zero codes
+      // Element code from the correctly rounded quotient y / S, y = RN(s / sqrt(b)).  With a
+      // power-of-two 1/sqrt(b) it is folded into the divisor (exactly): s / (S sqrt(b)).
+      const float Sd = inv_sqrt_block_is_pow2(Cfg::kBlock) ? S * (1.0f / c) : S;
+      const float rd = __frcp_rn(Sd);
+      const f32x2 rd2 = f2_pack(rd, rd), nSd2 = f2_pack(-Sd, -Sd);
 #pragma unroll
-    for (int j = 0; j < G / 8; ++j) {
-      const int chunk = q * (G / 8) + j;
-      float v[8];
+      for (int j = 0; j < G / 8; ++j) {
+        const int chunk = q * (G / 8) + j;
+        float v[8];
 #pragma unroll
-      for (int t = 0; t < 4; ++t) f2_unpack(f2_mul(p[4 * chunk + t], mm), v[2 * t], v[2 * t + 1]);
-      words[chunk] = (e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]) ^ chunk_sign_mask<Cfg::kBlock>(lx, chunk)) & keep;
+        for (int t = 0; t < 4; ++t) {
+          f32x2 y = p[4 * chunk + t];
+          if constexpr (!inv_sqrt_block_is_pow2(Cfg::kBlock)) {
+            constexpr float chi = inv_sqrt_block(Cfg::kBlock), clo = inv_sqrt_block_lo(Cfg::kBlock);
+            y = f2_fma(y, f2_pack(chi, chi), f2_mul(y, f2_pack(clo, clo)));
+          }
+          const f32x2 q0 = f2_mul(y, rd2);                  // Markstein correction, lane-wise
+          const f32x2 rem = f2_fma(q0, nSd2, y);
+          f2_unpack(f2_fma(rem, rd2, q0), v[2 * t], v[2 * t + 1]);
+        }
+        words[chunk] = (e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]) ^
+                        chunk_sign_mask<Cfg::kBlock>(lx, chunk)) & keep;
+      }
     }
   }
   // codes: E/2 bytes per unit
