@@ -130,6 +130,34 @@ fp4q_status fp4q_dequantize(fp4q_plan plan, const void* codes, const void* scale
                             const float* tensor_scale, int64_t M, int64_t K, int unrotate,
                             float* out_f32, void* stream);
 
+/* No-allocation NVFP4 dynamic-scale path.  The paper has no counterpart: this exists for
+ * callers that cannot allocate device memory themselves — for example a library loaded into
+ * a framework or serving runtime whose own allocator owns all device memory, or a service that
+ * must not allocate after start-up — and so cannot create an FP4Q_SCALE_NV_DYNAMIC plan, whose
+ * creation allocates the plan's partial-maximum array.
+ *
+ * Same computation and output layout as fp4q_rotate_quantize with a plan
+ * (FP4Q_NVFP4, 16, hadamard_block, FP4Q_SCALE_NV_DYNAMIC): x_bf16 device bf16 [M][K];
+ * codes_out device uint8 [M][K/2]; scales_out device uint8 [M][K/16]; tensor_scale_out
+ * device fp32, written with the s_g the call used.  The caller still owns and passes every
+ * input and output.
+ *
+ * Scratch: the per-CTA partial maxima live in a fixed array inside this library (4096 fp32
+ * values, 16 KB), reserved on every GPU that loads the library until the process exits.
+ * The call needs one value per CTA of its amax pass (a full wave: SM count x resident CTAs
+ * per SM); when that exceeds 4096 it returns FP4Q_ERR_UNSUPPORTED before launching anything
+ * and fp4q_last_cuda_error() names the limit.  Every call overwrites the values it reads, so
+ * nothing carries over from earlier calls; calls that overlap on the GPU (other streams, other
+ * host threads) share the array and race.
+ *
+ * Allocation: none — no cudaMalloc, cudaFree or allocating library routine.  The first call
+ * on each device does a one-time set-up there (it looks up the array's device address and
+ * configures the kernels); make that first call outside any stream capture. */
+fp4q_status fp4q_rotate_quantize_nvfp4_dynamic_noalloc(const void* x_bf16, int64_t M, int64_t K,
+                                                       int hadamard_block, void* codes_out,
+                                                       void* scales_out, float* tensor_scale_out,
+                                                       void* stream);
+
 /* Read and clear the device-side status word (FP4Q_OK, or FP4Q_ERR_TIMEOUT when a bounded
  * wait ran out in a kernel since the last read).  Synchronizes the current device. */
 fp4q_status fp4q_device_status(void);

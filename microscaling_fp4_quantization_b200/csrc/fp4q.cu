@@ -205,9 +205,100 @@ fp4q_status rotate_quantize_impl(fp4q_plan p, const void* x, int64_t M, int64_t 
   });
 }
 
+// ---- no-allocation NVFP4 dynamic path: partial maxima in a fixed device array
+
+constexpr int kNoAllocMaxPartials = 4096;
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+}  // namespace
+
+// Scratch of the no-allocation entry point (the host name below is only a stand-in; kernels
+// get the device address from cudaGetSymbolAddress).
+static __device__ __align__(256) float g_noalloc_partials[kNoAllocMaxPartials];
+
+namespace {
+
+// Device address of g_noalloc_partials on the current device, looked up once per device.
+fp4q_status noalloc_scratch(float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return FP4Q_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    float* ptr = nullptr;
+    e = cudaGetSymbolAddress(reinterpret_cast<void**>(&ptr), g_noalloc_partials);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FP4Q_OK;
+}
+
+template <class Cfg>
+fp4q_status noalloc_amax_launch(const uint16_t* x, int64_t n_elems, float* partials, int n_partials,
+                                cudaStream_t stream) {
+  rotated_amax_kernel<Cfg><<<n_partials, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(x, n_elems / Cfg::kE, partials);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "amax launch");
+  return FP4Q_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+fp4q_status fp4q_rotate_quantize_nvfp4_dynamic_noalloc(const void* x_bf16, int64_t M, int64_t K, int hadamard_block,
+                                                       void* codes_out, void* scales_out, float* tensor_scale_out,
+                                                       void* stream) {
+  if (hadamard_block < 1 || hadamard_block > 128 || (hadamard_block & (hadamard_block - 1)) != 0)
+    return FP4Q_ERR_UNSUPPORTED;
+  const int64_t unit = hadamard_block > 16 ? hadamard_block : 16;
+  if (M < 0 || K < 0 || K % unit != 0) return FP4Q_ERR_SHAPE;
+  if (M > 0 && K > 0 && M > (int64_t(1) << 40) / K) return FP4Q_ERR_SHAPE;
+  if (!tensor_scale_out) return FP4Q_ERR_ARG;
+  if (M * K == 0) return FP4Q_OK;
+  if (!x_bf16 || !codes_out || !scales_out) return FP4Q_ERR_ARG;
+  if (!aligned(x_bf16, 16) || !aligned(codes_out, 16) || !aligned(scales_out, 16) || !aligned(tensor_scale_out, 4))
+    return FP4Q_ERR_ALIGN;
+  float* partials = nullptr;
+  fp4q_status st = noalloc_scratch(&partials);
+  if (st != FP4Q_OK) return st;
+  int n_partials = 0;
+  st = amax_grid(hadamard_block, &n_partials);
+  if (st != FP4Q_OK) return st;
+  if (n_partials > kNoAllocMaxPartials) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+                  "fp4q_rotate_quantize_nvfp4_dynamic_noalloc: the amax pass needs %d partial maxima, "
+                  "the fixed scratch holds %d",
+                  n_partials, kNoAllocMaxPartials);
+    return FP4Q_ERR_UNSUPPORTED;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t n = M * K;
+  const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
+  RQArgs a;
+  a.x = x;
+  a.n_units = 0;
+  a.codes = static_cast<uint8_t*>(codes_out);
+  a.scales = static_cast<uint8_t*>(scales_out);
+  a.tensor_scale = tensor_scale_out;
+  a.partials = partials;
+  a.n_partials = n_partials;
+  a.y_dump = nullptr;
+  return with_block(hadamard_block, [&]<int B>() -> fp4q_status {
+    if (n % 32 == 0) {
+      fp4q_status r = noalloc_amax_launch<AmaxCfg<B, 32>>(x, n, partials, n_partials, s);
+      if (r != FP4Q_OK) return r;
+      return launch_rq<RQConfig<kNV, B, kRuleNvDynamic, false, 32>>(a, n, s);
+    }
+    fp4q_status r = noalloc_amax_launch<AmaxCfg<B, 16>>(x, n, partials, n_partials, s);
+    if (r != FP4Q_OK) return r;
+    return launch_rq<RQConfig<kNV, B, kRuleNvDynamic, false, 16>>(a, n, s);
+  });
+}
 
 fp4q_status fp4q_plan_create(fp4q_plan* out, int format, int group, int hadamard_block, int scale_rule) {
   if (!out) return FP4Q_ERR_ARG;

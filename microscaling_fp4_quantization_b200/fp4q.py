@@ -37,6 +37,7 @@ _SIGS = {
     "fp4q_rotate_quantize_dump": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
     "fp4q_amax": (_int, [_vp, _vp, _i64, _i64, _vp, _vp]),
     "fp4q_dequantize": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _int, _vp, _vp]),
+    "fp4q_rotate_quantize_nvfp4_dynamic_noalloc": (_int, [_vp, _i64, _i64, _int, _vp, _vp, _vp, _vp]),
     "fp4q_device_status": (_int, []),
     "fp4q_status_string": (ctypes.c_char_p, [_int]),
     "fp4q_last_cuda_error": (ctypes.c_char_p, []),
@@ -135,6 +136,16 @@ def fp4q_dequantize(plan: Plan, codes, scales, tensor_scale, M: int, K: int, unr
                     stream=None) -> None:
     _check(_lib.fp4q_dequantize(plan.handle, _ptr(codes), _ptr(scales), _ptr(tensor_scale), M, K,
                                 int(bool(unrotate)), _ptr(out_f32), _stream(stream)), "fp4q_dequantize")
+
+
+def fp4q_rotate_quantize_nvfp4_dynamic_noalloc(x, M: int, K: int, hadamard_block: int, codes_out, scales_out,
+                                                tensor_scale_out, stream=None) -> None:
+    """NVFP4 dynamic-scale rotate + quantize without any device allocation (its scratch is a
+    fixed array inside the library); for callers that cannot allocate device memory."""
+    _check(_lib.fp4q_rotate_quantize_nvfp4_dynamic_noalloc(_ptr(x), M, K, hadamard_block, _ptr(codes_out),
+                                                           _ptr(scales_out), _ptr(tensor_scale_out),
+                                                           _stream(stream)),
+           "fp4q_rotate_quantize_nvfp4_dynamic_noalloc")
 
 
 def fp4q_device_status() -> int:
