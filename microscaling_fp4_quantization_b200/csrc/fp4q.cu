@@ -7,6 +7,7 @@
 #include <mutex>
 #include <new>
 #include <unordered_map>
+#include <utility>
 
 #include "fp4q.h"
 #include "fp4q_kernels.cuh"
@@ -72,6 +73,25 @@ fp4q_status kernel_info(K kernel, int smem_bytes, int threads, KernelInfo* out) 
   return FP4Q_OK;
 }
 
+// Launch with programmatic stream serialization, so the kernel's start overlaps the tail of
+// the previous kernel on the stream (the kernels wait on the dependency before touching
+// global memory).
+template <class... KArgs, class... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // Call f.template operator()<B>() for the runtime Hadamard block b.
 template <class F>
 fp4q_status with_block(int b, F&& f) {
@@ -99,8 +119,7 @@ fp4q_status launch_rq(RQArgs a, int64_t n_elems, cudaStream_t stream) {
   int64_t ctas = (warps_needed + Cfg::kWarps - 1) / Cfg::kWarps;
   const int64_t max_ctas = static_cast<int64_t>(ki.sm_count) * ki.ctas_per_sm;
   if (ctas > max_ctas) ctas = max_ctas;
-  kernel<<<static_cast<unsigned>(ctas), Cfg::kThreads, Cfg::kSmemBytes, stream>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(kernel, dim3(static_cast<unsigned>(ctas)), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, a);
   if (e != cudaSuccess) return cuda_fail(e, "rotate_quantize launch");
   return FP4Q_OK;
 }
@@ -126,9 +145,8 @@ fp4q_status amax_grid(int b, int* n) {
 
 template <class Cfg>
 fp4q_status launch_amax_cfg(fp4q_plan p, const uint16_t* x, int64_t n_elems, cudaStream_t stream) {
-  rotated_amax_kernel<Cfg><<<p->n_partials, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(x, n_elems / Cfg::kE,
-                                                                                        p->partials);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(rotated_amax_kernel<Cfg>, dim3(p->n_partials), dim3(Cfg::kThreads), Cfg::kSmemBytes,
+                             stream, x, n_elems / Cfg::kE, p->partials);
   if (e != cudaSuccess) return cuda_fail(e, "amax launch");
   return FP4Q_OK;
 }
@@ -378,8 +396,9 @@ fp4q_status fp4q_amax(fp4q_plan plan, const void* x_bf16, int64_t M, int64_t K, 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   st = launch_amax(plan, static_cast<const uint16_t*>(x_bf16), M * K, s);
   if (st != FP4Q_OK) return st;
-  tensor_scale_finalize_kernel<<<1, 32, 0, s>>>(plan->partials, plan->n_partials, tensor_scale_out);
-  cudaError_t e = cudaGetLastError();
+  const float* partials = plan->partials;
+  cudaError_t e = launch_pdl(tensor_scale_finalize_kernel, dim3(1), dim3(32), 0, s, partials, plan->n_partials,
+                             tensor_scale_out);
   if (e != cudaSuccess) return cuda_fail(e, "finalize launch");
   return FP4Q_OK;
 }

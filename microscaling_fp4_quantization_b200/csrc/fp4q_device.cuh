@@ -72,6 +72,12 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
   }
 }
 
+// Programmatic dependent launch.  launch_dependents lets the next kernel on the stream be
+// scheduled while this one runs; wait blocks until every kernel this one depends on has
+// finished and its memory is visible (a no-op when launched without the attribute).
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Bulk copy (no tensor map) global -> shared, completion signalled on an mbarrier as
 // transaction bytes.  dst, src 16-byte aligned; bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {

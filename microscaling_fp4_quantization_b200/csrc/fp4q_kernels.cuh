@@ -118,7 +118,7 @@ struct RQConfig {
   static constexpr int kR = cmax(1, 32 / kE);
   static constexpr int kUnitsPerStage = 32 * kR;
   static constexpr int kStageBytes = kUnitsPerStage * kE * 2;
-  static constexpr int kStages = kE >= 64 ? 3 : 4;
+  static constexpr int kStages = kE >= 64 ? 3 : 2;
   static constexpr int kWarps = kE >= 128 ? 2 : 4;        // warps per CTA
   static constexpr int kThreads = kWarps * 32;
   // Chunk-index XOR (see the file comment): as many low chunk bits as make a quarter-warp
@@ -378,8 +378,12 @@ __device__ __forceinline__ bool stream_units(const uint16_t* __restrict__ x, int
   if (lane == 0) {
     for (int s = 0; s < S; ++s) mbar_init(bar0 + 8u * s, 1);
     fence_mbar_init();
-    for (int64_t t = 0; t < S && t < n_stages; ++t) issue(t);
   }
+  // Nothing below reads or writes global memory before the kernels this one depends on
+  // (for example the producer of x) have finished.
+  pdl_wait();
+  if (lane == 0)
+    for (int64_t t = 0; t < S && t < n_stages; ++t) issue(t);
   __syncwarp();
 
   bool ok = true;
@@ -433,10 +437,12 @@ template <class Cfg>
 __global__ void __launch_bounds__(Cfg::kThreads) rotate_quantize_kernel(RQArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float s_tensor_scale;
+  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5;
   const LaneXor lx = lane_xor<Cfg>(threadIdx.x & 31);
   float s_g = 1.0f;
   if constexpr (Cfg::kFmt == kNV) {
+    pdl_wait();   // the tensor scale or the partial maxima come from an earlier kernel
     if constexpr (Cfg::kRule == kRuleNvDynamic) {
       if (warp == 0) {
         float m = 0.0f;
@@ -469,6 +475,7 @@ __global__ void __launch_bounds__(Cfg::kThreads) rotated_amax_kernel(const uint1
                                                                      float* __restrict__ partials) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float s_max[Cfg::kWarps];
+  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5;
   const LaneXor lx = lane_xor<Cfg>(threadIdx.x & 31);
   float m = 0.0f;
@@ -488,6 +495,8 @@ __global__ void __launch_bounds__(Cfg::kThreads) rotated_amax_kernel(const uint1
 
 // s_g = fp32(max(partials) / 2688), 1 for an all-zero tensor.  One warp.
 __global__ void tensor_scale_finalize_kernel(const float* __restrict__ partials, int n, float* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait();
   float m = 0.0f;
   for (int i = threadIdx.x; i < n; i += 32) m = fmaxf(m, partials[i]);
 #pragma unroll
