@@ -39,11 +39,19 @@ sys.path.insert(0, ROOT)
 from microscaling_fp4_quantization_b200 import workloads as W  # noqa: E402
 
 METRIC = "fused rotate+FP4-quantize GB/s (bf16 in + packed out), % of B200 HBM peak"
+KERNELS = {"auto": 0, "butterfly": 1, "tensor_core": 2}
+
+
+def kernel_name(w, requested: str) -> str:
+    """The kernel a plan with this request runs (auto: tensor core when b >= 16 and b >= g)."""
+    if requested != "auto":
+        return requested
+    return "tensor_core" if (w.block >= 16 and w.block >= w.group) else "butterfly"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 SPEC_HBM_GBS = 8000.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "rotate_quantize_nvfp4_b16_4096x4096.md")
-KERNEL_SOURCES = ["fp4q.cu", "fp4q_kernels.cuh", "fp4q_device.cuh"]
+KERNEL_SOURCES = ["fp4q.cu", "fp4q_kernels.cuh", "fp4q_device.cuh", "fp4q_mma.cuh"]
 
 
 def kernel_source_hash() -> str:
@@ -187,6 +195,7 @@ def run_gpu(args):
     w = workload_for(args)
     M, K = w.M, w.K
     plan = F.fp4q_plan_create(w.fmt, w.group, w.block, w.rule)
+    F.fp4q_plan_set_kernel(plan, KERNELS[args.kernel])
     x_np = w.generate()
     bytes_call = w.bytes_per_call()
     n_buf = max(1, math.ceil(3 * L2_BYTES / bytes_call)) if bytes_call < 2 * L2_BYTES else 1
@@ -314,9 +323,14 @@ def run_gpu(args):
 
     # the other workloads' throughput, each timed the same way (rank 0, when asked)
     others = {}
+    if rank == 0 and kernel_name(w, "auto") == "tensor_core" and args.kernel == "auto":
+        # the measured alternative: the same workload on the butterfly kernel
+        extra["butterfly_kernel"] = time_other(torch, F, w, dev, stream, peak, kernel="butterfly")
     if args.all_workloads and rank == 0:
-        for ow in (W.MX_8K_FLOOR, W.MX_8K_CEIL, W.PREFILL_NV, W.PREFILL_MX) + W.DECODE:
+        for ow in (W.SMALL_MX, W.MX_8K_FLOOR, W.MX_8K_CEIL, W.PREFILL_NV, W.PREFILL_MX) + W.DECODE:
             others[ow.name] = time_other(torch, F, ow, dev, stream, peak)
+            if kernel_name(ow, "auto") == "tensor_core":
+                others[ow.name + " [butterfly kernel]"] = time_other(torch, F, ow, dev, stream, peak, kernel="butterfly")
 
     if rank == 0:
         cpu = cpu_baseline(w, args) if world == 1 and not args.no_cpu_baseline else None
@@ -338,6 +352,7 @@ def run_gpu(args):
                 "workload": w.name, "M": M, "K": K,
                 "format": "NVFP4" if is_nv else "MXFP4", "group": w.group, "hadamard_block": w.block,
                 "scale_rule": W.RULE_NAMES[w.rule], "bytes_per_step": bytes_call,
+                "kernel": kernel_name(w, args.kernel),
                 "l2": f"inputs larger than L2 per step: {n_buf} rotating buffer sets "
                       f"({n_buf * bytes_call / 1e6:.0f} MB in total)" if n_buf > 1 else "input larger than L2",
                 "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
@@ -354,7 +369,8 @@ def run_gpu(args):
                 "traffic": traffic,
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                 else "fallback 6650 GB/s",
-                "kernel": "rotate_quantize_kernel", "us_per_launch": round(kernel_us, 3),
+                "kernel": ("rotate_quantize_mma_kernel" if kernel_name(w, args.kernel) == "tensor_core"
+                           else "rotate_quantize_kernel"), "us_per_launch": round(kernel_us, 3),
             },
             "gpu_launches": args.steps,
             "clocks": sampler.summary(),
@@ -383,6 +399,7 @@ def run_kernel_only(args):
     torch.cuda.set_device(0)
     w = workload_for(args)
     plan = F.fp4q_plan_create(w.fmt, w.group, w.block, w.rule)
+    F.fp4q_plan_set_kernel(plan, KERNELS[args.kernel])
     x = torch.from_numpy(w.generate().view(np.int16)).view(torch.bfloat16).cuda()
     codes = torch.empty((w.M, w.K // 2), dtype=torch.uint8, device="cuda")
     scales = torch.empty((w.M, w.K // w.group), dtype=torch.uint8, device="cuda")
@@ -396,9 +413,10 @@ def run_kernel_only(args):
     print(f"kernel-only: {w.name} M={w.M} K={w.K} launches={args.warmup + args.steps}", flush=True)
 
 
-def time_other(torch, F, w, dev, stream, peak):
+def time_other(torch, F, w, dev, stream, peak, kernel="auto"):
     M, K = w.M, w.K
     plan = F.fp4q_plan_create(w.fmt, w.group, w.block, w.rule)
+    F.fp4q_plan_set_kernel(plan, KERNELS[kernel])
     x_np = w.generate()
     bytes_call = w.bytes_per_call()
     n_buf = max(1, math.ceil(3 * L2_BYTES / bytes_call)) if bytes_call < 2 * L2_BYTES else 1
@@ -430,7 +448,7 @@ def time_other(torch, F, w, dev, stream, peak):
     us = a0.elapsed_time(a1) * 1e3 / steps
     gbs = bytes_call / us / 1e3
     out = {"GBps": round(gbs, 1), "pct_of_hbm_peak": round(100 * gbs / peak, 2), "us_per_call": round(us, 3),
-           "bytes_per_call": bytes_call, "buffers": n_buf}
+           "bytes_per_call": bytes_call, "buffers": n_buf, "kernel": kernel_name(w, kernel)}
     del xs, codes, scales
     torch.cuda.empty_cache()
     return out
@@ -508,6 +526,8 @@ def main():
     ap.add_argument("--all-workloads", action="store_true", help="also time the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rows", type=int, default=0, help="override the workload's row count M")
+    ap.add_argument("--kernel", default="auto", choices=["auto", "butterfly", "tensor_core"],
+                    help="which rotate + quantize kernel the plan uses")
     ap.add_argument("--kernel-only", action="store_true",
                     help="only W + K plain launches of the workload (a case for profilers), no JSON line")
     args = ap.parse_args()

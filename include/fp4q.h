@@ -36,7 +36,7 @@
  * Layout (all row-major, contiguous):
  *   x        bf16  [M][K]          device memory, 16-byte aligned
  *   codes    uint8 [M][K/2]        device memory, 16-byte aligned
- *   scales   uint8 [M][K/g]        device memory, 16-byte aligned when K/g*M >= 16
+ *   scales   uint8 [M][K/g]        device memory, 16-byte aligned
  *                                  (E8M0 bytes for MXFP4, E4M3 bytes for NVFP4)
  *   tensor_scale  one fp32 in device memory (NVFP4 only; NULL for MXFP4)
  *
@@ -96,6 +96,21 @@ typedef struct fp4q_plan_s* fp4q_plan;
  * maximum array on the current CUDA device, which every later call must also use. */
 fp4q_status fp4q_plan_create(fp4q_plan* out, int format, int group, int hadamard_block,
                              int scale_rule);
+
+/* Which kernel a plan's rotate + quantize calls run on. */
+typedef enum {
+  FP4Q_KERNEL_AUTO = 0,        /* the tensor-core kernel when every Hadamard block holds whole
+                                  scale groups (b >= 16 and b >= g), else the butterfly kernel */
+  FP4Q_KERNEL_BUTTERFLY = 1,   /* in-register fast Walsh-Hadamard butterfly on CUDA cores    */
+  FP4Q_KERNEL_TENSOR_CORE = 2  /* tcgen05 MMA against H_b with TMEM accumulators            */
+} fp4q_kernel;
+
+/* Choose the kernel for later rotate + quantize calls of this plan (not thread-safe against
+ * calls running on the same plan).  Returns FP4Q_ERR_UNSUPPORTED for FP4Q_KERNEL_TENSOR_CORE
+ * when b < 16 or b < g.  Both kernels compute the same function (see fp4q_rotate_quantize);
+ * they round the butterfly sums differently, so rare codes within the parity tolerance of a
+ * rounding boundary can differ between them. */
+fp4q_status fp4q_plan_set_kernel(fp4q_plan plan, int kernel);
 
 /* Free a plan (NULL is accepted).  Synchronizes nothing: the caller must make sure no
  * call using the plan is still running on the device. */

@@ -18,7 +18,7 @@ LIB_DIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIB_DIR, "libfp4q.so")
 
 SOURCES = ["fp4q.cu"]
-DEPS = ["fp4q.cu", "fp4q_kernels.cuh", "fp4q_device.cuh"]
+DEPS = ["fp4q.cu", "fp4q_kernels.cuh", "fp4q_device.cuh", "fp4q_mma.cuh"]
 
 
 def nvcc() -> str:

@@ -11,6 +11,7 @@
 
 #include "fp4q.h"
 #include "fp4q_kernels.cuh"
+#include "fp4q_mma.cuh"
 
 using namespace fp4q;
 
@@ -21,6 +22,7 @@ struct fp4q_plan_s {
   int device;
   float* partials; // NV plans: per-CTA rotated amaxima (device)
   int n_partials;
+  int kernel;      // fp4q_kernel
 };
 
 namespace {
@@ -124,6 +126,79 @@ fp4q_status launch_rq(RQArgs a, int64_t n_elems, cudaStream_t stream) {
   return FP4Q_OK;
 }
 
+// ---- tensor-core kernel: TMA tensor map over the rows of one Hadamard block each
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::mutex g_encode_mu;
+EncodeTiledFn g_encode = nullptr;
+
+fp4q_status encode_fn(EncodeTiledFn* out) {
+  std::lock_guard<std::mutex> lk(g_encode_mu);
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)");
+    if (q != cudaDriverEntryPointSuccess || !fn) return cuda_fail(cudaErrorNotSupported, "cuTensorMapEncodeTiled");
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  *out = g_encode;
+  return FP4Q_OK;
+}
+
+template <class Cfg>
+fp4q_status launch_mma(const uint16_t* x, int64_t n_elems, const RQArgs& ra, cudaStream_t stream) {
+  EncodeTiledFn enc;
+  fp4q_status st = encode_fn(&enc);
+  if (st != FP4Q_OK) return st;
+  MmaArgs a;
+  a.n_rows = n_elems / Cfg::kBlock;
+  a.n_super = (a.n_rows + Cfg::kRowsPerTile - 1) / Cfg::kRowsPerTile;
+  a.codes = ra.codes;
+  a.scales = ra.scales;
+  a.tensor_scale = ra.tensor_scale;
+  a.partials = ra.partials;
+  a.n_partials = ra.n_partials;
+  a.y_dump = ra.y_dump;
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(Cfg::kBlock), static_cast<cuuint64_t>(a.n_rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(Cfg::kBlock) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(Cfg::kKB), static_cast<cuuint32_t>(Cfg::kBoxRows)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw = Cfg::kRB == 32   ? CU_TENSOR_MAP_SWIZZLE_32B
+                                : Cfg::kRB == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                 : CU_TENSOR_MAP_SWIZZLE_128B;
+  CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(x), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return FP4Q_ERR_CUDA;
+  }
+  auto kernel = rotate_quantize_mma_kernel<Cfg>;
+  KernelInfo ki;
+  st = kernel_info(kernel, Cfg::kSmemBytes, Cfg::kThreads, &ki);
+  if (st != FP4Q_OK) return st;
+  int per_sm = ki.ctas_per_sm;
+  if (per_sm > 512 / Cfg::kTmemCols) per_sm = 512 / Cfg::kTmemCols;   // tensor memory: 512 columns per SM
+  int64_t ctas = static_cast<int64_t>(ki.sm_count) * per_sm;
+  if (ctas > a.n_super) ctas = a.n_super;
+  cudaError_t e = launch_pdl(kernel, dim3(static_cast<unsigned>(ctas)), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream,
+                             map, a);
+  if (e != cudaSuccess) return cuda_fail(e, "rotate_quantize (tensor core) launch");
+  return FP4Q_OK;
+}
+
+// Whether the tensor-core kernel serves this plan.
+bool mma_capable(fp4q_plan p) { return p->block >= 16 && p->block >= p->group; }
+bool use_mma(fp4q_plan p) {
+  if (!mma_capable(p)) return false;
+  return p->kernel == FP4Q_KERNEL_AUTO || p->kernel == FP4Q_KERNEL_TENSOR_CORE;
+}
+
 template <int B, int MINU>
 using AmaxCfg = RQConfig<kNV, B, kRuleNvStatic, false, MINU>;
 
@@ -190,6 +265,35 @@ fp4q_status rotate_quantize_impl(fp4q_plan p, const void* x, int64_t M, int64_t 
   if (p->format == FP4Q_NVFP4 && p->rule == FP4Q_SCALE_NV_DYNAMIC) {
     st = launch_amax(p, a.x, n, s);
     if (st != FP4Q_OK) return st;
+  }
+  if (use_mma(p)) {
+    return with_block(p->block, [&]<int B>() -> fp4q_status {
+      if constexpr (B >= 16) {
+        if (p->format == FP4Q_MXFP4) {
+          if constexpr (B >= 32) {
+            switch (p->rule) {
+              case FP4Q_SCALE_FLOOR_OCP:
+                return dump ? launch_mma<MmaConfig<kMX, B, kRuleFloor, true>>(a.x, n, a, s)
+                            : launch_mma<MmaConfig<kMX, B, kRuleFloor, false>>(a.x, n, a, s);
+              case FP4Q_SCALE_CEIL_NOCLIP:
+                return dump ? launch_mma<MmaConfig<kMX, B, kRuleCeil, true>>(a.x, n, a, s)
+                            : launch_mma<MmaConfig<kMX, B, kRuleCeil, false>>(a.x, n, a, s);
+              case FP4Q_SCALE_OAS:
+                return dump ? launch_mma<MmaConfig<kMX, B, kRuleOas, true>>(a.x, n, a, s)
+                            : launch_mma<MmaConfig<kMX, B, kRuleOas, false>>(a.x, n, a, s);
+              default: return FP4Q_ERR_UNSUPPORTED;
+            }
+          }
+          return FP4Q_ERR_UNSUPPORTED;
+        }
+        if (p->rule == FP4Q_SCALE_NV_DYNAMIC)
+          return dump ? launch_mma<MmaConfig<kNV, B, kRuleNvDynamic, true>>(a.x, n, a, s)
+                      : launch_mma<MmaConfig<kNV, B, kRuleNvDynamic, false>>(a.x, n, a, s);
+        return dump ? launch_mma<MmaConfig<kNV, B, kRuleNvStatic, true>>(a.x, n, a, s)
+                    : launch_mma<MmaConfig<kNV, B, kRuleNvStatic, false>>(a.x, n, a, s);
+      }
+      return FP4Q_ERR_UNSUPPORTED;
+    });
   }
   return with_block(p->block, [&]<int B>() -> fp4q_status {
     if (p->format == FP4Q_MXFP4) {
@@ -344,6 +448,7 @@ fp4q_status fp4q_plan_create(fp4q_plan* out, int format, int group, int hadamard
   p->device = -1;
   p->partials = nullptr;
   p->n_partials = 0;
+  p->kernel = FP4Q_KERNEL_AUTO;
   if (format == FP4Q_NVFP4) {
     cudaError_t e = cudaGetDevice(&p->device);
     fp4q_status st = e == cudaSuccess ? amax_grid(hadamard_block, &p->n_partials) : cuda_fail(e, "cudaGetDevice");
@@ -358,6 +463,15 @@ fp4q_status fp4q_plan_create(fp4q_plan* out, int format, int group, int hadamard
     }
   }
   *out = p;
+  return FP4Q_OK;
+}
+
+fp4q_status fp4q_plan_set_kernel(fp4q_plan plan, int kernel) {
+  if (!valid_plan(plan)) return FP4Q_ERR_ARG;
+  if (kernel != FP4Q_KERNEL_AUTO && kernel != FP4Q_KERNEL_BUTTERFLY && kernel != FP4Q_KERNEL_TENSOR_CORE)
+    return FP4Q_ERR_ARG;
+  if (kernel == FP4Q_KERNEL_TENSOR_CORE && !mma_capable(plan)) return FP4Q_ERR_UNSUPPORTED;
+  plan->kernel = kernel;
   return FP4Q_OK;
 }
 

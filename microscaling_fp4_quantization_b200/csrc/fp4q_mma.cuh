@@ -1,0 +1,412 @@
+// Tensor-core variant of the fused rotate + FP4 quantize kernel (sm_100a tcgen05).
+//
+// The flat stream of M*K bf16 values is read as R = M*K/b rows of one Hadamard block each,
+// and the rotation is the product Y = X_rows * H_b: an M = 128, N = b, K = b bf16 MMA with
+// fp32 accumulation in tensor memory (TMEM).  The products x * (+-1) are exact; the sums
+// are accumulated in fp32 by the tensor core.
+//
+// Work is cut into super-tiles of 128 rows by 64 TMEM columns (b <= 64: 64 / b row-tiles of
+// 128 rows, 16 KB of input) or 128 columns (b = 128, 32 KB).
+// Roles, per CTA of 6 warps:
+//   warp 0        producer: TMA tensor loads (2-D map over the rows, swizzled K-major
+//                 layout) into a ring of shared-memory stages, completion on mbarriers;
+//   warp 1        TMEM owner (alloc / dealloc of two accumulator buffers) and MMA issuer:
+//                 4 or 8 MMAs per super-tile into one of the buffers, then tcgen05.commit to
+//                 free the stage and to hand the buffer to the epilogue;
+//   warps 2..5    epilogue: warp w reads TMEM lanes 32 * (w % 4) .. + 31 (tcgen05.ld), so
+//                 each thread owns one row = one rotated block, and does the amax, scale,
+//                 E2M1 rounding, packing and stores of that block in its registers.
+// H_b is written into shared memory once per CTA, in the same swizzled layout.
+// Every wait is bounded in time; a wait that runs out records kStatusTimeout, and the CTA
+// lets its issued copies and MMAs land before it frees TMEM and leaves.
+#pragma once
+
+#include <cuda.h>
+
+#include <cstdint>
+
+#include "fp4q_device.cuh"
+#include "fp4q_kernels.cuh"
+
+namespace fp4q {
+
+template <int FMT, int B, int RULE, bool DUMP>
+struct MmaConfig {
+  static constexpr int kFmt = FMT;
+  static constexpr int kBlock = B;
+  static constexpr int kRule = RULE;
+  static constexpr bool kDump = DUMP;
+  static constexpr int kGroup = FMT == kMX ? 32 : 16;
+  static_assert(B >= 16 && B >= kGroup && B <= 128, "one block holds whole groups");
+  static constexpr int kKB = B > 64 ? 64 : B;        // K elements per swizzled row (one TMA box row)
+  static constexpr int kRB = 2 * kKB;                // bytes per swizzled row
+  static constexpr int kHalves = B / kKB;            // K-halves (2 for b = 128)
+  static constexpr uint32_t kLayout = kRB == 32 ? 6u : kRB == 64 ? 4u : 2u;   // SW32 / SW64 / SW128
+  static constexpr int kSwzBits = kRB == 32 ? 1 : kRB == 64 ? 2 : 3;
+  // A super-tile is kSuperCols TMEM columns of 128 rows: 64 columns (8192 elements, 16 KB) for
+  // b <= 64, 128 columns (16384 elements, 32 KB) for b = 128.
+  static constexpr int kSuperCols = B >= 128 ? 128 : 64;
+  static constexpr int kRowTiles = kSuperCols / B;   // row-tiles of 128 rows per super-tile
+  static constexpr int kRowsPerTile = 128 * kRowTiles;
+  static constexpr int kStageBytes = kSuperCols * 256;
+  static constexpr int kStages = B >= 128 ? 2 : 4;
+  static constexpr int kHBytes = B * B * 2;
+  // TMA boxes per stage: up to 256 rows of kKB elements
+  static constexpr int kBoxRows = B >= 128 ? 128 : (kRowsPerTile < 256 ? kRowsPerTile : 256);
+  static constexpr int kBoxes = B >= 128 ? 2 : kRowsPerTile / kBoxRows;
+  static constexpr int kBoxBytes = kBoxRows * kRB;
+  static constexpr int kThreads = 192;
+  static constexpr int kTmemCols = 2 * kSuperCols;   // two accumulator buffers
+  static constexpr float kC = inv_sqrt_block(B);
+  // shared memory: [align pad][stages][H][barriers]
+  static constexpr int kBarOffset = kStages * kStageBytes + kHBytes;
+  static constexpr int kSmemBytes = 1024 + kBarOffset + 128;
+  static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(B >> 3) << 17) |
+                                     (static_cast<uint32_t>(128 >> 4) << 24);
+};
+
+struct MmaArgs {
+  int64_t n_rows;          // R = M*K / b
+  int64_t n_super;         // super-tiles
+  uint8_t* codes;
+  uint8_t* scales;
+  float* tensor_scale;
+  const float* partials;
+  int n_partials;
+  float* y_dump;
+};
+
+// Offset of byte `off` inside a swizzled K-major tile (rows of 32 / 64 / 128 bytes): the
+// 16-byte chunk index is XORed with the row bits above it, as the TMA swizzle modes lay
+// them out (and as the MMA descriptors' layout types read them).
+template <int BITS>
+__device__ __forceinline__ uint32_t swizzle_off(uint32_t off) {
+  return off ^ (((off >> 7) & ((1u << BITS) - 1u)) << 4);
+}
+
+__device__ __forceinline__ uint64_t umma_smem_desc(uint32_t addr, uint32_t sbo_bytes, uint32_t layout) {
+  return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
+         (static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32) | (static_cast<uint64_t>(1) << 46) |
+         (static_cast<uint64_t>(layout) << 61);
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(map), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(tmem_d),
+      "l"(da), "l"(db), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 16 consecutive TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Quantize one group of G rotated sums s (unnormalised, as produced by the MMA): E2M1 code
+// words (G / 8) and the scale byte.
+template <class Cfg, int G>
+__device__ __forceinline__ uint32_t quantize_group(const float (&s)[G], uint32_t (&words)[G / 8], float s_g,
+                                                   float nv_den, float nv_rden) {
+  constexpr float c = Cfg::kC;
+  f32x2 p[G / 2];
+#pragma unroll
+  for (int k = 0; k < G / 2; ++k) p[k] = f2_pack(s[2 * k], s[2 * k + 1]);
+  const float A = scale_by_inv_sqrt<Cfg::kBlock>(pairs_amax<G / 2>(p));
+  uint32_t byte;
+  if constexpr (Cfg::kFmt == kMX) {
+    byte = static_cast<uint32_t>(mx_scale_byte<Cfg::kRule>(A));
+    const float mult = c * mx_inv_scale(static_cast<int>(byte));
+    const f32x2 mm = f2_pack(mult, mult);
+#pragma unroll
+    for (int j = 0; j < G / 8; ++j) {
+      float v[8];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) f2_unpack(f2_mul(p[4 * j + t], mm), v[2 * t], v[2 * t + 1]);
+      words[j] = e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+    }
+  } else {
+    const float s_b = div_rn_markstein(A, nv_den, nv_rden);
+    byte = e4m3_encode(s_b);
+    const float S = e4m3_decode(byte) * s_g;
+    const uint32_t keep = S == 0.0f ? 0u : 0xFFFFFFFFu;
+    const float Sd = inv_sqrt_block_is_pow2(Cfg::kBlock) ? S * (1.0f / c) : S;
+    const float rd = __frcp_rn(Sd);
+    const f32x2 rd2 = f2_pack(rd, rd), nSd2 = f2_pack(-Sd, -Sd);
+#pragma unroll
+    for (int j = 0; j < G / 8; ++j) {
+      float v[8];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        f32x2 y = p[4 * j + t];
+        if constexpr (!inv_sqrt_block_is_pow2(Cfg::kBlock)) {
+          constexpr float chi = inv_sqrt_block(Cfg::kBlock), clo = inv_sqrt_block_lo(Cfg::kBlock);
+          y = f2_fma(y, f2_pack(chi, chi), f2_mul(y, f2_pack(clo, clo)));
+        }
+        const f32x2 q0 = f2_mul(y, rd2);
+        const f32x2 rem = f2_fma(q0, nSd2, y);
+        f2_unpack(f2_fma(rem, rd2, q0), v[2 * t], v[2 * t + 1]);
+      }
+      words[j] = e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]) & keep;
+    }
+  }
+  return byte;
+}
+
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::kThreads, 2)
+    rotate_quantize_mma_kernel(const __grid_constant__ CUtensorMap xmap, MmaArgs a) {
+  constexpr int B = Cfg::kBlock, G = Cfg::kGroup, S = Cfg::kStages;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ uint32_t s_tmem_base;
+  __shared__ float s_tensor_scale;
+  pdl_launch_dependents();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  const uint32_t stage0 = smem_addr(smem);
+  const uint32_t hbase = stage0 + S * Cfg::kStageBytes;
+  const uint32_t bars = stage0 + Cfg::kBarOffset;
+  auto full_bar = [&](int s) { return bars + 8u * s; };
+  auto empty_bar = [&](int s) { return bars + 8u * (S + s); };
+  auto tfull_bar = [&](int d) { return bars + 8u * (2 * S + d); };
+  auto tempty_bar = [&](int d) { return bars + 8u * (2 * S + 2 + d); };
+
+  // H_b, K-major, swizzled like the activation tiles: row n holds H[n][0..b) (H is symmetric)
+  uint8_t* hs = smem + S * Cfg::kStageBytes;
+  for (int i = tid; i < B * B; i += Cfg::kThreads) {
+    const int n = i / B, k = i % B;
+    const int h = k / Cfg::kKB, kk = k % Cfg::kKB;
+    const uint32_t off = h * (B * Cfg::kRB) + swizzle_off<Cfg::kSwzBits>(n * Cfg::kRB + kk * 2);
+    *reinterpret_cast<uint16_t*>(hs + off) = (__popc(n & k) & 1) ? 0xBF80u : 0x3F80u;   // bf16 -1 / +1
+  }
+  fence_proxy_async_smem();
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int d = 0; d < 2; ++d) {
+      mbar_init(tfull_bar(d), 1);
+      mbar_init(tempty_bar(d), 4);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&s_tmem_base)),
+                 "r"(Cfg::kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  // everything below may touch memory written by the kernels this one depends on
+  pdl_wait();
+  float s_g = 1.0f;
+  if constexpr (Cfg::kFmt == kNV) {
+    if (warp == 2) {
+      if constexpr (Cfg::kRule == kRuleNvDynamic) {
+        float m = 0.0f;
+        for (int i = lane; i < a.n_partials; i += 32) m = fmaxf(m, a.partials[i]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        if (lane == 0) {
+          const float sg = m == 0.0f ? 1.0f : __fdiv_rn(m, 2688.0f);
+          s_tensor_scale = sg;
+          if (blockIdx.x == 0) *a.tensor_scale = sg;
+        }
+      } else {
+        if (lane == 0) s_tensor_scale = *a.tensor_scale;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if constexpr (Cfg::kFmt == kNV) s_g = s_tensor_scale;
+  const uint32_t tmem_base = s_tmem_base;
+  const int64_t n_super = a.n_super;
+
+  if (warp == 0) {
+    // ---------------- producer
+    if (lane == 0) {
+      int64_t i = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < n_super; t += gridDim.x, ++i) {
+        const int s = static_cast<int>(i % S);
+        const uint32_t ph = static_cast<uint32_t>((i / S) & 1);
+        if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u)) {
+          ok = false;
+          break;
+        }
+        const int64_t row0 = t * Cfg::kRowsPerTile;
+        const uint32_t dst = stage0 + s * Cfg::kStageBytes;
+        if constexpr (B >= 128) {
+          mbar_arrive_expect_tx(full_bar(s), 2u * Cfg::kBoxBytes);
+          tma_load_2d(dst, &xmap, 0, static_cast<int>(row0), full_bar(s));
+          tma_load_2d(dst + Cfg::kBoxBytes, &xmap, 64, static_cast<int>(row0), full_bar(s));
+        } else {
+          int nb = 0;
+#pragma unroll
+          for (int k = 0; k < Cfg::kBoxes; ++k) nb += (row0 + k * Cfg::kBoxRows < a.n_rows) ? 1 : 0;
+          mbar_arrive_expect_tx(full_bar(s), static_cast<uint32_t>(nb) * Cfg::kBoxBytes);
+#pragma unroll
+          for (int k = 0; k < Cfg::kBoxes; ++k)
+            if (row0 + k * Cfg::kBoxRows < a.n_rows)
+              tma_load_2d(dst + k * Cfg::kBoxBytes, &xmap, 0, static_cast<int>(row0 + k * Cfg::kBoxRows), full_bar(s));
+        }
+      }
+      // let every issued copy land before the CTA can leave
+      const int64_t issued = i;
+      for (int64_t j = (issued > S ? issued - S : 0); j < issued; ++j)
+        mbar_wait_bounded(full_bar(static_cast<int>(j % S)), static_cast<uint32_t>((j / S) & 1));
+      (void)ok;
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      int64_t i = 0;
+      for (int64_t t = blockIdx.x; t < n_super; t += gridDim.x, ++i) {
+        const int s = static_cast<int>(i % S);
+        const uint32_t ph = static_cast<uint32_t>((i / S) & 1);
+        const int d = static_cast<int>(i & 1);
+        const uint32_t dph = static_cast<uint32_t>((i >> 1) & 1);
+        if (!mbar_wait_bounded(full_bar(s), ph)) break;
+        if (!mbar_wait_bounded(tempty_bar(d), dph ^ 1u)) break;
+        tc_fence_after();
+        const uint32_t a0 = stage0 + s * Cfg::kStageBytes;
+        const uint32_t dcol = tmem_base + d * Cfg::kSuperCols;
+#pragma unroll
+        for (int j = 0; j < Cfg::kRowTiles; ++j) {
+#pragma unroll
+          for (int k = 0; k < B / 16; ++k) {
+            const int h = (16 * k) / Cfg::kKB, kk = (16 * k) % Cfg::kKB;
+            const uint32_t aa = a0 + j * (128 * Cfg::kRB) + h * (128 * Cfg::kRB) + kk * 2;
+            const uint32_t ha = hbase + h * (B * Cfg::kRB) + kk * 2;
+            umma_bf16(dcol + j * B, umma_smem_desc(aa, 8 * Cfg::kRB, Cfg::kLayout),
+                      umma_smem_desc(ha, 8 * Cfg::kRB, Cfg::kLayout), Cfg::kIdesc, k > 0 ? 1u : 0u);
+          }
+        }
+        umma_commit(empty_bar(s));
+        umma_commit(tfull_bar(d));
+      }
+      // the last commits must have landed before TMEM is freed
+      if (i > 0) {
+        const int64_t j = i - 1;
+        mbar_wait_bounded(tfull_bar(static_cast<int>(j & 1)), static_cast<uint32_t>((j >> 1) & 1));
+      }
+    }
+  } else {
+    // ---------------- epilogue: warps 2..5, TMEM lane quarter warp % 4
+    const int quarter = warp & 3;
+    const int lane_row = 32 * quarter + lane;
+    const float nv_den = 6.0f * s_g;
+    const float nv_rden = __frcp_rn(nv_den);
+    int64_t i = 0;
+    for (int64_t t = blockIdx.x; t < n_super; t += gridDim.x, ++i) {
+      const int d = static_cast<int>(i & 1);
+      const uint32_t dph = static_cast<uint32_t>((i >> 1) & 1);
+      const bool mine = mbar_wait_bounded(tfull_bar(d), dph);
+      if (!__all_sync(0xFFFFFFFFu, mine)) break;
+      tc_fence_after();
+      const uint32_t tq = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + d * Cfg::kSuperCols;
+      constexpr int NG = B / G;
+      uint32_t words[B / 8];
+      uint32_t sbytes[NG];
+#pragma unroll
+      for (int c0 = 0; c0 < Cfg::kSuperCols; c0 += 64) {
+        // 64 columns of this lane: 64 / b whole blocks (b <= 64) or half a block (b = 128)
+        float v[64];
+#pragma unroll
+        for (int c16 = 0; c16 < 4; ++c16) {
+          float w16[16];
+          tmem_ld16(tq + c0 + 16 * c16, w16);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[16 * c16 + e] = w16[e];
+        }
+        tmem_wait_ld();
+#pragma unroll
+        for (int gq = 0; gq < 64 / G; ++gq) {
+          const int col = c0 + gq * G;                 // column within the super-tile
+          const int j = col / B;                       // row-tile = block of this lane
+          const int q = (col % B) / G;                 // group within the block
+          const int64_t row = t * Cfg::kRowsPerTile + j * 128 + lane_row;
+          float gv[G];
+#pragma unroll
+          for (int e = 0; e < G; ++e) gv[e] = v[gq * G + e];
+          uint32_t gw[G / 8];
+          sbytes[q] = quantize_group<Cfg, G>(gv, gw, s_g, nv_den, nv_rden);
+#pragma unroll
+          for (int e = 0; e < G / 8; ++e) words[q * (G / 8) + e] = gw[e];
+          if constexpr (Cfg::kDump) {
+            if (row < a.n_rows) {
+              float* yp = a.y_dump + row * B + q * G;
+#pragma unroll
+              for (int e = 0; e < G; e += 4)
+                *reinterpret_cast<float4*>(yp + e) =
+                    make_float4(scale_by_inv_sqrt<B>(gv[e]), scale_by_inv_sqrt<B>(gv[e + 1]),
+                                scale_by_inv_sqrt<B>(gv[e + 2]), scale_by_inv_sqrt<B>(gv[e + 3]));
+            }
+          }
+          if (q == NG - 1 && row < a.n_rows) {         // the block is complete: store it
+            uint8_t* cp = a.codes + row * (B / 2);
+            if constexpr (B == 16) {
+              stg64(cp, words[0], words[1]);
+            } else {
+#pragma unroll
+              for (int k = 0; k < B / 32; ++k)
+                stg128(cp + 16 * k, words[4 * k], words[4 * k + 1], words[4 * k + 2], words[4 * k + 3]);
+            }
+            uint8_t* sp = a.scales + row * NG;
+            if constexpr (NG == 1) {
+              *sp = static_cast<uint8_t>(sbytes[0]);
+            } else if constexpr (NG == 2) {
+              *reinterpret_cast<uint16_t*>(sp) = static_cast<uint16_t>(sbytes[0] | (sbytes[1] << 8));
+            } else if constexpr (NG == 4) {
+              *reinterpret_cast<uint32_t*>(sp) = sbytes[0] | (sbytes[1] << 8) | (sbytes[2] << 16) | (sbytes[3] << 24);
+            } else {
+              stg64(sp, sbytes[0] | (sbytes[1] << 8) | (sbytes[2] << 16) | (sbytes[3] << 24),
+                    sbytes[4] | (sbytes[5] << 8) | (sbytes[6] << 16) | (sbytes[7] << 24));
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(d));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(Cfg::kTmemCols)
+                 : "memory");
+  }
+}
+
+}  // namespace fp4q

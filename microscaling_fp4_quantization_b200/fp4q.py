@@ -23,6 +23,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 FP4Q_OK, FP4Q_ERR_ARG, FP4Q_ERR_SHAPE, FP4Q_ERR_ALIGN, FP4Q_ERR_UNSUPPORTED, FP4Q_ERR_CUDA, FP4Q_ERR_TIMEOUT = range(7)
 FP4Q_MXFP4, FP4Q_NVFP4 = 0, 1
+FP4Q_KERNEL_AUTO, FP4Q_KERNEL_BUTTERFLY, FP4Q_KERNEL_TENSOR_CORE = 0, 1, 2
 (FP4Q_SCALE_FLOOR_OCP, FP4Q_SCALE_CEIL_NOCLIP, FP4Q_SCALE_OAS,
  FP4Q_SCALE_NV_STATIC, FP4Q_SCALE_NV_DYNAMIC) = range(5)
 
@@ -33,6 +34,7 @@ _int = ctypes.c_int
 _SIGS = {
     "fp4q_plan_create": (_int, [ctypes.POINTER(_vp), _int, _int, _int, _int]),
     "fp4q_plan_destroy": (_int, [_vp]),
+    "fp4q_plan_set_kernel": (_int, [_vp, _int]),
     "fp4q_rotate_quantize": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp]),
     "fp4q_rotate_quantize_dump": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
     "fp4q_amax": (_int, [_vp, _vp, _i64, _i64, _vp, _vp]),
@@ -88,6 +90,7 @@ class Plan:
     def __init__(self, handle: int, fmt: int, group: int, block: int, rule: int):
         self.handle = handle
         self.fmt, self.group, self.block, self.rule = fmt, group, block, rule
+        self.kernel = FP4Q_KERNEL_AUTO
 
     def __del__(self):
         h, self.handle = getattr(self, "handle", None), None
@@ -108,6 +111,11 @@ def fp4q_plan_create(fmt: int, group: int, hadamard_block: int, scale_rule: int)
     h = _vp()
     _check(_lib.fp4q_plan_create(ctypes.byref(h), fmt, group, hadamard_block, scale_rule), "fp4q_plan_create")
     return Plan(h.value, fmt, group, hadamard_block, scale_rule)
+
+
+def fp4q_plan_set_kernel(plan: Plan, kernel: int) -> None:
+    _check(_lib.fp4q_plan_set_kernel(plan.handle, kernel), "fp4q_plan_set_kernel")
+    plan.kernel = kernel
 
 
 def fp4q_plan_destroy(plan: Plan) -> None:

@@ -56,6 +56,16 @@ def test_plan_validation_without_gpu(F):
     assert F.raw_call("fp4q_plan_destroy", None) == F.FP4Q_OK
 
 
+def test_kernel_selection_without_gpu(F):
+    p = F.fp4q_plan_create(F.FP4Q_MXFP4, 32, 1, F.FP4Q_SCALE_FLOOR_OCP)
+    assert F.raw_call("fp4q_plan_set_kernel", p.handle, F.FP4Q_KERNEL_TENSOR_CORE) == F.FP4Q_ERR_UNSUPPORTED
+    assert F.raw_call("fp4q_plan_set_kernel", p.handle, 7) == F.FP4Q_ERR_ARG
+    assert F.raw_call("fp4q_plan_set_kernel", None, 0) == F.FP4Q_ERR_ARG
+    q = F.fp4q_plan_create(F.FP4Q_MXFP4, 32, 128, F.FP4Q_SCALE_CEIL_NOCLIP)
+    for k in (F.FP4Q_KERNEL_TENSOR_CORE, F.FP4Q_KERNEL_BUTTERFLY, F.FP4Q_KERNEL_AUTO):
+        F.fp4q_plan_set_kernel(q, k)
+
+
 def test_call_validation_without_gpu(F):
     p = F.fp4q_plan_create(F.FP4Q_MXFP4, 32, 128, F.FP4Q_SCALE_FLOOR_OCP)
     rq = lambda *a: F.raw_call("fp4q_rotate_quantize", *a)

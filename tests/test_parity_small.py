@@ -49,11 +49,22 @@ def F(cuda_device):
     return fp4q
 
 
-@pytest.mark.parametrize("combo", COMBOS, ids=[combo_id(c) for c in COMBOS])
-def test_rotate_quantize_matches_oracle(F, combo):
+def mma_capable(combo):
+    fmt, g, b, rule = combo
+    return b >= 16 and b >= g
+
+
+KERNEL_CASES = ([(c, 1) for c in COMBOS] + [(c, 2) for c in COMBOS if mma_capable(c)])
+
+
+@pytest.mark.parametrize("combo,kernel", KERNEL_CASES,
+                         ids=[combo_id(c) + ("-tc" if k == 2 else "-bf") for c, k in KERNEL_CASES])
+def test_rotate_quantize_matches_oracle(F, combo, kernel):
+    """kernel 1: the butterfly kernel; 2: the tensor-core kernel."""
     import gpu_util as gu
     fmt, g, b, rule = combo
     plan = F.fp4q_plan_create(fmt, g, b, rule)
+    F.fp4q_plan_set_kernel(plan, kernel)
     unit = max(g, b)
     for i, (M, K) in enumerate(shapes_for(unit)):
         x = make_input(M, K, seed=100 * b + 10 * rule + i)

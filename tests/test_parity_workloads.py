@@ -27,9 +27,9 @@ def sample_rows(M, n=192, seed=0):
 
 
 def check_workload(F, w, rows=None, x=None):
+    """Both kernels (butterfly and tensor core) against the oracle on the same input."""
     import gpu_util as gu
     x = w.generate() if x is None else x
-    plan = F.fp4q_plan_create(w.fmt, w.group, w.block, w.rule)
     ts = None
     if w.fmt == o.NVFP4:
         ts = o.nv_tensor_scale(o.rotated_amax(x, w.block))
@@ -37,13 +37,18 @@ def check_workload(F, w, rows=None, x=None):
         nv_plan = F.fp4q_plan_create(o.NVFP4, 16, w.block, o.SCALE_NV_STATIC)
         ours = gu.run_amax(F, nv_plan, x)
         assert abs(float(ours) - float(ts)) <= 2.5e-7 * float(ts), (ours, ts)
-    out = gu.run_rotate_quantize(F, plan, x, tensor_scale=ts, dump=True, rows=rows)
     xs = x if rows is None else x[rows]
     res = o.rotate_quantize(xs, w.fmt, w.group, w.block, w.rule, tensor_scale=ts)
-    rep = assert_parity(res, out["codes"], out["scales"], w.name)
-    err = rotated_value_error(out["y"], res)
-    assert err <= 1e-5, (w.name, err)
-    return rep, x
+    reps = {}
+    for kernel in (F.FP4Q_KERNEL_BUTTERFLY, F.FP4Q_KERNEL_TENSOR_CORE):
+        plan = F.fp4q_plan_create(w.fmt, w.group, w.block, w.rule)
+        F.fp4q_plan_set_kernel(plan, kernel)
+        out = gu.run_rotate_quantize(F, plan, x, tensor_scale=ts, dump=True, rows=rows)
+        reps[kernel] = assert_parity(res, out["codes"], out["scales"], f"{w.name} kernel {kernel}")
+        err = rotated_value_error(out["y"], res)
+        assert err <= 1e-5, (w.name, kernel, err)
+        del out
+    return reps, x
 
 
 def test_small_mx(F):

@@ -6,8 +6,9 @@ allocate after start-up), so they cannot create the dynamic-scale plan, which al
 partial-maximum array.  fp4q_rotate_quantize_nvfp4_dynamic_noalloc keeps that array in a
 fixed buffer inside the library instead.  This test calls it twice in a row through the C
 ABI, on different inputs, and requires the same codes, scales and tensor scale as
-fp4q_rotate_quantize with an FP4Q_SCALE_NV_DYNAMIC plan (exact equality, inside the parity
-tolerance the other tests use).  This file is collected last on purpose."""
+fp4q_rotate_quantize with an FP4Q_SCALE_NV_DYNAMIC plan on the same (butterfly) kernel —
+exact equality, inside the parity tolerance the other tests use.  This file is collected
+last on purpose."""
 
 import numpy as np
 import pytest
@@ -22,6 +23,7 @@ pytestmark = pytest.mark.gpu
 def test_noalloc_matches_planned_entry_point(cuda_device, b):
     from microscaling_fp4_quantization_b200 import fp4q as F
     plan = F.fp4q_plan_create(F.FP4Q_NVFP4, 16, b, F.FP4Q_SCALE_NV_DYNAMIC)
+    F.fp4q_plan_set_kernel(plan, F.FP4Q_KERNEL_BUTTERFLY)
     shapes = [(512, 4096), (37, 6 * max(b, 32))]
     for call, (M, K) in enumerate(shapes):             # two calls in a row, different inputs
         w = W.Workload(f"noalloc_{call}", M, K, 40 + call, "normal", max(1, K // 200), 50.0,
