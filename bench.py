@@ -43,10 +43,11 @@ KERNELS = {"auto": 0, "butterfly": 1, "tensor_core": 2}
 
 
 def kernel_name(w, requested: str) -> str:
-    """The kernel a plan with this request runs (auto: tensor core when b >= 16 and b >= g)."""
+    """The kernel a plan with this request runs (auto: tensor core when b >= 16, b >= g and
+    M*K >= 2^22)."""
     if requested != "auto":
         return requested
-    return "tensor_core" if (w.block >= 16 and w.block >= w.group) else "butterfly"
+    return "tensor_core" if (w.block >= 16 and w.block >= w.group and w.numel >= (1 << 22)) else "butterfly"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 SPEC_HBM_GBS = 8000.0
@@ -329,8 +330,9 @@ def run_gpu(args):
     if args.all_workloads and rank == 0:
         for ow in (W.SMALL_MX, W.MX_8K_FLOOR, W.MX_8K_CEIL, W.PREFILL_NV, W.PREFILL_MX) + W.DECODE:
             others[ow.name] = time_other(torch, F, ow, dev, stream, peak)
-            if kernel_name(ow, "auto") == "tensor_core":
-                others[ow.name + " [butterfly kernel]"] = time_other(torch, F, ow, dev, stream, peak, kernel="butterfly")
+            if ow.block >= 16 and ow.block >= ow.group:
+                alt = "butterfly" if kernel_name(ow, "auto") == "tensor_core" else "tensor_core"
+                others[ow.name + f" [{alt} kernel]"] = time_other(torch, F, ow, dev, stream, peak, kernel=alt)
 
     if rank == 0:
         cpu = cpu_baseline(w, args) if world == 1 and not args.no_cpu_baseline else None

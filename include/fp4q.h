@@ -100,7 +100,8 @@ fp4q_status fp4q_plan_create(fp4q_plan* out, int format, int group, int hadamard
 /* Which kernel a plan's rotate + quantize calls run on. */
 typedef enum {
   FP4Q_KERNEL_AUTO = 0,        /* the tensor-core kernel when every Hadamard block holds whole
-                                  scale groups (b >= 16 and b >= g), else the butterfly kernel */
+                                  scale groups (b >= 16 and b >= g) and M*K >= 2^22, else the
+                                  butterfly kernel (which starts faster on small tensors)     */
   FP4Q_KERNEL_BUTTERFLY = 1,   /* in-register fast Walsh-Hadamard butterfly on CUDA cores    */
   FP4Q_KERNEL_TENSOR_CORE = 2  /* tcgen05 MMA against H_b with TMEM accumulators            */
 } fp4q_kernel;

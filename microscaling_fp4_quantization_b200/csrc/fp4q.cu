@@ -67,6 +67,9 @@ fp4q_status kernel_info(K kernel, int smem_bytes, int threads, KernelInfo* out) 
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  // all of the unified L1 / shared storage as shared memory: these kernels stage through it
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(carveout)");
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ki.ctas_per_sm, kernel, threads, smem_bytes);
   if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
   if (ki.ctas_per_sm < 1) ki.ctas_per_sm = 1;
@@ -155,6 +158,7 @@ fp4q_status launch_mma(const uint16_t* x, int64_t n_elems, const RQArgs& ra, cud
   fp4q_status st = encode_fn(&enc);
   if (st != FP4Q_OK) return st;
   MmaArgs a;
+  a.x = x;
   a.n_rows = n_elems / Cfg::kBlock;
   a.n_super = (a.n_rows + Cfg::kRowsPerTile - 1) / Cfg::kRowsPerTile;
   a.codes = ra.codes;
@@ -182,8 +186,10 @@ fp4q_status launch_mma(const uint16_t* x, int64_t n_elems, const RQArgs& ra, cud
   KernelInfo ki;
   st = kernel_info(kernel, Cfg::kSmemBytes, Cfg::kThreads, &ki);
   if (st != FP4Q_OK) return st;
-  int per_sm = ki.ctas_per_sm;
-  if (per_sm > 512 / Cfg::kTmemCols) per_sm = 512 / Cfg::kTmemCols;   // tensor memory: 512 columns per SM
+  // CTAs per SM from measurement (the kernel's CTAs are independent, so a CTA that does not
+  // fit next to the others simply starts later); tensor memory holds 512 columns per SM
+  int per_sm = Cfg::kCtasPerSm;
+  if (per_sm > 512 / Cfg::kTmemCols) per_sm = 512 / Cfg::kTmemCols;
   int64_t ctas = static_cast<int64_t>(ki.sm_count) * per_sm;
   if (ctas > a.n_super) ctas = a.n_super;
   cudaError_t e = launch_pdl(kernel, dim3(static_cast<unsigned>(ctas)), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream,
@@ -192,11 +198,15 @@ fp4q_status launch_mma(const uint16_t* x, int64_t n_elems, const RQArgs& ra, cud
   return FP4Q_OK;
 }
 
-// Whether the tensor-core kernel serves this plan.
+// Whether the tensor-core kernel serves this plan.  AUTO takes it for tensors of at least
+// kMmaMinElems elements: below that its fixed start-up (TMEM allocation, H_b, filling a
+// three-stage pipeline) costs more than the butterfly kernel's extra instructions.
+constexpr int64_t kMmaMinElems = int64_t(1) << 22;
 bool mma_capable(fp4q_plan p) { return p->block >= 16 && p->block >= p->group; }
-bool use_mma(fp4q_plan p) {
+bool use_mma(fp4q_plan p, int64_t n_elems) {
   if (!mma_capable(p)) return false;
-  return p->kernel == FP4Q_KERNEL_AUTO || p->kernel == FP4Q_KERNEL_TENSOR_CORE;
+  if (p->kernel == FP4Q_KERNEL_TENSOR_CORE) return true;
+  return p->kernel == FP4Q_KERNEL_AUTO && n_elems >= kMmaMinElems;
 }
 
 template <int B, int MINU>
@@ -266,7 +276,7 @@ fp4q_status rotate_quantize_impl(fp4q_plan p, const void* x, int64_t M, int64_t 
     st = launch_amax(p, a.x, n, s);
     if (st != FP4Q_OK) return st;
   }
-  if (use_mma(p)) {
+  if (use_mma(p, n)) {
     return with_block(p->block, [&]<int B>() -> fp4q_status {
       if constexpr (B >= 16) {
         if (p->format == FP4Q_MXFP4) {

@@ -9,13 +9,15 @@
 // 128 rows, 16 KB of input) or 128 columns (b = 128, 32 KB).
 // Roles, per CTA of 6 warps:
 //   warp 0        producer: TMA tensor loads (2-D map over the rows, swizzled K-major
-//                 layout) into a ring of shared-memory stages, completion on mbarriers;
+//                 layout; for b <= 32 one contiguous bulk copy per stage) into a ring of
+//                 shared-memory stages, completion on mbarriers;
 //   warp 1        TMEM owner (alloc / dealloc of two accumulator buffers) and MMA issuer:
 //                 4 or 8 MMAs per super-tile into one of the buffers, then tcgen05.commit to
 //                 free the stage and to hand the buffer to the epilogue;
-//   warps 2..5    epilogue: warp w reads TMEM lanes 32 * (w % 4) .. + 31 (tcgen05.ld), so
-//                 each thread owns one row = one rotated block, and does the amax, scale,
-//                 E2M1 rounding, packing and stores of that block in its registers.
+//   warps 2..     epilogue (8 or 16 warps): warp w reads TMEM lanes 32 * (w % 4) .. + 31
+//                 (tcgen05.ld), one slice of the super-tile's columns each, so each thread owns
+//                 one row (one rotated block, or a part of one) and does the amax, scale, E2M1
+//                 rounding, packing and stores of it in its registers.
 // H_b is written into shared memory once per CTA, in the same swizzled layout.
 // Every wait is bounded in time; a wait that runs out records kStatusTimeout, and the CTA
 // lets its issued copies and MMAs land before it frees TMEM and leaves.
@@ -43,29 +45,45 @@ struct MmaConfig {
   static constexpr int kHalves = B / kKB;            // K-halves (2 for b = 128)
   static constexpr uint32_t kLayout = kRB == 32 ? 6u : kRB == 64 ? 4u : 2u;   // SW32 / SW64 / SW128
   static constexpr int kSwzBits = kRB == 32 ? 1 : kRB == 64 ? 2 : 3;
-  // A super-tile is kSuperCols TMEM columns of 128 rows: 64 columns (8192 elements, 16 KB) for
-  // b <= 64, 128 columns (16384 elements, 32 KB) for b = 128.
-  static constexpr int kSuperCols = B >= 128 ? 128 : 64;
+  // A super-tile is 128 TMEM columns of 128 rows: 16384 elements, 32 KB of input.
+  static constexpr int kSuperCols = 128;
   static constexpr int kRowTiles = kSuperCols / B;   // row-tiles of 128 rows per super-tile
   static constexpr int kRowsPerTile = 128 * kRowTiles;
   static constexpr int kStageBytes = kSuperCols * 256;
-  static constexpr int kStages = B >= 128 ? 2 : 4;
+  static constexpr int kStages = B >= 128 ? 2 : 3;
   static constexpr int kHBytes = B * B * 2;
   // TMA boxes per stage: up to 256 rows of kKB elements
   static constexpr int kBoxRows = B >= 128 ? 128 : (kRowsPerTile < 256 ? kRowsPerTile : 256);
   static constexpr int kBoxes = B >= 128 ? 2 : kRowsPerTile / kBoxRows;
   static constexpr int kBoxBytes = kBoxRows * kRB;
-  static constexpr int kThreads = 192;
+  // Epilogue warps: kSlices per TMEM lane quarter, each taking kEpiCols of the super-tile's
+  // columns.  NVFP4 (the heavier per-element work) gets four per quarter for b <= 64, the others
+  // two.  CTAs per SM: 1 for NVFP4 b <= 64 (18 warps), else 2 (tensor memory allows two).
+  static constexpr int kSlices = (FMT == kNV && B <= 64) ? 4 : 2;
+  static constexpr int kEpiWarps = 4 * kSlices;
+  static constexpr int kEpiCols = kSuperCols / kSlices;   // columns per epilogue warp
+  static constexpr int kCtasPerSm = (FMT == kNV && B <= 64) ? 1 : 2;
+  static constexpr int kThreads = 32 * (2 + kEpiWarps);
   static constexpr int kTmemCols = 2 * kSuperCols;   // two accumulator buffers
   static constexpr float kC = inv_sqrt_block(B);
   // shared memory: [align pad][stages][H][barriers]
-  static constexpr int kBarOffset = kStages * kStageBytes + kHBytes;
+  static constexpr int kTableBytes = FMT == kNV ? 256 * 8 : 0;   // NV: divisor and reciprocal per E4M3 byte
+  // b <= 32: rows of 32 / 64 bytes make TMA tensor boxes slow, so a stage is one contiguous bulk
+  // copy, left unswizzled.  Read through the swizzled descriptor, row r's K index comes out
+  // XORed with 8 * t(r) (t = (r >> 2) & 1 for 32-byte rows, (r >> 1) & 3 for 64-byte rows), which
+  // turns into a sign flip of output column n when popcount(n & 8 t(r)) is odd (H[k ^ T][n] =
+  // (-1)^popcount(T & n) H[k][n]); the epilogue undoes it on the packed codes.
+  static constexpr bool kBulk = B <= 32;
+  static constexpr int kFlipShift = kRB == 32 ? 2 : 1;
+  static constexpr int kFlipMask = kRB == 32 ? 1 : 3;
+  static constexpr int kBarOffset = kStages * kStageBytes + kHBytes + kTableBytes;
   static constexpr int kSmemBytes = 1024 + kBarOffset + 128;
   static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(B >> 3) << 17) |
                                      (static_cast<uint32_t>(128 >> 4) << 24);
 };
 
 struct MmaArgs {
+  const uint16_t* x;       // bf16 [R][b] (the bulk-copy loads)
   int64_t n_rows;          // R = M*K / b
   int64_t n_super;         // super-tiles
   uint8_t* codes;
@@ -133,7 +151,7 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 // Quantize one group of G rotated sums s (unnormalised, as produced by the MMA): E2M1 code
 // words (G / 8) and the scale byte.
 template <class Cfg, int G>
-__device__ __forceinline__ uint32_t quantize_group(const float (&s)[G], uint32_t (&words)[G / 8], float s_g,
+__device__ __forceinline__ uint32_t quantize_group(const float (&s)[G], uint32_t (&words)[G / 8], const float2* nv_tab,
                                                    float nv_den, float nv_rden) {
   constexpr float c = Cfg::kC;
   f32x2 p[G / 2];
@@ -155,10 +173,9 @@ __device__ __forceinline__ uint32_t quantize_group(const float (&s)[G], uint32_t
   } else {
     const float s_b = div_rn_markstein(A, nv_den, nv_rden);
     byte = e4m3_encode(s_b);
-    const float S = e4m3_decode(byte) * s_g;
-    const uint32_t keep = S == 0.0f ? 0u : 0xFFFFFFFFu;
-    const float Sd = inv_sqrt_block_is_pow2(Cfg::kBlock) ? S * (1.0f / c) : S;
-    const float rd = __frcp_rn(Sd);
+    const uint32_t keep = byte == 0u ? 0u : 0xFFFFFFFFu;   // E4M3 byte 0 is the only zero scale
+    const float2 tab = nv_tab[byte];                        // divisor and its RN reciprocal
+    const float Sd = tab.x, rd = tab.y;
     const f32x2 rd2 = f2_pack(rd, rd), nSd2 = f2_pack(-Sd, -Sd);
 #pragma unroll
     for (int j = 0; j < G / 8; ++j) {
@@ -214,7 +231,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 2)
     }
     for (int d = 0; d < 2; ++d) {
       mbar_init(tfull_bar(d), 1);
-      mbar_init(tempty_bar(d), 4);
+      mbar_init(tempty_bar(d), Cfg::kEpiWarps);
     }
     fence_mbar_init();
   }
@@ -224,36 +241,17 @@ __global__ void __launch_bounds__(Cfg::kThreads, 2)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  // everything below may touch memory written by the kernels this one depends on
-  pdl_wait();
-  float s_g = 1.0f;
-  if constexpr (Cfg::kFmt == kNV) {
-    if (warp == 2) {
-      if constexpr (Cfg::kRule == kRuleNvDynamic) {
-        float m = 0.0f;
-        for (int i = lane; i < a.n_partials; i += 32) m = fmaxf(m, a.partials[i]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-        if (lane == 0) {
-          const float sg = m == 0.0f ? 1.0f : __fdiv_rn(m, 2688.0f);
-          s_tensor_scale = sg;
-          if (blockIdx.x == 0) *a.tensor_scale = sg;
-        }
-      } else {
-        if (lane == 0) s_tensor_scale = *a.tensor_scale;
-      }
-    }
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if constexpr (Cfg::kFmt == kNV) s_g = s_tensor_scale;
   const uint32_t tmem_base = s_tmem_base;
   const int64_t n_super = a.n_super;
+  float2* nv_tab = reinterpret_cast<float2*>(smem + S * Cfg::kStageBytes + Cfg::kHBytes);
 
   if (warp == 0) {
     // ---------------- producer
     if (lane == 0) {
+      pdl_wait();   // x may come from the kernel this one depends on
       int64_t i = 0;
       bool ok = true;
       for (int64_t t = blockIdx.x; t < n_super; t += gridDim.x, ++i) {
@@ -265,7 +263,12 @@ __global__ void __launch_bounds__(Cfg::kThreads, 2)
         }
         const int64_t row0 = t * Cfg::kRowsPerTile;
         const uint32_t dst = stage0 + s * Cfg::kStageBytes;
-        if constexpr (B >= 128) {
+        if constexpr (Cfg::kBulk) {
+          const int64_t rows = (a.n_rows - row0) < Cfg::kRowsPerTile ? (a.n_rows - row0) : Cfg::kRowsPerTile;
+          const uint32_t bytes = static_cast<uint32_t>(rows) * (2 * B);
+          mbar_arrive_expect_tx(full_bar(s), bytes);
+          bulk_g2s(dst, a.x + row0 * B, bytes, full_bar(s));
+        } else if constexpr (B >= 128) {
           mbar_arrive_expect_tx(full_bar(s), 2u * Cfg::kBoxBytes);
           tma_load_2d(dst, &xmap, 0, static_cast<int>(row0), full_bar(s));
           tma_load_2d(dst + Cfg::kBoxBytes, &xmap, 64, static_cast<int>(row0), full_bar(s));
@@ -321,11 +324,46 @@ __global__ void __launch_bounds__(Cfg::kThreads, 2)
       }
     }
   } else {
-    // ---------------- epilogue: warps 2..5, TMEM lane quarter warp % 4
+    // ---------------- epilogue: warps 2.., TMEM lane quarter warp % 4, column slice (warp - 2) / 4
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;                  // slice index, 0 .. kSlices - 1
     const int lane_row = 32 * quarter + lane;
+    pdl_wait();   // the tensor scale (or the partial maxima) and the outputs belong to earlier kernels
+    float s_g = 1.0f;
+    if constexpr (Cfg::kFmt == kNV) {
+      constexpr int kEpiThreads = 32 * Cfg::kEpiWarps;
+      if (warp == 2) {
+        if constexpr (Cfg::kRule == kRuleNvDynamic) {
+          float m = 0.0f;
+          for (int i2 = lane; i2 < a.n_partials; i2 += 32) m = fmaxf(m, a.partials[i2]);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+          if (lane == 0) {
+            const float sg = m == 0.0f ? 1.0f : __fdiv_rn(m, 2688.0f);
+            s_tensor_scale = sg;
+            if (blockIdx.x == 0) *a.tensor_scale = sg;
+          }
+        } else {
+          if (lane == 0) s_tensor_scale = *a.tensor_scale;
+        }
+      }
+      asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
+      s_g = s_tensor_scale;
+      // for every E4M3 byte: the element divisor S = fp32(E4M3(byte) s_g) in the units of the
+      // butterfly sums (a power-of-two 1/sqrt(b) folded in exactly) and its RN reciprocal
+      for (int byte = tid - 64; byte < 256; byte += kEpiThreads) {
+        const float Sv = e4m3_decode(static_cast<uint32_t>(byte & 0x7F)) * s_g;
+        const float Sd = inv_sqrt_block_is_pow2(B) ? Sv * (1.0f / Cfg::kC) : Sv;
+        nv_tab[byte] = make_float2(Sd, Sd == 0.0f ? 0.0f : __frcp_rn(Sd));
+      }
+      asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
+    }
+    // bulk-copied stages: which 8-column chunks of this lane's rows come out sign-flipped
+    const int flip_t = Cfg::kBulk ? ((lane_row >> Cfg::kFlipShift) & Cfg::kFlipMask) : 0;
     const float nv_den = 6.0f * s_g;
     const float nv_rden = __frcp_rn(nv_den);
+    constexpr int EC = Cfg::kEpiCols;                 // 16, 32 or 64 columns
+    constexpr int NGW = EC / G;                        // groups per warp slice
     int64_t i = 0;
     for (int64_t t = blockIdx.x; t < n_super; t += gridDim.x, ++i) {
       const int d = static_cast<int>(i & 1);
@@ -333,71 +371,83 @@ __global__ void __launch_bounds__(Cfg::kThreads, 2)
       const bool mine = mbar_wait_bounded(tfull_bar(d), dph);
       if (!__all_sync(0xFFFFFFFFu, mine)) break;
       tc_fence_after();
-      const uint32_t tq = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + d * Cfg::kSuperCols;
-      constexpr int NG = B / G;
-      uint32_t words[B / 8];
-      uint32_t sbytes[NG];
+      const int col0 = half * EC;                      // first column of this warp's slice
+      const uint32_t tq = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + d * Cfg::kSuperCols + col0;
+      float v[EC];
 #pragma unroll
-      for (int c0 = 0; c0 < Cfg::kSuperCols; c0 += 64) {
-        // 64 columns of this lane: 64 / b whole blocks (b <= 64) or half a block (b = 128)
-        float v[64];
+      for (int c16 = 0; c16 < EC / 16; ++c16) {
+        float w16[16];
+        tmem_ld16(tq + 16 * c16, w16);
 #pragma unroll
-        for (int c16 = 0; c16 < 4; ++c16) {
-          float w16[16];
-          tmem_ld16(tq + c0 + 16 * c16, w16);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) v[16 * c16 + e] = w16[e];
-        }
-        tmem_wait_ld();
-#pragma unroll
-        for (int gq = 0; gq < 64 / G; ++gq) {
-          const int col = c0 + gq * G;                 // column within the super-tile
-          const int j = col / B;                       // row-tile = block of this lane
-          const int q = (col % B) / G;                 // group within the block
-          const int64_t row = t * Cfg::kRowsPerTile + j * 128 + lane_row;
-          float gv[G];
-#pragma unroll
-          for (int e = 0; e < G; ++e) gv[e] = v[gq * G + e];
-          uint32_t gw[G / 8];
-          sbytes[q] = quantize_group<Cfg, G>(gv, gw, s_g, nv_den, nv_rden);
-#pragma unroll
-          for (int e = 0; e < G / 8; ++e) words[q * (G / 8) + e] = gw[e];
-          if constexpr (Cfg::kDump) {
-            if (row < a.n_rows) {
-              float* yp = a.y_dump + row * B + q * G;
-#pragma unroll
-              for (int e = 0; e < G; e += 4)
-                *reinterpret_cast<float4*>(yp + e) =
-                    make_float4(scale_by_inv_sqrt<B>(gv[e]), scale_by_inv_sqrt<B>(gv[e + 1]),
-                                scale_by_inv_sqrt<B>(gv[e + 2]), scale_by_inv_sqrt<B>(gv[e + 3]));
-            }
-          }
-          if (q == NG - 1 && row < a.n_rows) {         // the block is complete: store it
-            uint8_t* cp = a.codes + row * (B / 2);
-            if constexpr (B == 16) {
-              stg64(cp, words[0], words[1]);
-            } else {
-#pragma unroll
-              for (int k = 0; k < B / 32; ++k)
-                stg128(cp + 16 * k, words[4 * k], words[4 * k + 1], words[4 * k + 2], words[4 * k + 3]);
-            }
-            uint8_t* sp = a.scales + row * NG;
-            if constexpr (NG == 1) {
-              *sp = static_cast<uint8_t>(sbytes[0]);
-            } else if constexpr (NG == 2) {
-              *reinterpret_cast<uint16_t*>(sp) = static_cast<uint16_t>(sbytes[0] | (sbytes[1] << 8));
-            } else if constexpr (NG == 4) {
-              *reinterpret_cast<uint32_t*>(sp) = sbytes[0] | (sbytes[1] << 8) | (sbytes[2] << 16) | (sbytes[3] << 24);
-            } else {
-              stg64(sp, sbytes[0] | (sbytes[1] << 8) | (sbytes[2] << 16) | (sbytes[3] << 24),
-                    sbytes[4] | (sbytes[5] << 8) | (sbytes[6] << 16) | (sbytes[7] << 24));
-            }
-          }
-        }
+        for (int e = 0; e < 16; ++e) v[16 * c16 + e] = w16[e];
       }
+      tmem_wait_ld();
+      // the accumulator buffer can be reused as soon as every epilogue warp has its slice
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty_bar(d));
+      // The slice holds whole blocks (b < EC), exactly one block (b == EC) or half of one.
+      constexpr int BW = B < EC ? B : EC;              // block elements in one slice piece
+      constexpr int PIECES = EC / BW;                  // block pieces in the slice
+#pragma unroll
+      for (int pc = 0; pc < PIECES; ++pc) {
+        const int col = col0 + pc * BW;                // column within the super-tile
+        const int j = col / B;                         // row-tile = block of this lane
+        const int off = col % B;                       // element offset inside the block
+        const int64_t row = t * Cfg::kRowsPerTile + j * 128 + lane_row;
+        uint32_t words[BW / 8];
+        uint32_t sbytes[BW / G];
+#pragma unroll
+        for (int q = 0; q < BW / G; ++q) {
+          float gv[G];
+#pragma unroll
+          for (int e = 0; e < G; ++e) gv[e] = v[pc * BW + q * G + e];
+          uint32_t gw[G / 8];
+          sbytes[q] = quantize_group<Cfg, G>(gv, gw, nv_tab, nv_den, nv_rden);
+#pragma unroll
+          for (int e = 0; e < G / 8; ++e) {
+            const int chunk = (off + q * G) / 8 + e;   // 8-column chunk inside the block
+            uint32_t w = gw[e];
+            if constexpr (Cfg::kBulk)
+              if (__popc(chunk & flip_t) & 1) w ^= 0x88888888u;
+            words[q * (G / 8) + e] = w;
+          }
+          if constexpr (Cfg::kDump) {
+            if (row < a.n_rows) {
+              float* yp = a.y_dump + row * B + off + q * G;
+#pragma unroll
+              for (int e = 0; e < G; e += 4) {
+                const int chunk = (off + q * G + e) / 8;
+                const float sg = (Cfg::kBulk && (__popc(chunk & flip_t) & 1)) ? -1.0f : 1.0f;
+                *reinterpret_cast<float4*>(yp + e) =
+                    make_float4(sg * scale_by_inv_sqrt<B>(gv[e]), sg * scale_by_inv_sqrt<B>(gv[e + 1]),
+                                sg * scale_by_inv_sqrt<B>(gv[e + 2]), sg * scale_by_inv_sqrt<B>(gv[e + 3]));
+              }
+            }
+          }
+        }
+        if (row < a.n_rows) {
+          uint8_t* cp = a.codes + row * (B / 2) + off / 2;
+          if constexpr (BW == 16) {
+            stg64(cp, words[0], words[1]);
+          } else {
+#pragma unroll
+            for (int k = 0; k < BW / 32; ++k)
+              stg128(cp + 16 * k, words[4 * k], words[4 * k + 1], words[4 * k + 2], words[4 * k + 3]);
+          }
+          uint8_t* sp = a.scales + row * (B / G) + off / G;
+          constexpr int NG = BW / G;
+          if constexpr (NG == 1) {
+            *sp = static_cast<uint8_t>(sbytes[0]);
+          } else if constexpr (NG == 2) {
+            *reinterpret_cast<uint16_t*>(sp) = static_cast<uint16_t>(sbytes[0] | (sbytes[1] << 8));
+          } else {
+            static_assert(NG == 4, "a slice piece holds 1, 2 or 4 groups");
+            *reinterpret_cast<uint32_t*>(sp) = sbytes[0] | (sbytes[1] << 8) | (sbytes[2] << 16) | (sbytes[3] << 24);
+          }
+        }
+      }
+      (void)NGW;
     }
   }
   tc_fence_before();
