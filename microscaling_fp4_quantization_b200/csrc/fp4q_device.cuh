@@ -158,6 +158,13 @@ __device__ __forceinline__ f32x2 bf16_pair_butterfly_oddneg(uint32_t w) {
   return f2_pack(s, d);
 }
 
+// max(a, b, c) in one instruction (three-input max.f32, sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // Approximate reciprocal (the hardware's rcp.approx: relative error below 2^-22).
 __device__ __forceinline__ float rcp_approx(float x) {
   float r;

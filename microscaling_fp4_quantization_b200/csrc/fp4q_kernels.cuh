@@ -208,21 +208,28 @@ __device__ __forceinline__ void load_rotate_unit(uint32_t saddr, int tau, f32x2 
   }
 }
 
-// max |value| over N pairs, as a tree for instruction-level parallelism.
+// max |value| over N pairs (N a power of two), with three-input maxima: each step folds
+// both values of one pair into a running maximum.
 template <int N>
 __device__ __forceinline__ float pairs_amax(const f32x2* p) {
-  float t[N];
+  // four independent chains for instruction-level parallelism, merged at the end
+  constexpr int C = N >= 4 ? 4 : N;
+  float m[C];
 #pragma unroll
-  for (int k = 0; k < N; ++k) {
+  for (int c = 0; c < C; ++c) {
     float lo, hi;
-    f2_unpack(p[k], lo, hi);
-    t[k] = fmaxf(fabsf(lo), fabsf(hi));
+    f2_unpack(p[c], lo, hi);
+    m[c] = fmaxf(fabsf(lo), fabsf(hi));
   }
 #pragma unroll
-  for (int s = N / 2; s >= 1; s /= 2)
-#pragma unroll
-    for (int k = 0; k < s; ++k) t[k] = fmaxf(t[k], t[k + s]);
-  return t[0];
+  for (int k = C; k < N; ++k) {
+    float lo, hi;
+    f2_unpack(p[k], lo, hi);
+    m[k % C] = fmax3(m[k % C], fabsf(lo), fabsf(hi));
+  }
+  if constexpr (C == 4) return fmax3(fmaxf(m[0], m[1]), m[2], m[3]);
+  if constexpr (C == 2) return fmaxf(m[0], m[1]);
+  return m[0];
 }
 
 // MX scale byte from the fp32 group amax A >= 0 (see fp4q.h for the rules).

@@ -58,7 +58,7 @@ struct MmaConfig {
   static constexpr int kBoxBytes = kBoxRows * kRB;
   // Epilogue warps: kSlices per TMEM lane quarter, each taking kEpiCols of the super-tile's
   // columns.  NVFP4 (the heavier per-element work) gets four per quarter for b <= 64, the others
-  // two.  CTAs per SM: 1 for NVFP4 b <= 64 (18 warps), else 2 (tensor memory allows two).
+  // two.  CTAs per SM, from measurement: 1 for NVFP4 b <= 64 (18 warps), else 2.
   static constexpr int kSlices = (FMT == kNV && B <= 64) ? 4 : 2;
   static constexpr int kEpiWarps = 4 * kSlices;
   static constexpr int kEpiCols = kSuperCols / kSlices;   // columns per epilogue warp
@@ -67,7 +67,7 @@ struct MmaConfig {
   static constexpr int kTmemCols = 2 * kSuperCols;   // two accumulator buffers
   static constexpr float kC = inv_sqrt_block(B);
   // shared memory: [align pad][stages][H][barriers]
-  static constexpr int kTableBytes = FMT == kNV ? 256 * 8 : 0;   // NV: divisor and reciprocal per E4M3 byte
+  static constexpr int kTableBytes = FMT == kNV ? 256 * 4 : 0;   // NV: element multiplier per E4M3 byte
   // b <= 32: rows of 32 / 64 bytes make TMA tensor boxes slow, so a stage is one contiguous bulk
   // copy, left unswizzled.  Read through the swizzled descriptor, row r's K index comes out
   // XORed with 8 * t(r) (t = (r >> 2) & 1 for 32-byte rows, (r >> 1) & 3 for 64-byte rows), which
@@ -151,7 +151,7 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 // Quantize one group of G rotated sums s (unnormalised, as produced by the MMA): E2M1 code
 // words (G / 8) and the scale byte.
 template <class Cfg, int G>
-__device__ __forceinline__ uint32_t quantize_group(const float (&s)[G], uint32_t (&words)[G / 8], const float2* nv_tab,
+__device__ __forceinline__ uint32_t quantize_group(const float (&s)[G], uint32_t (&words)[G / 8], const float* nv_tab,
                                                    float nv_den, float nv_rden) {
   constexpr float c = Cfg::kC;
   f32x2 p[G / 2];
@@ -174,23 +174,16 @@ __device__ __forceinline__ uint32_t quantize_group(const float (&s)[G], uint32_t
     const float s_b = div_rn_markstein(A, nv_den, nv_rden);
     byte = e4m3_encode(s_b);
     const uint32_t keep = byte == 0u ? 0u : 0xFFFFFFFFu;   // E4M3 byte 0 is the only zero scale
-    const float2 tab = nv_tab[byte];                        // divisor and its RN reciprocal
-    const float Sd = tab.x, rd = tab.y;
-    const f32x2 rd2 = f2_pack(rd, rd), nSd2 = f2_pack(-Sd, -Sd);
+    // Element quotient y / S as the product s * RN(1 / (S sqrt(b))): within about one ulp of
+    // the correctly rounded quotient, so an element's code can only move where its exact
+    // quotient lies within a few 2^-24 (relative) of an E2M1 rounding midpoint.
+    const float rq = nv_tab[byte];
+    const f32x2 rq2 = f2_pack(rq, rq);
 #pragma unroll
     for (int j = 0; j < G / 8; ++j) {
       float v[8];
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        f32x2 y = p[4 * j + t];
-        if constexpr (!inv_sqrt_block_is_pow2(Cfg::kBlock)) {
-          constexpr float chi = inv_sqrt_block(Cfg::kBlock), clo = inv_sqrt_block_lo(Cfg::kBlock);
-          y = f2_fma(y, f2_pack(chi, chi), f2_mul(y, f2_pack(clo, clo)));
-        }
-        const f32x2 q0 = f2_mul(y, rd2);
-        const f32x2 rem = f2_fma(q0, nSd2, y);
-        f2_unpack(f2_fma(rem, rd2, q0), v[2 * t], v[2 * t + 1]);
-      }
+      for (int t = 0; t < 4; ++t) f2_unpack(f2_mul(p[4 * j + t], rq2), v[2 * t], v[2 * t + 1]);
       words[j] = e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]) & keep;
     }
   }
@@ -246,7 +239,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 2)
   tc_fence_after();
   const uint32_t tmem_base = s_tmem_base;
   const int64_t n_super = a.n_super;
-  float2* nv_tab = reinterpret_cast<float2*>(smem + S * Cfg::kStageBytes + Cfg::kHBytes);
+  float* nv_tab = reinterpret_cast<float*>(smem + S * Cfg::kStageBytes + Cfg::kHBytes);
 
   if (warp == 0) {
     // ---------------- producer
@@ -349,17 +342,19 @@ __global__ void __launch_bounds__(Cfg::kThreads, 2)
       }
       asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
       s_g = s_tensor_scale;
-      // for every E4M3 byte: the element divisor S = fp32(E4M3(byte) s_g) in the units of the
-      // butterfly sums (a power-of-two 1/sqrt(b) folded in exactly) and its RN reciprocal
+      // for every E4M3 byte: the multiplier that takes a raw MMA sum s to the element quotient,
+      // RN(1 / (S sqrt(b))) with S = fp32(E4M3(byte) s_g), from one fp64 division
       for (int byte = tid - 64; byte < 256; byte += kEpiThreads) {
         const float Sv = e4m3_decode(static_cast<uint32_t>(byte & 0x7F)) * s_g;
-        const float Sd = inv_sqrt_block_is_pow2(B) ? Sv * (1.0f / Cfg::kC) : Sv;
-        nv_tab[byte] = make_float2(Sd, Sd == 0.0f ? 0.0f : __frcp_rn(Sd));
+        nv_tab[byte] = Sv == 0.0f ? 0.0f : static_cast<float>(inv_sqrt_block_f64(B) / static_cast<double>(Sv));
       }
       asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
     }
-    // bulk-copied stages: which 8-column chunks of this lane's rows come out sign-flipped
+    // bulk-copied stages: chunk c of this lane's rows comes out sign-flipped when
+    // popcount(c & t) is odd; flip_basis[k] is the code-word mask for bit k of t
     const int flip_t = Cfg::kBulk ? ((lane_row >> Cfg::kFlipShift) & Cfg::kFlipMask) : 0;
+    const uint32_t flip_basis0 = (flip_t & 1) ? 0x88888888u : 0u;
+    const uint32_t flip_basis1 = (flip_t & 2) ? 0x88888888u : 0u;
     const float nv_den = 6.0f * s_g;
     const float nv_rden = __frcp_rn(nv_den);
     constexpr int EC = Cfg::kEpiCols;                 // 16, 32 or 64 columns
@@ -408,8 +403,10 @@ __global__ void __launch_bounds__(Cfg::kThreads, 2)
           for (int e = 0; e < G / 8; ++e) {
             const int chunk = (off + q * G) / 8 + e;   // 8-column chunk inside the block
             uint32_t w = gw[e];
-            if constexpr (Cfg::kBulk)
-              if (__popc(chunk & flip_t) & 1) w ^= 0x88888888u;
+            if constexpr (Cfg::kBulk) {
+              if (chunk & 1) w ^= flip_basis0;
+              if (chunk & 2) w ^= flip_basis1;
+            }
             words[q * (G / 8) + e] = w;
           }
           if constexpr (Cfg::kDump) {
