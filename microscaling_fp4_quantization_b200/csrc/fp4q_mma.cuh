@@ -5,19 +5,21 @@
 // fp32 accumulation in tensor memory (TMEM).  The products x * (+-1) are exact; the sums
 // are accumulated in fp32 by the tensor core.
 //
-// Work is cut into super-tiles of 128 rows by 64 TMEM columns (b <= 64: 64 / b row-tiles of
-// 128 rows, 16 KB of input) or 128 columns (b = 128, 32 KB).
-// Roles, per CTA of 6 warps:
-//   warp 0        producer: TMA tensor loads (2-D map over the rows, swizzled K-major
-//                 layout; for b <= 32 one contiguous bulk copy per stage) into a ring of
-//                 shared-memory stages, completion on mbarriers;
+// Work is cut into super-tiles of 128 TMEM columns: 128 / b row-tiles of 128 rows, 16384
+// elements, 32 KB of input.  CTAs are persistent (one or two per SM) and take super-tiles
+// round-robin.  Roles, per CTA of 2 + 8 or 2 + 16 warps:
+//   warp 0        producer: for b <= 32 one contiguous bulk copy per stage (left unswizzled,
+//                 see MmaConfig::kBulk), else TMA tensor loads (2-D map over the rows, swizzled
+//                 K-major layout), into a ring of shared-memory stages, completion on mbarriers;
 //   warp 1        TMEM owner (alloc / dealloc of two accumulator buffers) and MMA issuer:
-//                 4 or 8 MMAs per super-tile into one of the buffers, then tcgen05.commit to
-//                 free the stage and to hand the buffer to the epilogue;
-//   warps 2..     epilogue (8 or 16 warps): warp w reads TMEM lanes 32 * (w % 4) .. + 31
-//                 (tcgen05.ld), one slice of the super-tile's columns each, so each thread owns
-//                 one row (one rotated block, or a part of one) and does the amax, scale, E2M1
-//                 rounding, packing and stores of it in its registers.
+//                 b / 16 MMAs per row-tile into one of the buffers, then tcgen05.commit to free
+//                 the stage and to hand the buffer to the epilogue;
+//   warps 2..     epilogue: warp w reads TMEM lanes 32 * (w % 4) .. + 31 (tcgen05.ld), one
+//                 column slice of the super-tile each, so each thread owns one row (one rotated
+//                 block, or a part of one) and does the amax, scale, E2M1 rounding, packing and
+//                 stores of it in its registers; it frees the buffer as soon as its slice is read.
+// All roles wait on the grid dependency (programmatic dependent launch) before touching global
+// memory, so the set-up overlaps the end of the kernel this one follows.
 // H_b is written into shared memory once per CTA, in the same swizzled layout.
 // Every wait is bounded in time; a wait that runs out records kStatusTimeout, and the CTA
 // lets its issued copies and MMAs land before it frees TMEM and leaves.
