@@ -394,3 +394,43 @@ def flags(res: dict, tol: float = 1e-5):
         near = np.minimum(np.abs(s_b - mids[idx - 1]) / mids[idx - 1], np.abs(s_b - mids[idx]) / mids[idx])
         gr = near <= tol
     return el.reshape(M, K), gr
+
+
+# ----------------------------------------------------------------------------------
+# Quantization error ([BG] Technische Zusammenfassung, 2. Methodik, "Theoretische Analyse
+# der Fehler": the mean squared quantization error; [UP] Methodologie 1: the gain of OAS
+# is stated in QSNR, the quantization signal-to-noise ratio, in dB)
+# ----------------------------------------------------------------------------------
+
+def quant_error(x_bits: np.ndarray, fmt: int, group: int, block: int, rule: int,
+                tensor_scale=None, chunk_rows: int = 512) -> dict:
+    """Signal and error energy of rotate + quantize on X, and the QSNR.
+
+    signal = sum of y^2 and noise = sum of (y - yhat)^2 over all elements, where y are the
+    exact rotated values (fp64) and yhat the dequantized codes, exact in fp64: q * 2^e for
+    MXFP4, q * E4M3(s_b) * s_g for NVFP4.  qsnr_db = 10 log10(signal / noise), +inf when
+    noise is 0.  The rotation is orthonormal, so these are also the energies in the
+    unrotated domain.  The sums are additive over rows: row chunks are summed in order.
+
+    NVFP4 takes ``tensor_scale`` like ``rotate_quantize``; the dynamic rule computes it
+    from the whole tensor's rotated amax when it is None."""
+    check_plan(fmt, group, block, rule)
+    x_bits = np.asarray(x_bits, np.uint16)
+    M, K = x_bits.shape
+    if fmt == NVFP4 and tensor_scale is None:
+        if rule != SCALE_NV_DYNAMIC:
+            raise ValueError("the static NV rule needs the tensor scale")
+        tensor_scale = nv_tensor_scale(rotated_amax(x_bits, block))
+    signal = 0.0
+    noise = 0.0
+    for r in range(0, M, chunk_rows):
+        res = rotate_quantize(x_bits[r:r + chunk_rows], fmt, group, block, rule, tensor_scale)
+        y = res["y64"]
+        m = y.shape[0]
+        q = e2m1_decode(unpack_nibbles(res["codes"])).reshape(m, K // group, group)
+        yhat = (q * res["S64"][..., None]).reshape(m, K)
+        signal += float(np.sum(y * y))
+        noise += float(np.sum((y - yhat) ** 2))
+    qsnr = math.inf if noise == 0.0 else 10.0 * math.log10(signal / noise) if signal > 0 else -math.inf
+    return {"signal": signal, "noise": noise, "qsnr_db": qsnr,
+            "mse": noise / (M * K) if M * K else 0.0, "tensor_scale": tensor_scale}

@@ -150,3 +150,55 @@ def test_nv_divisor_mistake_is_caught(monkeypatch):
 
     patch(monkeypatch, "rotate_quantize", wrong)
     assert fails(pins.test_nv_worked_groups)
+
+
+# ---- quantization-error energies (pins in test_oracle_qsnr.py)
+
+import test_oracle_qsnr as qpins  # noqa: E402
+
+
+def _quant_error_variant(kind):
+    def qe(x_bits, fmt, group, block, rule, tensor_scale=None, chunk_rows=512):
+        x_bits = np.asarray(x_bits, np.uint16)
+        M, K = x_bits.shape
+        if fmt == o.NVFP4 and tensor_scale is None:
+            tensor_scale = o.nv_tensor_scale(o.rotated_amax(x_bits, block))
+        res = o.rotate_quantize(x_bits, fmt, group, block, rule, tensor_scale)
+        y = res["y64"]
+        q = o.e2m1_decode(o.unpack_nibbles(res["codes"])).reshape(M, K // group, group)
+        S = res["S64"]
+        if kind == "no_tensor_scale" and fmt == o.NVFP4:
+            S = S / np.float64(tensor_scale)
+        yhat = (q * S[..., None]).reshape(M, K)
+        ref = o.bf16_to_f64(x_bits) if kind == "mixed_domain" else y
+        err = ref - yhat
+        noise = float(np.sum(np.abs(err))) if kind == "abs_error" else float(np.sum(err * err))
+        signal = float(np.sum(y * y)) * (block if kind == "unnormalised_signal" else 1)
+        qsnr = math.inf if noise == 0 else 10 * math.log10(signal / noise) if signal > 0 else -math.inf
+        return {"signal": signal, "noise": noise, "qsnr_db": qsnr, "mse": noise / max(M * K, 1),
+                "tensor_scale": tensor_scale}
+    qe.__name__ = "quant_error_" + kind
+    return qe
+
+
+QE_MUTATIONS = [
+    ("abs_error", [qpins.test_hand_worked_mx_group, qpins.test_hand_worked_nv_group]),
+    ("mixed_domain", [qpins.test_energies_match_the_unrotated_domain]),
+    ("no_tensor_scale", [qpins.test_energies_match_the_unrotated_domain]),
+    ("unnormalised_signal", [qpins.test_energies_match_the_unrotated_domain]),
+]
+
+
+@pytest.mark.parametrize("kind,catchers", QE_MUTATIONS, ids=[m[0] for m in QE_MUTATIONS])
+def test_qsnr_pins_catch_planted_mistake(monkeypatch, kind, catchers):
+    patch(monkeypatch, "quant_error", _quant_error_variant(kind))
+    for catcher in catchers:
+        assert fails(catcher), f"{catcher.__name__} missed quant_error_{kind}"
+
+
+def test_qsnr_variant_without_mistake_passes(monkeypatch):
+    """The mutation harness itself: the variant with no planted mistake passes every pin."""
+    patch(monkeypatch, "quant_error", _quant_error_variant("none"))
+    for pin in (qpins.test_energies_match_the_unrotated_domain, qpins.test_hand_worked_mx_group,
+                qpins.test_hand_worked_nv_group):
+        pin()
