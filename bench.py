@@ -295,6 +295,11 @@ def run_gpu(args):
                            "bytes_per_call": nbytes}
         extra["dynamic_mode"]["note"] = "reads X twice (amax pass, then quantize); bytes are the algorithmic ones"
 
+    # the quantization-error pass (signal / error energies and QSNR) on the same workload
+    if rank == 0:
+        extra["quant_error"] = time_quant_error(torch, F, w, plan, xs, ts if is_nv else None, stream, peak,
+                                                max(50, min(args.steps, 400)))
+
     # e2e: the public API with host buffers, H2D of X and D2H of codes + scales inside the region
     e2e = None
     if rank == 0 or world > 1:
@@ -422,6 +427,36 @@ def run_kernel_only(args):
     print(f"kernel-only: {w.name} M={w.M} K={w.K} launches={args.warmup + args.steps}", flush=True)
 
 
+def time_quant_error(torch, F, w, plan, xs, ts, stream, peak, steps):
+    """fp4q_quant_error on the workload's rotating inputs: device time per call (one kernel),
+    GB/s on its algorithmic bytes (X read once, 24 bytes out) and the QSNR."""
+    M, K = w.M, w.K
+    out = torch.empty(3, dtype=torch.float64, device=xs[0].device)
+
+    def launch(i):
+        F.fp4q_quant_error(plan, xs[i], M, K, ts, out, stream=torch.cuda.current_stream())
+
+    with torch.cuda.stream(stream):
+        g, g_rem, reps = time_graph_steps(torch, launch, len(xs), steps, 3, stream)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        a1.record(stream)
+    torch.cuda.synchronize()
+    us = a0.elapsed_time(a1) * 1e3 / steps
+    launch(0)
+    torch.cuda.synchronize()
+    sig, err, q = out.tolist()
+    nbytes = 2 * M * K + 24
+    gbs = nbytes / us / 1e3
+    return {"us_per_call": round(us, 3), "GBps": round(gbs, 1), "pct_of_hbm_peak": round(100 * gbs / peak, 2),
+            "bytes_per_call": nbytes, "launches_per_call": 1, "qsnr_db": round(q, 4), "signal": sig, "error": err,
+            "mse": err / (M * K)}
+
+
 def time_other(torch, F, w, dev, stream, peak, kernel="auto"):
     M, K = w.M, w.K
     plan = F.fp4q_plan_create(w.fmt, w.group, w.block, w.rule)
@@ -458,6 +493,9 @@ def time_other(torch, F, w, dev, stream, peak, kernel="auto"):
     gbs = bytes_call / us / 1e3
     out = {"GBps": round(gbs, 1), "pct_of_hbm_peak": round(100 * gbs / peak, 2), "us_per_call": round(us, 3),
            "bytes_per_call": bytes_call, "buffers": n_buf, "kernel": kernel_name(w, kernel)}
+    if kernel == "auto":
+        out["quant_error"] = time_quant_error(torch, F, w, plan, xs, ts if w.fmt == W.NVFP4 else None, stream, peak,
+                                              steps // 2)
     del xs, codes, scales
     torch.cuda.empty_cache()
     return out

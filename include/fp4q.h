@@ -146,6 +146,27 @@ fp4q_status fp4q_dequantize(fp4q_plan plan, const void* codes, const void* scale
                             const float* tensor_scale, int64_t M, int64_t K, int unrotate,
                             float* out_f32, void* stream);
 
+/* Quantization error of rotate + quantize on X, without storing codes or scales: the
+ * signal and error energies sum y^2 and sum (y - yhat)^2 over all M*K elements and the QSNR
+ * 10 log10(signal / error) in dB.  y are the rotated values and yhat the dequantized codes
+ * the plan's fp4q_rotate_quantize would produce (the same scale decisions and codes).  The
+ * rotation is orthonormal, so both energies are also those of X against its dequantized,
+ * rotated-back copy.  This is the measure of the error analysis in "Bridging the Gap Between
+ * Promise and Performance for Microscaling FP4 Quantization" (Technische Zusammenfassung,
+ * 2. Methodik: quantization MSE = error / (M*K)) and of the QSNR gains in "Unveiling the
+ * Potential of Quantization with MXFP4" (Methodologie 1).
+ *
+ * x_bf16: device bf16 [M][K]; tensor_scale: device fp32 as for fp4q_rotate_quantize (NV
+ * static: read; NV dynamic: written; MX: ignored, may be NULL); out: device fp64 [3] =
+ * {signal, error, QSNR dB}, +inf dB when the error is 0 (an empty X gives {0, 0, +inf}).
+ * The result is deterministic: per-CTA partial sums in fp64 (in a scratch array the plan
+ * owns, allocated when the plan is made on a machine with a CUDA device), then one
+ * fixed-order reduction.  Calls on one plan must not overlap on the GPU.  Returns
+ * FP4Q_ERR_UNSUPPORTED for a plan made without a CUDA device; argument errors as for
+ * fp4q_rotate_quantize, and out must be 8-byte aligned. */
+fp4q_status fp4q_quant_error(fp4q_plan plan, const void* x_bf16, int64_t M, int64_t K,
+                             float* tensor_scale, double* out, void* stream);
+
 /* No-allocation NVFP4 dynamic-scale path.  The paper has no counterpart: this exists for
  * callers that cannot allocate device memory themselves — for example a library loaded into
  * a framework or serving runtime whose own allocator owns all device memory, or a service that

@@ -23,6 +23,9 @@ struct fp4q_plan_s {
   float* partials; // NV plans: per-CTA rotated amaxima (device)
   int n_partials;
   int kernel;      // fp4q_kernel
+  double* err_partials;  // fp4q_quant_error scratch (device; null without a device): per-CTA signal and
+                         // error energy, then a ticket counter
+  int n_err_partials;    // CTAs those hold room for
 };
 
 namespace {
@@ -337,6 +340,62 @@ fp4q_status rotate_quantize_impl(fp4q_plan p, const void* x, int64_t M, int64_t 
   });
 }
 
+// ---- quantization error energies (butterfly kernel for every block size)
+
+// Call f.template operator()<Cfg>() for the butterfly configuration of (format, block, rule);
+// NVFP4 takes 32-element units when the element count allows (u32), else 16.
+template <class F>
+fp4q_status with_rq_cfg(int format, int block, int rule, bool u32, F&& f) {
+  return with_block(block, [&]<int B>() -> fp4q_status {
+    if (format == FP4Q_MXFP4) {
+      switch (rule) {
+        case FP4Q_SCALE_FLOOR_OCP: return f.template operator()<RQConfig<kMX, B, kRuleFloor, false>>();
+        case FP4Q_SCALE_CEIL_NOCLIP: return f.template operator()<RQConfig<kMX, B, kRuleCeil, false>>();
+        case FP4Q_SCALE_OAS: return f.template operator()<RQConfig<kMX, B, kRuleOas, false>>();
+        default: return FP4Q_ERR_UNSUPPORTED;
+      }
+    }
+    if (rule == FP4Q_SCALE_NV_DYNAMIC)
+      return u32 ? f.template operator()<RQConfig<kNV, B, kRuleNvDynamic, false, 32>>()
+                 : f.template operator()<RQConfig<kNV, B, kRuleNvDynamic, false, 16>>();
+    return u32 ? f.template operator()<RQConfig<kNV, B, kRuleNvStatic, false, 32>>()
+               : f.template operator()<RQConfig<kNV, B, kRuleNvStatic, false, 16>>();
+  });
+}
+
+// CTAs of one full wave of the error kernel for the plan, over both unit sizes.
+fp4q_status qe_grid(int format, int block, int rule, int* n) {
+  *n = 0;
+  for (int u32 = 0; u32 < 2; ++u32) {
+    fp4q_status st = with_rq_cfg(format, block, rule, u32 != 0, [&]<class Cfg>() -> fp4q_status {
+      KernelInfo ki;
+      fp4q_status r = kernel_info(quant_error_kernel<Cfg>, Cfg::kSmemBytes, Cfg::kThreads, &ki);
+      if (r == FP4Q_OK && ki.sm_count * ki.ctas_per_sm > *n) *n = ki.sm_count * ki.ctas_per_sm;
+      return r;
+    });
+    if (st != FP4Q_OK) return st;
+  }
+  return FP4Q_OK;
+}
+
+template <class Cfg>
+fp4q_status launch_qe(fp4q_plan p, QEArgs a, int64_t n_elems, double* out, cudaStream_t stream) {
+  a.n_units = n_elems / Cfg::kE;
+  auto kernel = quant_error_kernel<Cfg>;
+  KernelInfo ki;
+  fp4q_status st = kernel_info(kernel, Cfg::kSmemBytes, Cfg::kThreads, &ki);
+  if (st != FP4Q_OK) return st;
+  const int64_t warps_needed = (a.n_units + Cfg::kUnitsPerStage - 1) / Cfg::kUnitsPerStage;
+  int64_t ctas = (warps_needed + Cfg::kWarps - 1) / Cfg::kWarps;
+  const int64_t max_ctas = static_cast<int64_t>(ki.sm_count) * ki.ctas_per_sm;
+  if (ctas > max_ctas) ctas = max_ctas;
+  if (ctas > p->n_err_partials) ctas = p->n_err_partials;
+  a.out = out;
+  cudaError_t e = launch_pdl(kernel, dim3(static_cast<unsigned>(ctas)), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, a);
+  if (e != cudaSuccess) return cuda_fail(e, "quant_error launch");
+  return FP4Q_OK;
+}
+
 // ---- no-allocation NVFP4 dynamic path: partial maxima in a fixed device array
 
 constexpr int kNoAllocMaxPartials = 4096;
@@ -459,18 +518,40 @@ fp4q_status fp4q_plan_create(fp4q_plan* out, int format, int group, int hadamard
   p->partials = nullptr;
   p->n_partials = 0;
   p->kernel = FP4Q_KERNEL_AUTO;
+  p->err_partials = nullptr;
+  p->n_err_partials = 0;
+  fp4q_status st = FP4Q_OK;
   if (format == FP4Q_NVFP4) {
     cudaError_t e = cudaGetDevice(&p->device);
-    fp4q_status st = e == cudaSuccess ? amax_grid(hadamard_block, &p->n_partials) : cuda_fail(e, "cudaGetDevice");
+    st = e == cudaSuccess ? amax_grid(hadamard_block, &p->n_partials) : cuda_fail(e, "cudaGetDevice");
     if (st == FP4Q_OK) {
       e = cudaMalloc(&p->partials, sizeof(float) * static_cast<size_t>(p->n_partials));
       if (e != cudaSuccess) st = cuda_fail(e, "cudaMalloc partials");
     }
-    if (st != FP4Q_OK) {
-      p->magic = 0;
-      delete p;
-      return st;
+  } else {
+    // an MX plan needs a device only for fp4q_quant_error's scratch: without one it is still made
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+      (void)cudaGetLastError();
+      *out = p;
+      return FP4Q_OK;
     }
+    cudaError_t e = cudaGetDevice(&p->device);
+    if (e != cudaSuccess) st = cuda_fail(e, "cudaGetDevice");
+  }
+  if (st == FP4Q_OK) st = qe_grid(format, hadamard_block, scale_rule, &p->n_err_partials);
+  if (st == FP4Q_OK) {
+    // the partial pairs, then the ticket counter (zeroed once; each call's last CTA re-zeroes it)
+    const size_t bytes = (2 * static_cast<size_t>(p->n_err_partials) + 1) * sizeof(double);
+    cudaError_t e = cudaMalloc(&p->err_partials, bytes);
+    if (e == cudaSuccess) e = cudaMemset(p->err_partials, 0, bytes);
+    if (e != cudaSuccess) st = cuda_fail(e, "cudaMalloc error partials");
+  }
+  if (st != FP4Q_OK) {
+    if (p->partials) cudaFree(p->partials);
+    p->magic = 0;
+    delete p;
+    return st;
   }
   *out = p;
   return FP4Q_OK;
@@ -492,6 +573,10 @@ fp4q_status fp4q_plan_destroy(fp4q_plan plan) {
   if (plan->partials) {
     cudaError_t e = cudaFree(plan->partials);
     if (e != cudaSuccess) st = cuda_fail(e, "cudaFree partials");
+  }
+  if (plan->err_partials) {
+    cudaError_t e = cudaFree(plan->err_partials);
+    if (e != cudaSuccess) st = cuda_fail(e, "cudaFree error partials");
   }
   plan->magic = 0;
   delete plan;
@@ -525,6 +610,45 @@ fp4q_status fp4q_amax(fp4q_plan plan, const void* x_bf16, int64_t M, int64_t K, 
                              tensor_scale_out);
   if (e != cudaSuccess) return cuda_fail(e, "finalize launch");
   return FP4Q_OK;
+}
+
+fp4q_status fp4q_quant_error(fp4q_plan plan, const void* x_bf16, int64_t M, int64_t K, float* tensor_scale,
+                             double* out, void* stream) {
+  if (!valid_plan(plan)) return FP4Q_ERR_ARG;
+  fp4q_status st = check_shape(plan, M, K);
+  if (st != FP4Q_OK) return st;
+  if (!out) return FP4Q_ERR_ARG;
+  if (plan->format == FP4Q_NVFP4 && !tensor_scale) return FP4Q_ERR_ARG;
+  if (M * K > 0 && !x_bf16) return FP4Q_ERR_ARG;
+  if ((x_bf16 && !aligned(x_bf16, 16)) || !aligned(out, 8) || (tensor_scale && !aligned(tensor_scale, 4)))
+    return FP4Q_ERR_ALIGN;
+  if (!plan->err_partials) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+                  "fp4q_quant_error: the plan was made without a CUDA device, so it holds no scratch");
+    return FP4Q_ERR_UNSUPPORTED;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t n = M * K;
+  if (n == 0) {
+    cudaError_t e = launch_pdl(quant_error_empty_kernel, dim3(1), dim3(32), 0, s,
+                               static_cast<const double*>(plan->err_partials), out);
+    return e == cudaSuccess ? FP4Q_OK : cuda_fail(e, "quant_error finalize launch");
+  }
+  QEArgs a;
+  a.x = static_cast<const uint16_t*>(x_bf16);
+  a.n_units = 0;
+  a.tensor_scale = tensor_scale;
+  a.partials = plan->partials;
+  a.n_partials = plan->n_partials;
+  a.out_partials = plan->err_partials;
+  a.ticket = reinterpret_cast<unsigned int*>(plan->err_partials + 2 * static_cast<int64_t>(plan->n_err_partials));
+  a.out = out;
+  if (plan->format == FP4Q_NVFP4 && plan->rule == FP4Q_SCALE_NV_DYNAMIC) {
+    st = launch_amax(plan, a.x, n, s);
+    if (st != FP4Q_OK) return st;
+  }
+  return with_rq_cfg(plan->format, plan->block, plan->rule, n % 32 == 0,
+                     [&]<class Cfg>() -> fp4q_status { return launch_qe<Cfg>(plan, a, n, out, s); });
 }
 
 fp4q_status fp4q_dequantize(fp4q_plan plan, const void* codes, const void* scales, const float* tensor_scale,

@@ -260,6 +260,56 @@ __device__ __forceinline__ float div_rn_markstein(float a, float d, float rd) {
   return fmaf(r, rd, q0);
 }
 
+// Element quotients v = y / X of N pairs of unnormalised sums s (y = RN(s / sqrt(b))), in the
+// pairs' own (raw butterfly) signs.
+//
+// MX: X = 2^e, so v = s * (c 2^-e), c = fp32(1/sqrt(b)): one product with a power-of-two
+// multiple of c.
+template <int N>
+__device__ __forceinline__ void mx_quotients(const f32x2* s, int byte, float c, f32x2 (&v)[N]) {
+  const float mult = c * mx_inv_scale(byte);
+  const f32x2 mm = f2_pack(mult, mult);
+#pragma unroll
+  for (int t = 0; t < N; ++t) v[t] = f2_mul(s[t], mm);
+}
+
+// NV: the correctly rounded quotient y / S.  With a power-of-two 1/sqrt(b) it is folded into
+// the divisor (exactly): s / (S sqrt(b)); otherwise y is first rounded from s with the
+// two-term constant.  Sd is the divisor, rd = RN(1 / Sd).
+struct NvDivisor {
+  float Sd, rd;
+};
+
+template <int B>
+__device__ __forceinline__ NvDivisor nv_divisor(float S) {
+  const float Sd = inv_sqrt_block_is_pow2(B) ? S * (1.0f / inv_sqrt_block(B)) : S;
+  return {Sd, __frcp_rn(Sd)};
+}
+
+template <int B, int N>
+__device__ __forceinline__ void nv_quotients(const f32x2* s, NvDivisor dv, f32x2 (&v)[N]) {
+  const f32x2 rd2 = f2_pack(dv.rd, dv.rd), nSd2 = f2_pack(-dv.Sd, -dv.Sd);
+#pragma unroll
+  for (int t = 0; t < N; ++t) {
+    f32x2 y = s[t];
+    if constexpr (!inv_sqrt_block_is_pow2(B)) {
+      constexpr float chi = inv_sqrt_block(B), clo = inv_sqrt_block_lo(B);
+      y = f2_fma(y, f2_pack(chi, chi), f2_mul(y, f2_pack(clo, clo)));
+    }
+    const f32x2 q0 = f2_mul(y, rd2);   // Markstein correction, lane-wise
+    const f32x2 rem = f2_fma(q0, nSd2, y);
+    v[t] = f2_fma(rem, rd2, q0);
+  }
+}
+
+// E2M1 code word of four pairs (element 0 in the low nibble).
+__device__ __forceinline__ uint32_t e2m1x8_pairs(const f32x2 (&v)[4]) {
+  float e[8];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) f2_unpack(v[t], e[2 * t], e[2 * t + 1]);
+  return e2m1x8(e[0], e[1], e[2], e[3], e[4], e[5], e[6], e[7]);
+}
+
 // Quantize one rotated unit (pairs p, unnormalised butterfly sums) and store its codes and
 // scales.  `lx` undoes the chunk XOR's sign flips.
 template <class Cfg>
@@ -276,15 +326,12 @@ __device__ __forceinline__ void quantize_store_unit(const f32x2 (&p)[Cfg::kPairs
     if constexpr (Cfg::kFmt == kMX) {
       const int byte = mx_scale_byte<Cfg::kRule>(A);
       sbytes[q] = static_cast<uint32_t>(byte);
-      const float mult = c * mx_inv_scale(byte);   // a power-of-two multiple of c
-      const f32x2 mm = f2_pack(mult, mult);
 #pragma unroll
       for (int j = 0; j < G / 8; ++j) {
         const int chunk = q * (G / 8) + j;
-        float v[8];
-#pragma unroll
-        for (int t = 0; t < 4; ++t) f2_unpack(f2_mul(p[4 * chunk + t], mm), v[2 * t], v[2 * t + 1]);
-        words[chunk] = e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]) ^ chunk_sign_mask<Cfg::kBlock>(lx, chunk);
+        f32x2 v[4];
+        mx_quotients<4>(&p[4 * chunk], byte, c, v);
+        words[chunk] = e2m1x8_pairs(v) ^ chunk_sign_mask<Cfg::kBlock>(lx, chunk);
       }
     } else {
       const float s_b = div_rn_markstein(A, nv_den, nv_rden);
@@ -292,28 +339,13 @@ __device__ __forceinline__ void quantize_store_unit(const f32x2 (&p)[Cfg::kPairs
       sbytes[q] = byte;
       const float S = e4m3_decode(byte) * s_g;
       const uint32_t keep = S == 0.0f ? 0u : 0xFFFFFFFFu;   // a zero block scale gives zero codes
-      // Element code from the correctly rounded quotient y / S, y = RN(s / sqrt(b)).  With a
-      // power-of-two 1/sqrt(b) it is folded into the divisor (exactly): s / (S sqrt(b)).
-      const float Sd = inv_sqrt_block_is_pow2(Cfg::kBlock) ? S * (1.0f / c) : S;
-      const float rd = __frcp_rn(Sd);
-      const f32x2 rd2 = f2_pack(rd, rd), nSd2 = f2_pack(-Sd, -Sd);
+      const NvDivisor dv = nv_divisor<Cfg::kBlock>(S);
 #pragma unroll
       for (int j = 0; j < G / 8; ++j) {
         const int chunk = q * (G / 8) + j;
-        float v[8];
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          f32x2 y = p[4 * chunk + t];
-          if constexpr (!inv_sqrt_block_is_pow2(Cfg::kBlock)) {
-            constexpr float chi = inv_sqrt_block(Cfg::kBlock), clo = inv_sqrt_block_lo(Cfg::kBlock);
-            y = f2_fma(y, f2_pack(chi, chi), f2_mul(y, f2_pack(clo, clo)));
-          }
-          const f32x2 q0 = f2_mul(y, rd2);                  // Markstein correction, lane-wise
-          const f32x2 rem = f2_fma(q0, nSd2, y);
-          f2_unpack(f2_fma(rem, rd2, q0), v[2 * t], v[2 * t + 1]);
-        }
-        words[chunk] = (e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]) ^
-                        chunk_sign_mask<Cfg::kBlock>(lx, chunk)) & keep;
+        f32x2 v[4];
+        nv_quotients<Cfg::kBlock, 4>(&p[4 * chunk], dv, v);
+        words[chunk] = (e2m1x8_pairs(v) ^ chunk_sign_mask<Cfg::kBlock>(lx, chunk)) & keep;
       }
     }
   }
@@ -440,6 +472,32 @@ __device__ __forceinline__ bool stream_units(const uint16_t* __restrict__ x, int
   return ok;
 }
 
+// NV tensor scale s_g for every thread of the CTA: read (static rule), or reduced from the
+// amax pass's per-CTA partial maxima (dynamic rule; CTA 0 also writes it out).  Contains a
+// __syncthreads; every thread of the CTA calls it.
+template <class Cfg>
+__device__ __forceinline__ float cta_tensor_scale(float* tensor_scale, const float* partials, int n_partials,
+                                                  float* s_slot) {
+  pdl_wait();   // the tensor scale or the partial maxima come from an earlier kernel
+  if constexpr (Cfg::kRule == kRuleNvDynamic) {
+    if (threadIdx.x < 32) {
+      float m = 0.0f;
+      for (int i = threadIdx.x; i < n_partials; i += 32) m = fmaxf(m, partials[i]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+      if (threadIdx.x == 0) {
+        const float sg = m == 0.0f ? 1.0f : __fdiv_rn(m, 2688.0f);
+        *s_slot = sg;
+        if (blockIdx.x == 0) *tensor_scale = sg;
+      }
+    }
+  } else {
+    if (threadIdx.x == 0) *s_slot = *tensor_scale;
+  }
+  __syncthreads();
+  return *s_slot;
+}
+
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::kThreads) rotate_quantize_kernel(RQArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -448,32 +506,196 @@ __global__ void __launch_bounds__(Cfg::kThreads) rotate_quantize_kernel(RQArgs a
   const int warp = threadIdx.x >> 5;
   const LaneXor lx = lane_xor<Cfg>(threadIdx.x & 31);
   float s_g = 1.0f;
-  if constexpr (Cfg::kFmt == kNV) {
-    pdl_wait();   // the tensor scale or the partial maxima come from an earlier kernel
-    if constexpr (Cfg::kRule == kRuleNvDynamic) {
-      if (warp == 0) {
-        float m = 0.0f;
-        for (int i = threadIdx.x; i < a.n_partials; i += 32) m = fmaxf(m, a.partials[i]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-        if (threadIdx.x == 0) {
-          const float sg = m == 0.0f ? 1.0f : __fdiv_rn(m, 2688.0f);
-          s_tensor_scale = sg;
-          if (blockIdx.x == 0) *a.tensor_scale = sg;
-        }
-      }
-    } else {
-      if (threadIdx.x == 0) s_tensor_scale = *a.tensor_scale;
-    }
-    __syncthreads();
-    s_g = s_tensor_scale;
-  }
+  if constexpr (Cfg::kFmt == kNV) s_g = cta_tensor_scale<Cfg>(a.tensor_scale, a.partials, a.n_partials, &s_tensor_scale);
   const float nv_den = 6.0f * s_g;
   const float nv_rden = __frcp_rn(nv_den);
   stream_units<Cfg>(a.x, a.n_units, smem + warp * Cfg::kWarpSmem, lx.tau,
                     [&](const f32x2 (&p)[Cfg::kPairs], int64_t unit) {
                       quantize_store_unit<Cfg>(p, unit, lx, s_g, nv_den, nv_rden, a);
                     });
+}
+
+// ---------------------------------------------------------------- quantization error
+
+// E2M1 code word (element 0 in the low nibble) -> the eight values, as four fp32 pairs.
+// Nibble c = s|k (k = magnitude code) becomes the fp32 bit pattern s<<31 | k<<22, which is
+// 2^-126 * {0, 0.5, 1, 1.5, 2, 3, 4, 6}[k] (k = 1 a subnormal), then an exact product by
+// 2^126 (subnormals are kept: nothing here is compiled with flush-to-zero).
+__device__ __forceinline__ void e2m1x8_decode(uint32_t w, f32x2 (&d)[4]) {
+  const f32x2 up = f2_pack(0x1p126f, 0x1p126f);
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const uint32_t n0 = w >> (8 * t), n1 = w >> (8 * t + 4);
+    const uint32_t b0 = ((n0 & 7u) << 22) | ((n0 & 8u) << 28);
+    const uint32_t b1 = ((n1 & 7u) << 22) | ((n1 & 8u) << 28);
+    d[t] = f2_mul(f2_pack(__uint_as_float(b0), __uint_as_float(b1)), up);
+  }
+}
+
+// Error energy of one group of quotients v (= y / X) against their E2M1 codes, and its
+// signal energy, both in units of X^2: sum (v - q)^2 and sum v^2 (fp32, pairwise lanes).
+template <int NP>
+__device__ __forceinline__ void group_energies(const f32x2 (&v)[NP], float& sig, float& err) {
+  f32x2 as = f2_pack(0.0f, 0.0f), ae = f2_pack(0.0f, 0.0f);
+#pragma unroll
+  for (int j = 0; j < NP / 4; ++j) {
+    f32x2 vv[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) vv[t] = v[4 * j + t];
+    f32x2 d[4];
+    e2m1x8_decode(e2m1x8_pairs(vv), d);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const f32x2 e = f2_sub(vv[t], d[t]);
+      as = f2_fma(vv[t], vv[t], as);
+      ae = f2_fma(e, e, ae);
+    }
+  }
+  float a0, a1, e0, e1;
+  f2_unpack(as, a0, a1);
+  f2_unpack(ae, e0, e1);
+  sig = a0 + a1;
+  err = e0 + e1;
+}
+
+// 2^(2(byte - 127)) as fp64: X^2 for an MX scale byte.
+__device__ __forceinline__ double mx_scale_sq(int byte) {
+  return __longlong_as_double(static_cast<long long>(1023 + 2 * (byte - 127)) << 52);
+}
+
+// Signal and error energy of one rotated unit, accumulated into fp64 running sums.  The
+// codes are those of quantize_store_unit (the same scale decisions and quotients).
+template <class Cfg>
+__device__ __forceinline__ void unit_energies(const f32x2 (&p)[Cfg::kPairs], float s_g, float nv_den, float nv_rden,
+                                              double& sig, double& err) {
+  constexpr int G = Cfg::kGroup, NG = Cfg::kGroupsPerUnit;
+  constexpr float c = Cfg::kC;
+#pragma unroll
+  for (int q = 0; q < NG; ++q) {
+    const f32x2* pg = &p[q * G / 2];
+    const float A = scale_by_inv_sqrt<Cfg::kBlock>(pairs_amax<G / 2>(pg));
+    f32x2 v[G / 2];
+    double X2;
+    if constexpr (Cfg::kFmt == kMX) {
+      const int byte = mx_scale_byte<Cfg::kRule>(A);
+      mx_quotients<G / 2>(pg, byte, c, v);
+      X2 = mx_scale_sq(byte);
+    } else {
+      const float s_b = div_rn_markstein(A, nv_den, nv_rden);
+      const uint32_t byte = e4m3_encode(s_b);
+      const float S = e4m3_decode(byte) * s_g;
+      if (S == 0.0f) {
+        // a zero block scale: every code is 0, the error is the whole signal
+        constexpr double c64 = inv_sqrt_block_f64(Cfg::kBlock);
+        double e2 = 0.0;
+#pragma unroll
+        for (int t = 0; t < G / 2; ++t) {
+          float lo, hi;
+          f2_unpack(pg[t], lo, hi);
+          const double a = lo * c64, b = hi * c64;
+          e2 = fma(a, a, fma(b, b, e2));
+        }
+        sig += e2;
+        err += e2;
+        continue;
+      }
+      nv_quotients<Cfg::kBlock, G / 2>(pg, nv_divisor<Cfg::kBlock>(S), v);
+      X2 = static_cast<double>(S) * static_cast<double>(S);
+    }
+    float gs, ge;
+    group_energies<G / 2>(v, gs, ge);
+    sig = fma(static_cast<double>(gs), X2, sig);
+    err = fma(static_cast<double>(ge), X2, err);
+  }
+}
+
+struct QEArgs {
+  const uint16_t* x;
+  int64_t n_units;
+  float* tensor_scale;      // NV: static -> read; dynamic -> written by CTA 0
+  const float* partials;    // NV dynamic: per-CTA rotated amaxima from the amax pass
+  int n_partials;
+  double* out_partials;     // [gridDim.x][2]: signal, error energy of each CTA
+  unsigned int* ticket;     // CTAs done so far; 0 between calls (the last CTA resets it)
+  double* out;              // [3]: signal, error, QSNR dB
+};
+
+// out = {signal, error, QSNR in dB} from n per-CTA partial pairs, by one warp in a fixed
+// order; +inf dB when the error is 0, -inf when only the signal is.
+__device__ __forceinline__ void qe_final_sum(const double* partials, int n, double* out) {
+  double s = 0.0, e = 0.0;
+  for (int i = threadIdx.x & 31; i < n; i += 32) {
+    s += __ldcg(partials + 2 * i);
+    e += __ldcg(partials + 2 * i + 1);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+    e += __shfl_xor_sync(0xFFFFFFFFu, e, o);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    out[0] = s;
+    out[1] = e;
+    out[2] = e == 0.0 ? __longlong_as_double(0x7FF0000000000000LL)
+                      : (s > 0.0 ? 10.0 * log10(s / e) : __longlong_as_double(static_cast<long long>(0xFFF0000000000000ULL)));
+  }
+}
+
+// Every CTA writes the signal and error energy of its warps' ranges to out_partials; the
+// last CTA to finish (a ticket counter, as in a threadfence reduction) sums them in CTA order
+// and writes out.  The ranges and the order of every sum are fixed by the grid, so the
+// result is deterministic.
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::kThreads) quant_error_kernel(QEArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ float s_tensor_scale;
+  __shared__ double s_part[Cfg::kWarps][2];
+  __shared__ bool s_last;
+  pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const LaneXor lx = lane_xor<Cfg>(lane);
+  float s_g = 1.0f;
+  if constexpr (Cfg::kFmt == kNV) s_g = cta_tensor_scale<Cfg>(a.tensor_scale, a.partials, a.n_partials, &s_tensor_scale);
+  const float nv_den = 6.0f * s_g;
+  const float nv_rden = __frcp_rn(nv_den);
+  double sig = 0.0, err = 0.0;
+  stream_units<Cfg>(a.x, a.n_units, smem + warp * Cfg::kWarpSmem, lx.tau,
+                    [&](const f32x2 (&p)[Cfg::kPairs], int64_t) { unit_energies<Cfg>(p, s_g, nv_den, nv_rden, sig, err); });
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sig += __shfl_xor_sync(0xFFFFFFFFu, sig, o);
+    err += __shfl_xor_sync(0xFFFFFFFFu, err, o);
+  }
+  if (lane == 0) {
+    s_part[warp][0] = sig;
+    s_part[warp][1] = err;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double ts = 0.0, te = 0.0;
+#pragma unroll
+    for (int i = 0; i < Cfg::kWarps; ++i) {
+      ts += s_part[i][0];
+      te += s_part[i][1];
+    }
+    a.out_partials[2 * blockIdx.x] = ts;
+    a.out_partials[2 * blockIdx.x + 1] = te;
+    __threadfence();
+    s_last = atomicAdd(a.ticket, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (s_last && warp == 0) {
+    __threadfence();
+    qe_final_sum(a.out_partials, static_cast<int>(gridDim.x), a.out);
+    if (lane == 0) *a.ticket = 0u;
+  }
+}
+
+// The same result for an empty X (no CTA to finish): {0, 0, +inf}.  One warp.
+__global__ void quant_error_empty_kernel(const double* __restrict__ partials, double* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait();
+  qe_final_sum(partials, 0, out);
 }
 
 // Rotated amax: every CTA writes max |fl(y)| over its warps' ranges to partials[blockIdx.x].

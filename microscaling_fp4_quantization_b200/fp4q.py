@@ -40,6 +40,7 @@ _SIGS = {
     "fp4q_amax": (_int, [_vp, _vp, _i64, _i64, _vp, _vp]),
     "fp4q_dequantize": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _int, _vp, _vp]),
     "fp4q_rotate_quantize_nvfp4_dynamic_noalloc": (_int, [_vp, _i64, _i64, _int, _vp, _vp, _vp, _vp]),
+    "fp4q_quant_error": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp]),
     "fp4q_device_status": (_int, []),
     "fp4q_status_string": (ctypes.c_char_p, [_int]),
     "fp4q_last_cuda_error": (ctypes.c_char_p, []),
@@ -156,6 +157,12 @@ def fp4q_rotate_quantize_nvfp4_dynamic_noalloc(x, M: int, K: int, hadamard_block
            "fp4q_rotate_quantize_nvfp4_dynamic_noalloc")
 
 
+def fp4q_quant_error(plan: Plan, x, M: int, K: int, tensor_scale, out_f64, stream=None) -> None:
+    """out_f64: device float64 [3] <- {signal energy, error energy, QSNR dB}."""
+    _check(_lib.fp4q_quant_error(plan.handle, _ptr(x), M, K, _ptr(tensor_scale), _ptr(out_f64), _stream(stream)),
+           "fp4q_quant_error")
+
+
 def fp4q_device_status() -> int:
     return _lib.fp4q_device_status()
 
@@ -196,3 +203,18 @@ def rotate_quantize(plan: Plan, x, tensor_scale=None, stream=None) -> Tuple[obje
         ts = tensor_scale
     fp4q_rotate_quantize(plan, x, M, K, codes, scales, ts if plan.fmt == FP4Q_NVFP4 else None, stream)
     return codes, scales, ts
+
+
+def quant_error(plan: Plan, x, tensor_scale=None, stream=None):
+    """x: bf16 CUDA tensor [M, K] -> (signal, error, qsnr_db) as Python floats (synchronises)."""
+    import torch
+    if x.dtype != torch.bfloat16 or not x.is_cuda or x.dim() != 2 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous 2-D bf16 CUDA tensor")
+    M, K = x.shape
+    out = torch.empty(3, dtype=torch.float64, device=x.device)
+    ts = tensor_scale
+    if plan.fmt == FP4Q_NVFP4 and ts is None:
+        ts = torch.empty(1, dtype=torch.float32, device=x.device)
+    fp4q_quant_error(plan, x, M, K, ts, out, stream)
+    s, e, q = out.tolist()
+    return s, e, q

@@ -50,7 +50,7 @@ def test_plan_validation_without_gpu(F):
             F.fp4q_plan_create(*args)
         assert e.value.status == F.FP4Q_ERR_UNSUPPORTED, args
     assert F.raw_call("fp4q_plan_create", None, 0, 32, 32, 0) == F.FP4Q_ERR_ARG
-    # MX plans allocate nothing on the device, so they can be made on a CPU-only machine
+    # MX plans need a device only for the error pass's scratch, so they can be made on a CPU-only machine
     p = F.fp4q_plan_create(F.FP4Q_MXFP4, 32, 32, F.FP4Q_SCALE_FLOOR_OCP)
     F.fp4q_plan_destroy(p)
     assert F.raw_call("fp4q_plan_destroy", None) == F.FP4Q_OK
@@ -86,6 +86,18 @@ def test_call_validation_without_gpu(F):
     assert dq(p.handle, A, A, None, 4, 128, 0, A + 4, None) == F.FP4Q_ERR_ALIGN
     am = lambda *a: F.raw_call("fp4q_amax", *a)
     assert am(p.handle, A, 4, 128, A, None) == F.FP4Q_ERR_UNSUPPORTED            # MX plan
+    qe = lambda *a: F.raw_call("fp4q_quant_error", *a)
+    assert qe(None, A, 4, 128, None, A, None) == F.FP4Q_ERR_ARG
+    assert qe(p.handle, A, 4, 96, None, A, None) == F.FP4Q_ERR_SHAPE
+    assert qe(p.handle, A, 4, 128, None, None, None) == F.FP4Q_ERR_ARG           # no output
+    assert qe(p.handle, None, 4, 128, None, A, None) == F.FP4Q_ERR_ARG
+    assert qe(p.handle, A + 8, 4, 128, None, A, None) == F.FP4Q_ERR_ALIGN
+    assert qe(p.handle, A, 4, 128, None, A + 4, None) == F.FP4Q_ERR_ALIGN         # out: 8 bytes
+    # an MX plan made without a CUDA device holds no scratch for the error pass (with a
+    # device the call would get past validation, so it is not made with the fake address)
+    from conftest import gpu_available
+    if not gpu_available():
+        assert qe(p.handle, A, 4, 128, None, A, None) == F.FP4Q_ERR_UNSUPPORTED
     F.fp4q_plan_destroy(p)
 
 
