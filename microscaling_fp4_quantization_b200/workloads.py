@@ -163,3 +163,26 @@ BY_NAME = {w.name: w for w in ALL}
 
 def lcm(a: int, b: int) -> int:
     return a * b // math.gcd(a, b)
+
+
+def random_sign_mask(K: int, seed: int) -> np.ndarray:
+    """Random per-channel sign bits for a randomised Hadamard rotation: ceil(K / 32) uint32
+    words from ``numpy.random.default_rng(seed)``, bits at or above K cleared.  (Bit k of
+    word k // 32 set means channel k is negated; the library and the oracle each read the
+    bits themselves.)"""
+    n = (K + 31) // 32
+    w = np.random.default_rng(seed).integers(0, 1 << 32, size=n, dtype=np.uint64).astype(np.uint32)
+    if K % 32:
+        w[-1] &= np.uint32((1 << (K % 32)) - 1)
+    return w
+
+
+def synthetic_weights(N: int, K: int, seed: int) -> np.ndarray:
+    """Synthetic weight matrix W (N x K bf16 bit patterns): Laplace(0, 0.02) entries, the
+    heavy-tailed shape the error analysis assigns to LLM weights, with 0.5 % of the input
+    channels scaled by 10 (outlier channels)."""
+    rng = np.random.default_rng(seed)
+    cols = rng.choice(K, max(1, round(0.005 * K)), replace=False)
+    w = rng.laplace(0.0, 0.02, size=(N, K)).astype(np.float32)
+    w[:, cols] *= np.float32(10.0)
+    return f32_to_bf16_bits(w)

@@ -31,7 +31,10 @@ Sources (page title and section):
 
 Readings where the pages are silent:
   * Hadamard: Sylvester construction, natural order, orthonormal 1/sqrt(b), applied to
-    every contiguous b-block of a row (the GEMM reduction axis), no random signs.
+    every contiguous b-block of a row (the GEMM reduction axis).  By default no random
+    signs; an optional per-channel sign vector s (QuaRot-style randomised Hadamard, "wie in
+    QuIP/QuaRot", [BG] 2. Methodik) is applied to the channels before the block rotation,
+    the same s on the activations online and in the weights offline.
   * E2M1: magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}; round to nearest, ties to the even
     code; saturate at 6; the sign bit is the sign of the rotated value.
   * MX scale X = 2^e, stored as the E8M0 byte e + 127, e clamped to [-127, 127]:
@@ -94,25 +97,44 @@ def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
     return u.view(np.float32).astype(np.float64)
 
 
-def rotate(x_bits: np.ndarray, b: int) -> np.ndarray:
-    """y[r, kb*b + j] = (1/sqrt(b)) * sum_l x[r, kb*b + l] * H_b[l, j], in float64.
+def sign_vector(mask_words: np.ndarray, K: int) -> np.ndarray:
+    """Per-channel signs from a bit mask: channel k is negated when bit (k mod 32) of word
+    k // 32 is set.  Returns float64 +-1 of length K."""
+    w = np.asarray(mask_words, np.uint32)
+    if w.size * 32 < K:
+        raise ValueError("the sign mask holds fewer than K bits")
+    k = np.arange(K)
+    bit = (w[k // 32] >> (k % 32).astype(np.uint32)) & np.uint32(1)
+    return np.where(bit == 1, -1.0, 1.0)
 
-    An explicit matrix product with the Sylvester matrix (not a fast transform)."""
+
+def rotate(x_bits: np.ndarray, b: int, signs=None) -> np.ndarray:
+    """y[r, kb*b + j] = (1/sqrt(b)) * sum_l s[kb*b + l] x[r, kb*b + l] H_b[l, j], in float64.
+
+    An explicit matrix product with the Sylvester matrix (not a fast transform).  ``signs``
+    (length K, +-1, or None for all +1) is the random diagonal of a QuaRot-style
+    randomised Hadamard transform, applied to the channels before the block rotation, so
+    that the rotation is Q = diag(s) (I kron H_b / sqrt(b))."""
     x = bf16_to_f64(x_bits)
     M, K = x.shape
     if K % b:
         raise ValueError("K must be a multiple of the Hadamard block")
+    if signs is not None:
+        x = x * np.asarray(signs, np.float64)[None, :]
     H = sylvester_hadamard(b).astype(np.float64)
     y = (x.reshape(M * (K // b), b) @ H) / math.sqrt(b)
     return y.reshape(M, K)
 
 
-def unrotate(y: np.ndarray, b: int) -> np.ndarray:
+def unrotate(y: np.ndarray, b: int, signs=None) -> np.ndarray:
     """Inverse rotation.  H_b / sqrt(b) is symmetric and orthogonal, so it is its own
-    inverse: the same product again."""
+    inverse: the same product again, then the signs again (Q^-1 = Q^T)."""
     M, K = y.shape
     H = sylvester_hadamard(b).astype(np.float64)
-    return ((np.asarray(y, np.float64).reshape(M * (K // b), b) @ H) / math.sqrt(b)).reshape(M, K)
+    x = ((np.asarray(y, np.float64).reshape(M * (K // b), b) @ H) / math.sqrt(b)).reshape(M, K)
+    if signs is not None:
+        x = x * np.asarray(signs, np.float64)[None, :]
+    return x
 
 
 # ----------------------------------------------------------------------------------
@@ -256,19 +278,19 @@ def check_plan(fmt: int, group: int, block: int, rule: int) -> None:
     sylvester_hadamard(block)
 
 
-def rotated_amax(x_bits: np.ndarray, block: int, chunk_rows: int = 512) -> np.float32:
+def rotated_amax(x_bits: np.ndarray, block: int, chunk_rows: int = 512, signs=None) -> np.float32:
     """max |y| over the whole tensor, taken on the fp32 rotated values (row chunks keep the
     fp64 intermediate small)."""
     m = np.float32(0)
     for r in range(0, x_bits.shape[0], chunk_rows):
-        y32 = rotate(x_bits[r:r + chunk_rows], block).astype(np.float32)
+        y32 = rotate(x_bits[r:r + chunk_rows], block, signs).astype(np.float32)
         if y32.size:
             m = max(m, np.float32(np.max(np.abs(y32))))
     return np.float32(m)
 
 
 def rotate_quantize(x_bits: np.ndarray, fmt: int, group: int, block: int, rule: int,
-                    tensor_scale=None) -> dict:
+                    tensor_scale=None, signs=None) -> dict:
     """Rotate then quantize X (M x K bf16 bit patterns).
 
     For NVFP4 ``tensor_scale`` is the fp32 s_g (the static rule needs it; the dynamic
@@ -281,7 +303,7 @@ def rotate_quantize(x_bits: np.ndarray, fmt: int, group: int, block: int, rule: 
     M, K = x_bits.shape
     if K % group or K % block:
         raise ValueError("K must be a multiple of the group and of the block")
-    y64 = rotate(x_bits, block)
+    y64 = rotate(x_bits, block, signs)
     y32 = y64.astype(np.float32)                     # one rounding to fp32
     yg = y32.reshape(M, K // group, group)
     A32 = np.max(np.abs(yg), axis=2) if K else np.zeros((M, 0), np.float32)
@@ -324,7 +346,7 @@ def rotate_quantize(x_bits: np.ndarray, fmt: int, group: int, block: int, rule: 
 
 
 def dequantize(codes: np.ndarray, scales: np.ndarray, fmt: int, group: int, block: int,
-               tensor_scale=None, unrotate_back: bool = False) -> np.ndarray:
+               tensor_scale=None, unrotate_back: bool = False, signs=None) -> np.ndarray:
     """codes x block scale (x tensor scale), optionally rotated back.
 
     MX: x = q * 2^(byte - 127), exact.  NV: x = fp32(q * fp32(E4M3(byte) * s_g)).
@@ -341,7 +363,7 @@ def dequantize(codes: np.ndarray, scales: np.ndarray, fmt: int, group: int, bloc
         x = (q.reshape(M, K // group, group).astype(np.float32) * S32[..., None]).astype(np.float32)
     x = x.reshape(M, K)
     if unrotate_back:
-        return unrotate(x.astype(np.float64), block)
+        return unrotate(x.astype(np.float64), block, signs)
     return x
 
 
@@ -403,7 +425,7 @@ def flags(res: dict, tol: float = 1e-5):
 # ----------------------------------------------------------------------------------
 
 def quant_error(x_bits: np.ndarray, fmt: int, group: int, block: int, rule: int,
-                tensor_scale=None, chunk_rows: int = 512) -> dict:
+                tensor_scale=None, chunk_rows: int = 512, signs=None) -> dict:
     """Signal and error energy of rotate + quantize on X, and the QSNR.
 
     signal = sum of y^2 and noise = sum of (y - yhat)^2 over all elements, where y are the
@@ -420,11 +442,11 @@ def quant_error(x_bits: np.ndarray, fmt: int, group: int, block: int, rule: int,
     if fmt == NVFP4 and tensor_scale is None:
         if rule != SCALE_NV_DYNAMIC:
             raise ValueError("the static NV rule needs the tensor scale")
-        tensor_scale = nv_tensor_scale(rotated_amax(x_bits, block))
+        tensor_scale = nv_tensor_scale(rotated_amax(x_bits, block, signs=signs))
     signal = 0.0
     noise = 0.0
     for r in range(0, M, chunk_rows):
-        res = rotate_quantize(x_bits[r:r + chunk_rows], fmt, group, block, rule, tensor_scale)
+        res = rotate_quantize(x_bits[r:r + chunk_rows], fmt, group, block, rule, tensor_scale, signs)
         y = res["y64"]
         m = y.shape[0]
         q = e2m1_decode(unpack_nibbles(res["codes"])).reshape(m, K // group, group)

@@ -202,3 +202,41 @@ def test_qsnr_variant_without_mistake_passes(monkeypatch):
     for pin in (qpins.test_energies_match_the_unrotated_domain, qpins.test_hand_worked_mx_group,
                 qpins.test_hand_worked_nv_group):
         pin()
+
+
+# ---- randomised rotation (pins in test_oracle_signs.py)
+
+import test_oracle_signs as spins  # noqa: E402
+
+_orig_sign_vector = core.sign_vector
+
+
+def rotate_signs_after(x_bits, b, signs=None):
+    """Applies the signs to the rotated values instead of the channels."""
+    y = _orig_rotate(x_bits, b)
+    return y if signs is None else y * np.asarray(signs, np.float64)[None, :]
+
+
+def rotate_signs_ignored(x_bits, b, signs=None):
+    return _orig_rotate(x_bits, b)
+
+
+def sign_vector_msb_first(mask_words, K):
+    w = np.asarray(mask_words, np.uint32)
+    k = np.arange(K)
+    bit = (w[k // 32] >> (31 - k % 32).astype(np.uint32)) & np.uint32(1)
+    return np.where(bit == 1, -1.0, 1.0)
+
+
+SIGN_MUTATIONS = [
+    ("rotate", rotate_signs_after, [spins.test_rotated_basis_vectors]),
+    ("rotate", rotate_signs_ignored, [spins.test_rotated_basis_vectors, spins.test_signs_reach_the_codes_and_the_error]),
+    ("sign_vector", sign_vector_msb_first, [spins.test_sign_mask_bit_layout]),
+]
+
+
+@pytest.mark.parametrize("name,fn,catchers", SIGN_MUTATIONS, ids=[m[1].__name__ for m in SIGN_MUTATIONS])
+def test_sign_pins_catch_planted_mistake(monkeypatch, name, fn, catchers):
+    patch(monkeypatch, name, fn)
+    for catcher in catchers:
+        assert fails(catcher), f"{catcher.__name__} missed {fn.__name__}"
