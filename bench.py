@@ -295,6 +295,11 @@ def run_gpu(args):
                            "bytes_per_call": nbytes}
         extra["dynamic_mode"]["note"] = "reads X twice (amax pass, then quantize); bytes are the algorithmic ones"
 
+    # the randomised rotation (per-channel random signs; butterfly kernel) on the same workload
+    if rank == 0:
+        extra["signed_rotation"] = time_signed(torch, F, w, xs, codes, scales, ts if is_nv else None, stream, peak,
+                                               max(50, min(args.steps, 400)))
+
     # the quantization-error pass (signal / error energies and QSNR) on the same workload
     if rank == 0:
         extra["quant_error"] = time_quant_error(torch, F, w, plan, xs, ts if is_nv else None, stream, peak,
@@ -425,6 +430,34 @@ def run_kernel_only(args):
     torch.cuda.synchronize()
     assert F.fp4q_device_status() == F.FP4Q_OK
     print(f"kernel-only: {w.name} M={w.M} K={w.K} launches={args.warmup + args.steps}", flush=True)
+
+
+def time_signed(torch, F, w, xs, codes, scales, ts, stream, peak, steps):
+    """fp4q_rotate_quantize with a plan carrying per-channel random signs (seeded mask): the
+    same bytes as the plain call, on the butterfly kernel."""
+    M, K = w.M, w.K
+    plan = F.fp4q_plan_create(w.fmt, w.group, w.block, w.rule)
+    mask = torch.from_numpy(W.random_sign_mask(K, 1234).view(np.int32)).to(xs[0].device)
+    F.fp4q_plan_set_signs(plan, mask, K)
+
+    def launch(i):
+        F.fp4q_rotate_quantize(plan, xs[i], M, K, codes[i], scales[i], ts, stream=torch.cuda.current_stream())
+
+    with torch.cuda.stream(stream):
+        g, g_rem, reps = time_graph_steps(torch, launch, len(xs), steps, 3, stream)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        a1.record(stream)
+    torch.cuda.synchronize()
+    us = a0.elapsed_time(a1) * 1e3 / steps
+    nbytes = w.bytes_per_call()
+    gbs = nbytes / us / 1e3
+    return {"us_per_call": round(us, 3), "GBps": round(gbs, 1), "pct_of_hbm_peak": round(100 * gbs / peak, 2),
+            "bytes_per_call": nbytes, "kernel": "butterfly"}
 
 
 def time_quant_error(torch, F, w, plan, xs, ts, stream, peak, steps):

@@ -117,6 +117,24 @@ fp4q_status fp4q_plan_set_kernel(fp4q_plan plan, int kernel);
  * call using the plan is still running on the device. */
 fp4q_status fp4q_plan_destroy(fp4q_plan plan);
 
+/* Per-channel random signs for the rotation (a randomised Hadamard transform, "wie in
+ * QuIP/QuaRot": "Bridging the Gap Between Promise and Performance for Microscaling FP4
+ * Quantization", Technische Zusammenfassung, 2. Methodik).  With signs s the rotation of
+ * every row is Q = diag(s) (I kron H_b / sqrt(b)): channel k is negated before the block
+ * rotation.  The same s must be used on the activations (online) and on the weights (offline,
+ * rotate + quantize of W with the same plan settings), so that (X Q)(W Q)^T = X W^T.
+ *
+ * signs: device uint32 [ceil(K / 32)]; bit (k mod 32) of word k / 32 set negates channel k.
+ * Borrowed: the caller keeps the array alive and unchanged while the plan uses it.  NULL
+ * clears the signs.  K: the row length the signs are for; a multiple of max(g, b), at most
+ * 2^34.  Afterwards every call on the plan must have this K (FP4Q_ERR_SHAPE otherwise), and
+ * fp4q_rotate_quantize(_dump), fp4q_amax, fp4q_quant_error and fp4q_dequantize (with
+ * unrotate) all use the signs.  A plan with signs runs the butterfly kernel: it returns
+ * FP4Q_ERR_UNSUPPORTED when the plan is forced to FP4Q_KERNEL_TENSOR_CORE, and
+ * fp4q_plan_set_kernel refuses TENSOR_CORE while signs are set.  signs must be 4-byte
+ * aligned. */
+fp4q_status fp4q_plan_set_signs(fp4q_plan plan, const uint32_t* signs, int64_t K);
+
 /* Rotate and quantize X in one pass over HBM (steps 1-5 above).
  * x_bf16: device bf16 [M][K]; codes_out: device uint8 [M][K/2]; scales_out: device
  * uint8 [M][K/g]; tensor_scale: device fp32 — NV static: read; NV dynamic: written with

@@ -23,6 +23,8 @@ struct fp4q_plan_s {
   float* partials; // NV plans: per-CTA rotated amaxima (device)
   int n_partials;
   int kernel;      // fp4q_kernel
+  const uint32_t* signs; // per-channel random signs (device, borrowed; null: none)
+  int64_t signs_K;       // the row length K the signs are for
   double* err_partials;  // fp4q_quant_error scratch (device; null without a device): per-CTA signal and
                          // error energy, then a ticket counter
   int n_err_partials;    // CTAs those hold room for
@@ -116,9 +118,18 @@ fp4q_status with_block(int b, F&& f) {
   }
 }
 
+// The kernels' view of the plan's channel signs for a configuration with E-element units.
 template <class Cfg>
-fp4q_status launch_rq(RQArgs a, int64_t n_elems, cudaStream_t stream) {
+ChannelSigns channel_signs(const uint32_t* mask, int64_t K) {
+  if (!mask) return ChannelSigns{nullptr, 1, 0};
+  const int upr = static_cast<int>(K / Cfg::kE);
+  return ChannelSigns{mask, upr, static_cast<int>(Cfg::kUnitsPerStage % upr)};
+}
+
+template <class Cfg>
+fp4q_status launch_rq(RQArgs a, int64_t n_elems, cudaStream_t stream, int64_t K = 0) {
   a.n_units = n_elems / Cfg::kE;
+  a.signs = channel_signs<Cfg>(a.signs.mask, K);
   auto kernel = rotate_quantize_kernel<Cfg>;
   KernelInfo ki;
   fp4q_status st = kernel_info(kernel, Cfg::kSmemBytes, Cfg::kThreads, &ki);
@@ -207,7 +218,7 @@ fp4q_status launch_mma(const uint16_t* x, int64_t n_elems, const RQArgs& ra, cud
 constexpr int64_t kMmaMinElems = int64_t(1) << 22;
 bool mma_capable(fp4q_plan p) { return p->block >= 16 && p->block >= p->group; }
 bool use_mma(fp4q_plan p, int64_t n_elems) {
-  if (!mma_capable(p)) return false;
+  if (!mma_capable(p) || p->signs) return false;   // channel signs: butterfly kernel only
   if (p->kernel == FP4Q_KERNEL_TENSOR_CORE) return true;
   return p->kernel == FP4Q_KERNEL_AUTO && n_elems >= kMmaMinElems;
 }
@@ -234,7 +245,7 @@ fp4q_status amax_grid(int b, int* n) {
 template <class Cfg>
 fp4q_status launch_amax_cfg(fp4q_plan p, const uint16_t* x, int64_t n_elems, cudaStream_t stream) {
   cudaError_t e = launch_pdl(rotated_amax_kernel<Cfg>, dim3(p->n_partials), dim3(Cfg::kThreads), Cfg::kSmemBytes,
-                             stream, x, n_elems / Cfg::kE, p->partials);
+                             stream, x, n_elems / Cfg::kE, p->partials, channel_signs<Cfg>(p->signs, p->signs_K));
   if (e != cudaSuccess) return cuda_fail(e, "amax launch");
   return FP4Q_OK;
 }
@@ -248,6 +259,7 @@ fp4q_status launch_amax(fp4q_plan p, const uint16_t* x, int64_t n_elems, cudaStr
 
 fp4q_status check_shape(fp4q_plan p, int64_t M, int64_t K) {
   if (M < 0 || K < 0) return FP4Q_ERR_SHAPE;
+  if (p->signs && K != p->signs_K) return FP4Q_ERR_SHAPE;   // the signs are for rows of signs_K
   if (K % p->unit != 0) return FP4Q_ERR_SHAPE;  // unit = lcm(group, block) for powers of two
   if (M > 0 && K > 0 && M > (int64_t(1) << 40) / K) return FP4Q_ERR_SHAPE;
   return FP4Q_OK;
@@ -275,6 +287,7 @@ fp4q_status rotate_quantize_impl(fp4q_plan p, const void* x, int64_t M, int64_t 
   a.partials = p->partials;
   a.n_partials = p->n_partials;
   a.y_dump = y_out;
+  a.signs = ChannelSigns{p->signs, 1, 0};
   if (p->format == FP4Q_NVFP4 && p->rule == FP4Q_SCALE_NV_DYNAMIC) {
     st = launch_amax(p, a.x, n, s);
     if (st != FP4Q_OK) return st;
@@ -312,14 +325,14 @@ fp4q_status rotate_quantize_impl(fp4q_plan p, const void* x, int64_t M, int64_t 
     if (p->format == FP4Q_MXFP4) {
       switch (p->rule) {
         case FP4Q_SCALE_FLOOR_OCP:
-          return dump ? launch_rq<RQConfig<kMX, B, kRuleFloor, true>>(a, n, s)
-                      : launch_rq<RQConfig<kMX, B, kRuleFloor, false>>(a, n, s);
+          return dump ? launch_rq<RQConfig<kMX, B, kRuleFloor, true>>(a, n, s, K)
+                      : launch_rq<RQConfig<kMX, B, kRuleFloor, false>>(a, n, s, K);
         case FP4Q_SCALE_CEIL_NOCLIP:
-          return dump ? launch_rq<RQConfig<kMX, B, kRuleCeil, true>>(a, n, s)
-                      : launch_rq<RQConfig<kMX, B, kRuleCeil, false>>(a, n, s);
+          return dump ? launch_rq<RQConfig<kMX, B, kRuleCeil, true>>(a, n, s, K)
+                      : launch_rq<RQConfig<kMX, B, kRuleCeil, false>>(a, n, s, K);
         case FP4Q_SCALE_OAS:
-          return dump ? launch_rq<RQConfig<kMX, B, kRuleOas, true>>(a, n, s)
-                      : launch_rq<RQConfig<kMX, B, kRuleOas, false>>(a, n, s);
+          return dump ? launch_rq<RQConfig<kMX, B, kRuleOas, true>>(a, n, s, K)
+                      : launch_rq<RQConfig<kMX, B, kRuleOas, false>>(a, n, s, K);
         default: return FP4Q_ERR_UNSUPPORTED;
       }
     }
@@ -327,16 +340,16 @@ fp4q_status rotate_quantize_impl(fp4q_plan p, const void* x, int64_t M, int64_t 
     const bool u32 = n % 32 == 0;
     if (p->rule == FP4Q_SCALE_NV_DYNAMIC) {
       if (u32)
-        return dump ? launch_rq<RQConfig<kNV, B, kRuleNvDynamic, true, 32>>(a, n, s)
-                    : launch_rq<RQConfig<kNV, B, kRuleNvDynamic, false, 32>>(a, n, s);
-      return dump ? launch_rq<RQConfig<kNV, B, kRuleNvDynamic, true, 16>>(a, n, s)
-                  : launch_rq<RQConfig<kNV, B, kRuleNvDynamic, false, 16>>(a, n, s);
+        return dump ? launch_rq<RQConfig<kNV, B, kRuleNvDynamic, true, 32>>(a, n, s, K)
+                    : launch_rq<RQConfig<kNV, B, kRuleNvDynamic, false, 32>>(a, n, s, K);
+      return dump ? launch_rq<RQConfig<kNV, B, kRuleNvDynamic, true, 16>>(a, n, s, K)
+                  : launch_rq<RQConfig<kNV, B, kRuleNvDynamic, false, 16>>(a, n, s, K);
     }
     if (u32)
-      return dump ? launch_rq<RQConfig<kNV, B, kRuleNvStatic, true, 32>>(a, n, s)
-                  : launch_rq<RQConfig<kNV, B, kRuleNvStatic, false, 32>>(a, n, s);
-    return dump ? launch_rq<RQConfig<kNV, B, kRuleNvStatic, true, 16>>(a, n, s)
-                : launch_rq<RQConfig<kNV, B, kRuleNvStatic, false, 16>>(a, n, s);
+      return dump ? launch_rq<RQConfig<kNV, B, kRuleNvStatic, true, 32>>(a, n, s, K)
+                  : launch_rq<RQConfig<kNV, B, kRuleNvStatic, false, 32>>(a, n, s, K);
+    return dump ? launch_rq<RQConfig<kNV, B, kRuleNvStatic, true, 16>>(a, n, s, K)
+                : launch_rq<RQConfig<kNV, B, kRuleNvStatic, false, 16>>(a, n, s, K);
   });
 }
 
@@ -381,6 +394,7 @@ fp4q_status qe_grid(int format, int block, int rule, int* n) {
 template <class Cfg>
 fp4q_status launch_qe(fp4q_plan p, QEArgs a, int64_t n_elems, double* out, cudaStream_t stream) {
   a.n_units = n_elems / Cfg::kE;
+  a.signs = channel_signs<Cfg>(p->signs, p->signs_K);
   auto kernel = quant_error_kernel<Cfg>;
   KernelInfo ki;
   fp4q_status st = kernel_info(kernel, Cfg::kSmemBytes, Cfg::kThreads, &ki);
@@ -431,7 +445,8 @@ fp4q_status noalloc_scratch(float** out) {
 template <class Cfg>
 fp4q_status noalloc_amax_launch(const uint16_t* x, int64_t n_elems, float* partials, int n_partials,
                                 cudaStream_t stream) {
-  rotated_amax_kernel<Cfg><<<n_partials, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(x, n_elems / Cfg::kE, partials);
+  rotated_amax_kernel<Cfg><<<n_partials, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(x, n_elems / Cfg::kE, partials,
+                                                                                  ChannelSigns{nullptr, 1, 0});
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "amax launch");
   return FP4Q_OK;
@@ -479,6 +494,7 @@ fp4q_status fp4q_rotate_quantize_nvfp4_dynamic_noalloc(const void* x_bf16, int64
   a.partials = partials;
   a.n_partials = n_partials;
   a.y_dump = nullptr;
+  a.signs = ChannelSigns{nullptr, 1, 0};
   return with_block(hadamard_block, [&]<int B>() -> fp4q_status {
     if (n % 32 == 0) {
       fp4q_status r = noalloc_amax_launch<AmaxCfg<B, 32>>(x, n, partials, n_partials, s);
@@ -520,6 +536,8 @@ fp4q_status fp4q_plan_create(fp4q_plan* out, int format, int group, int hadamard
   p->kernel = FP4Q_KERNEL_AUTO;
   p->err_partials = nullptr;
   p->n_err_partials = 0;
+  p->signs = nullptr;
+  p->signs_K = 0;
   fp4q_status st = FP4Q_OK;
   if (format == FP4Q_NVFP4) {
     cudaError_t e = cudaGetDevice(&p->device);
@@ -561,8 +579,23 @@ fp4q_status fp4q_plan_set_kernel(fp4q_plan plan, int kernel) {
   if (!valid_plan(plan)) return FP4Q_ERR_ARG;
   if (kernel != FP4Q_KERNEL_AUTO && kernel != FP4Q_KERNEL_BUTTERFLY && kernel != FP4Q_KERNEL_TENSOR_CORE)
     return FP4Q_ERR_ARG;
-  if (kernel == FP4Q_KERNEL_TENSOR_CORE && !mma_capable(plan)) return FP4Q_ERR_UNSUPPORTED;
+  if (kernel == FP4Q_KERNEL_TENSOR_CORE && (!mma_capable(plan) || plan->signs)) return FP4Q_ERR_UNSUPPORTED;
   plan->kernel = kernel;
+  return FP4Q_OK;
+}
+
+fp4q_status fp4q_plan_set_signs(fp4q_plan plan, const uint32_t* signs, int64_t K) {
+  if (!valid_plan(plan)) return FP4Q_ERR_ARG;
+  if (!signs) {
+    plan->signs = nullptr;
+    plan->signs_K = 0;
+    return FP4Q_OK;
+  }
+  if (K <= 0 || K % plan->unit != 0 || K > (int64_t(1) << 34)) return FP4Q_ERR_SHAPE;
+  if (!aligned(signs, 4)) return FP4Q_ERR_ALIGN;
+  if (plan->kernel == FP4Q_KERNEL_TENSOR_CORE) return FP4Q_ERR_UNSUPPORTED;
+  plan->signs = signs;
+  plan->signs_K = K;
   return FP4Q_OK;
 }
 
@@ -667,12 +700,15 @@ fp4q_status fp4q_dequantize(fp4q_plan plan, const void* codes, const void* scale
   const uint8_t* c = static_cast<const uint8_t*>(codes);
   const uint8_t* sc = static_cast<const uint8_t*>(scales);
   st = with_block(plan->block, [&]<int B>() -> fp4q_status {
+    // the dequantize kernel's unit is the plan's, E = max(g, b)
+    const ChannelSigns dsg = plan->signs ? ChannelSigns{plan->signs, static_cast<int>(plan->signs_K / plan->unit), 0}
+                                         : ChannelSigns{nullptr, 1, 0};
     if (plan->format == FP4Q_MXFP4) {
-      if (unrotate) dequantize_kernel<kMX, B, true><<<grid, 128, 0, s>>>(c, sc, tensor_scale, n_units, out_f32);
-      else dequantize_kernel<kMX, B, false><<<grid, 128, 0, s>>>(c, sc, tensor_scale, n_units, out_f32);
+      if (unrotate) dequantize_kernel<kMX, B, true><<<grid, 128, 0, s>>>(c, sc, tensor_scale, n_units, out_f32, dsg);
+      else dequantize_kernel<kMX, B, false><<<grid, 128, 0, s>>>(c, sc, tensor_scale, n_units, out_f32, dsg);
     } else {
-      if (unrotate) dequantize_kernel<kNV, B, true><<<grid, 128, 0, s>>>(c, sc, tensor_scale, n_units, out_f32);
-      else dequantize_kernel<kNV, B, false><<<grid, 128, 0, s>>>(c, sc, tensor_scale, n_units, out_f32);
+      if (unrotate) dequantize_kernel<kNV, B, true><<<grid, 128, 0, s>>>(c, sc, tensor_scale, n_units, out_f32, dsg);
+      else dequantize_kernel<kNV, B, false><<<grid, 128, 0, s>>>(c, sc, tensor_scale, n_units, out_f32, dsg);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");

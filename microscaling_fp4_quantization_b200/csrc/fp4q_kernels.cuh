@@ -131,6 +131,15 @@ struct RQConfig {
   static constexpr float kC = inv_sqrt_block(B);
 };
 
+// Per-channel random signs of a randomised Hadamard rotation (mask == nullptr: none).  Bit
+// (k mod 32) of mask[k / 32] set negates channel k; a unit of E elements sits at channel
+// (u mod upr) * E of its row, upr = K / E; stage_step = (units per stage) mod upr.
+struct ChannelSigns {
+  const uint32_t* mask;
+  int upr;
+  int stage_step;
+};
+
 struct RQArgs {
   const uint16_t* x;       // bf16 [n_units * E]
   int64_t n_units;
@@ -140,6 +149,7 @@ struct RQArgs {
   const float* partials;   // NV dynamic: per-CTA rotated amaxima from the amax pass
   int n_partials;
   float* y_dump;           // [n_units * E] when dumping
+  ChannelSigns signs;      // per-channel random signs (mask nullptr: none)
 };
 
 // Per-lane constants of the chunk XOR: tau, and for each of tau's (at most three) bits the
@@ -171,17 +181,70 @@ __device__ __forceinline__ uint32_t chunk_sign_mask(const LaneXor& lx, int j) {
   return m;
 }
 
+// The unit's E sign bits, as E/32 words (E = 16: the low 16 bits of one word).
+template <int E>
+struct UnitSigns {
+  uint32_t w[E >= 32 ? E / 32 : 1];
+};
+
+template <int E>
+__device__ __forceinline__ UnitSigns<E> unit_signs(const uint32_t* mask, int cu) {
+  UnitSigns<E> m;
+  const int c0 = cu * E;
+  if constexpr (E >= 32) {
+#pragma unroll
+    for (int i = 0; i < E / 32; ++i) m.w[i] = __ldg(mask + (c0 >> 5) + i);
+  } else {
+    m.w[0] = (__ldg(mask + (c0 >> 5)) >> (c0 & 31)) & 0xFFFFu;
+  }
+  return m;
+}
+
+// XOR masks that negate the bf16 elements of one 16-byte chunk (8 elements, word i holding
+// elements 2i and 2i+1) whose sign bits are set in byte `mb`.
+__device__ __forceinline__ uint4 chunk_sign_xor(uint32_t mb) {
+  uint4 r;
+  r.x = ((mb & 0x01u) << 15) | ((mb & 0x02u) << 30);
+  r.y = ((mb & 0x04u) << 13) | ((mb & 0x08u) << 28);
+  r.z = ((mb & 0x10u) << 11) | ((mb & 0x20u) << 26);
+  r.w = ((mb & 0x40u) << 9) | ((mb & 0x80u) << 24);
+  return r;
+}
+
+// Sign byte of original chunk q = j ^ tau of a unit (tau only touches the low three bits,
+// so the word is one of two known at compile time).
+template <int E>
+__device__ __forceinline__ uint32_t unit_sign_byte(const UnitSigns<E>& m, int j, int tau) {
+  const int q = j ^ tau;
+  uint32_t w;
+  if constexpr (E >= 64) {
+    const uint32_t a = m.w[(j >> 2)], b = m.w[(j >> 2) ^ 1];
+    w = ((j ^ q) & 4) ? b : a;
+  } else {
+    w = m.w[0];
+  }
+  return (w >> (8 * (q & 3))) & 0xFFu;
+}
+
 // Load one unit from shared memory (chunk j read from position j ^ tau), widen bf16 to
 // fp32 and run the butterfly of H_B on every B-block (unnormalised sums).  p[k] holds the
 // pair (element 2k, element 2k + 1).  The first stage (distance 1) is taken straight from
 // the bf16 pair; the others run on packed pairs, pair k against pair k + h/2.  Every element
 // sees the same additions, in the same order, as in the scalar butterfly; for B >= 2 the odd
 // elements come out negated (see bf16_pair_butterfly_oddneg).
-template <int B, int E>
-__device__ __forceinline__ void load_rotate_unit(uint32_t saddr, int tau, f32x2 (&p)[E / 2]) {
+template <int B, int E, bool SIGNED = false>
+__device__ __forceinline__ void load_rotate_unit(uint32_t saddr, int tau, f32x2 (&p)[E / 2],
+                                                 const UnitSigns<E>* sg = nullptr) {
 #pragma unroll
   for (int j = 0; j < E / 8; ++j) {
-    const uint4 w = lds128(saddr + 16u * static_cast<uint32_t>(j ^ tau));
+    uint4 w = lds128(saddr + 16u * static_cast<uint32_t>(j ^ tau));
+    if constexpr (SIGNED) {
+      const uint4 f = chunk_sign_xor(unit_sign_byte<E>(*sg, j, tau));
+      w.x ^= f.x;
+      w.y ^= f.y;
+      w.z ^= f.z;
+      w.w ^= f.w;
+    }
     if constexpr (B >= 2) {
       p[4 * j + 0] = bf16_pair_butterfly_oddneg(w.x);
       p[4 * j + 1] = bf16_pair_butterfly_oddneg(w.y);
@@ -390,9 +453,9 @@ __device__ __forceinline__ void quantize_store_unit(const f32x2 (&p)[Cfg::kPairs
 // Per-warp streaming skeleton shared by the quantize and the amax kernels.  `body(p, unit)`
 // is called once per unit with the rotated (unnormalised) pairs.  Returns false when a
 // bounded wait ran out.
-template <class Cfg, class Body>
+template <class Cfg, bool SIGNED = false, class Body>
 __device__ __forceinline__ bool stream_units(const uint16_t* __restrict__ x, int64_t n_units, uint8_t* warp_smem,
-                                             int tau, Body&& body) {
+                                             int tau, Body&& body, ChannelSigns sgn = {nullptr, 1, 0}) {
   constexpr int S = Cfg::kStages, SU = Cfg::kUnitsPerStage, E = Cfg::kE;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -425,6 +488,12 @@ __device__ __forceinline__ bool stream_units(const uint16_t* __restrict__ x, int
     for (int64_t t = 0; t < S && t < n_stages; ++t) issue(t);
   __syncwarp();
 
+  // SIGNED: channel-unit index (u mod upr) of this lane's r-th unit of the current stage
+  int cu[Cfg::kR];
+  if constexpr (SIGNED) {
+#pragma unroll
+    for (int r = 0; r < Cfg::kR; ++r) cu[r] = static_cast<int>((u0 + r * 32 + lane) % sgn.upr);
+  }
   bool ok = true;
 #pragma unroll 1
   for (int64_t t = 0; t < n_stages; ++t) {
@@ -449,7 +518,12 @@ __device__ __forceinline__ bool stream_units(const uint16_t* __restrict__ x, int
       for (int r = 0; r < Cfg::kR; ++r) {
         const int lu = r * 32 + lane;
         f32x2 p[Cfg::kPairs];
-        load_rotate_unit<Cfg::kBlock, E>(sbase + static_cast<uint32_t>(lu) * (E * 2), tau, p);
+        if constexpr (SIGNED) {
+          const UnitSigns<E> m = unit_signs<E>(sgn.mask, cu[r]);
+          load_rotate_unit<Cfg::kBlock, E, true>(sbase + static_cast<uint32_t>(lu) * (E * 2), tau, p, &m);
+        } else {
+          load_rotate_unit<Cfg::kBlock, E>(sbase + static_cast<uint32_t>(lu) * (E * 2), tau, p);
+        }
         body(p, us + lu);
       }
     } else {
@@ -458,9 +532,21 @@ __device__ __forceinline__ bool stream_units(const uint16_t* __restrict__ x, int
         const int lu = r * 32 + lane;
         if (lu < cnt) {
           f32x2 p[Cfg::kPairs];
-          load_rotate_unit<Cfg::kBlock, E>(sbase + static_cast<uint32_t>(lu) * (E * 2), tau, p);
+          if constexpr (SIGNED) {
+            const UnitSigns<E> m = unit_signs<E>(sgn.mask, cu[r]);
+            load_rotate_unit<Cfg::kBlock, E, true>(sbase + static_cast<uint32_t>(lu) * (E * 2), tau, p, &m);
+          } else {
+            load_rotate_unit<Cfg::kBlock, E>(sbase + static_cast<uint32_t>(lu) * (E * 2), tau, p);
+          }
           body(p, us + lu);
         }
+      }
+    }
+    if constexpr (SIGNED) {
+#pragma unroll
+      for (int r = 0; r < Cfg::kR; ++r) {
+        cu[r] += sgn.stage_step;
+        if (cu[r] >= sgn.upr) cu[r] -= sgn.upr;
       }
     }
     __syncwarp();
@@ -509,10 +595,13 @@ __global__ void __launch_bounds__(Cfg::kThreads) rotate_quantize_kernel(RQArgs a
   if constexpr (Cfg::kFmt == kNV) s_g = cta_tensor_scale<Cfg>(a.tensor_scale, a.partials, a.n_partials, &s_tensor_scale);
   const float nv_den = 6.0f * s_g;
   const float nv_rden = __frcp_rn(nv_den);
-  stream_units<Cfg>(a.x, a.n_units, smem + warp * Cfg::kWarpSmem, lx.tau,
-                    [&](const f32x2 (&p)[Cfg::kPairs], int64_t unit) {
-                      quantize_store_unit<Cfg>(p, unit, lx, s_g, nv_den, nv_rden, a);
-                    });
+  auto body = [&](const f32x2 (&p)[Cfg::kPairs], int64_t unit) {
+    quantize_store_unit<Cfg>(p, unit, lx, s_g, nv_den, nv_rden, a);
+  };
+  if (a.signs.mask)
+    stream_units<Cfg, true>(a.x, a.n_units, smem + warp * Cfg::kWarpSmem, lx.tau, body, a.signs);
+  else
+    stream_units<Cfg>(a.x, a.n_units, smem + warp * Cfg::kWarpSmem, lx.tau, body);
 }
 
 // ---------------------------------------------------------------- quantization error
@@ -618,6 +707,7 @@ struct QEArgs {
   double* out_partials;     // [gridDim.x][2]: signal, error energy of each CTA
   unsigned int* ticket;     // CTAs done so far; 0 between calls (the last CTA resets it)
   double* out;              // [3]: signal, error, QSNR dB
+  ChannelSigns signs;       // per-channel random signs (mask nullptr: none)
 };
 
 // out = {signal, error, QSNR in dB} from n per-CTA partial pairs, by one warp in a fixed
@@ -659,8 +749,11 @@ __global__ void __launch_bounds__(Cfg::kThreads) quant_error_kernel(QEArgs a) {
   const float nv_den = 6.0f * s_g;
   const float nv_rden = __frcp_rn(nv_den);
   double sig = 0.0, err = 0.0;
-  stream_units<Cfg>(a.x, a.n_units, smem + warp * Cfg::kWarpSmem, lx.tau,
-                    [&](const f32x2 (&p)[Cfg::kPairs], int64_t) { unit_energies<Cfg>(p, s_g, nv_den, nv_rden, sig, err); });
+  auto body = [&](const f32x2 (&p)[Cfg::kPairs], int64_t) { unit_energies<Cfg>(p, s_g, nv_den, nv_rden, sig, err); };
+  if (a.signs.mask)
+    stream_units<Cfg, true>(a.x, a.n_units, smem + warp * Cfg::kWarpSmem, lx.tau, body, a.signs);
+  else
+    stream_units<Cfg>(a.x, a.n_units, smem + warp * Cfg::kWarpSmem, lx.tau, body);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     sig += __shfl_xor_sync(0xFFFFFFFFu, sig, o);
@@ -701,15 +794,18 @@ __global__ void quant_error_empty_kernel(const double* __restrict__ partials, do
 // Rotated amax: every CTA writes max |fl(y)| over its warps' ranges to partials[blockIdx.x].
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::kThreads) rotated_amax_kernel(const uint16_t* __restrict__ x, int64_t n_units,
-                                                                     float* __restrict__ partials) {
+                                                                     float* __restrict__ partials, ChannelSigns signs) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float s_max[Cfg::kWarps];
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5;
   const LaneXor lx = lane_xor<Cfg>(threadIdx.x & 31);
   float m = 0.0f;
-  stream_units<Cfg>(x, n_units, smem + warp * Cfg::kWarpSmem, lx.tau,
-                    [&](const f32x2 (&p)[Cfg::kPairs], int64_t) { m = fmaxf(m, pairs_amax<Cfg::kPairs>(p)); });
+  auto body = [&](const f32x2 (&p)[Cfg::kPairs], int64_t) { m = fmaxf(m, pairs_amax<Cfg::kPairs>(p)); };
+  if (signs.mask)
+    stream_units<Cfg, true>(x, n_units, smem + warp * Cfg::kWarpSmem, lx.tau, body, signs);
+  else
+    stream_units<Cfg>(x, n_units, smem + warp * Cfg::kWarpSmem, lx.tau, body);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
   if ((threadIdx.x & 31) == 0) s_max[warp] = m;
@@ -738,7 +834,7 @@ template <int FMT, int B, bool UNROTATE>
 __global__ void __launch_bounds__(128) dequantize_kernel(const uint8_t* __restrict__ codes,
                                                          const uint8_t* __restrict__ scales,
                                                          const float* __restrict__ tensor_scale, int64_t n_units,
-                                                         float* __restrict__ out) {
+                                                         float* __restrict__ out, ChannelSigns signs) {
   constexpr int G = FMT == kMX ? 32 : 16;
   constexpr int E = cmax(B, G);
   const int64_t unit = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -767,6 +863,15 @@ __global__ void __launch_bounds__(128) dequantize_kernel(const uint8_t* __restri
     constexpr float c = inv_sqrt_block(B);
 #pragma unroll
     for (int i = 0; i < E; ++i) v[i] *= c;
+    if (signs.mask) {
+      // the channel signs again, after the block rotation (Q^-1 = Q^T)
+      const int c0 = static_cast<int>(unit % signs.upr) * E;
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+        const uint32_t bit = (__ldg(signs.mask + ((c0 + i) >> 5)) >> ((c0 + i) & 31)) & 1u;
+        v[i] = __uint_as_float(__float_as_uint(v[i]) ^ (bit << 31));
+      }
+    }
   }
   float4* op = reinterpret_cast<float4*>(out + unit * E);
 #pragma unroll

@@ -35,6 +35,7 @@ _SIGS = {
     "fp4q_plan_create": (_int, [ctypes.POINTER(_vp), _int, _int, _int, _int]),
     "fp4q_plan_destroy": (_int, [_vp]),
     "fp4q_plan_set_kernel": (_int, [_vp, _int]),
+    "fp4q_plan_set_signs": (_int, [_vp, _vp, _i64]),
     "fp4q_rotate_quantize": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp]),
     "fp4q_rotate_quantize_dump": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
     "fp4q_amax": (_int, [_vp, _vp, _i64, _i64, _vp, _vp]),
@@ -117,6 +118,13 @@ def fp4q_plan_create(fmt: int, group: int, hadamard_block: int, scale_rule: int)
 def fp4q_plan_set_kernel(plan: Plan, kernel: int) -> None:
     _check(_lib.fp4q_plan_set_kernel(plan.handle, kernel), "fp4q_plan_set_kernel")
     plan.kernel = kernel
+
+
+def fp4q_plan_set_signs(plan: Plan, signs, K: int) -> None:
+    """signs: device uint32 tensor [ceil(K/32)] (bit k negates channel k) or None to clear.
+    The plan keeps a reference to the tensor so that it stays alive."""
+    _check(_lib.fp4q_plan_set_signs(plan.handle, _ptr(signs), K), "fp4q_plan_set_signs")
+    plan.signs = signs
 
 
 def fp4q_plan_destroy(plan: Plan) -> None:

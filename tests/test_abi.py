@@ -66,6 +66,25 @@ def test_kernel_selection_without_gpu(F):
         F.fp4q_plan_set_kernel(q, k)
 
 
+def test_sign_validation_without_gpu(F):
+    p = F.fp4q_plan_create(F.FP4Q_MXFP4, 32, 128, F.FP4Q_SCALE_FLOOR_OCP)
+    ss = lambda *a: F.raw_call("fp4q_plan_set_signs", *a)
+    A = 1 << 20
+    assert ss(None, A, 128) == F.FP4Q_ERR_ARG
+    assert ss(p.handle, A, 100) == F.FP4Q_ERR_SHAPE            # not a multiple of max(g, b)
+    assert ss(p.handle, A, 0) == F.FP4Q_ERR_SHAPE
+    assert ss(p.handle, A, 1 << 35) == F.FP4Q_ERR_SHAPE
+    assert ss(p.handle, A + 2, 128) == F.FP4Q_ERR_ALIGN
+    assert ss(p.handle, A, 256) == F.FP4Q_OK
+    rq = lambda *a: F.raw_call("fp4q_rotate_quantize", *a)
+    assert rq(p.handle, A, 4, 128, A, A, None, None) == F.FP4Q_ERR_SHAPE      # K differs from the signs'
+    assert F.raw_call("fp4q_plan_set_kernel", p.handle, F.FP4Q_KERNEL_TENSOR_CORE) == F.FP4Q_ERR_UNSUPPORTED
+    assert ss(p.handle, None, 0) == F.FP4Q_OK                   # cleared
+    F.fp4q_plan_set_kernel(p, F.FP4Q_KERNEL_TENSOR_CORE)
+    assert ss(p.handle, A, 256) == F.FP4Q_ERR_UNSUPPORTED       # forced tensor-core kernel
+    F.fp4q_plan_destroy(p)
+
+
 def test_call_validation_without_gpu(F):
     p = F.fp4q_plan_create(F.FP4Q_MXFP4, 32, 128, F.FP4Q_SCALE_FLOOR_OCP)
     rq = lambda *a: F.raw_call("fp4q_rotate_quantize", *a)

@@ -1,0 +1,116 @@
+"""GPU parity of the randomised rotation (per-channel random signs, plan-level) with the
+CPU oracle, and the weight-side path it serves: the same signs on activations and weights,
+round-to-nearest FP4 weights, and the GEMM identity of the rotated operands.
+
+Source: "Bridging the Gap Between Promise and Performance for Microscaling FP4
+Quantization", Technische Zusammenfassung, 2. Methodik (block-wise Hadamard transforms
+of weights and activations, "wie in QuIP/QuaRot") and the English abstract (rotation
+fused into the weights, fast online computation of the activations)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as o
+from microscaling_fp4_quantization_b200 import workloads as W
+from parity import assert_parity, rotated_value_error
+from test_parity_small import COMBOS, combo_id, make_input
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def F(cuda_device):
+    from microscaling_fp4_quantization_b200 import fp4q
+    return fp4q
+
+
+def signed_plan(F, combo, K, seed):
+    fmt, g, b, rule = combo
+    plan = F.fp4q_plan_create(fmt, g, b, rule)
+    mask = W.random_sign_mask(K, seed)
+    md = torch.from_numpy(mask.view(np.int32)).cuda()
+    F.fp4q_plan_set_signs(plan, md, K)
+    return plan, o.sign_vector(mask, K)
+
+
+@pytest.mark.parametrize("combo", COMBOS, ids=[combo_id(c) for c in COMBOS])
+def test_signed_rotate_quantize_matches_oracle(F, combo):
+    import gpu_util as gu
+    fmt, g, b, rule = combo
+    unit = max(g, b)
+    for i, (M, K) in enumerate([(3, 2 * unit), (37, 6 * unit), (130, 4096 // unit * unit), (200, 1536)]):
+        plan, s = signed_plan(F, combo, K, seed=500 + i)
+        x = make_input(M, K, seed=9000 + 100 * b + 10 * rule + i, adversarial=M >= 8)
+        s_g = o.nv_tensor_scale(o.rotated_amax(x, b, signs=s)) if rule == o.SCALE_NV_STATIC else None
+        res = o.rotate_quantize(x, fmt, g, b, rule, tensor_scale=s_g, signs=s)
+        out = gu.run_rotate_quantize(F, plan, x, tensor_scale=s_g, dump=True)
+        adversarial = M >= 8
+        assert_parity(res, out["codes"], out["scales"], f"{combo_id(combo)} {M}x{K} signed",
+                      count_bound=not adversarial)
+        assert rotated_value_error(out["y"], res) <= 1e-5, (M, K)
+        if rule == o.SCALE_NV_DYNAMIC:
+            assert abs(float(out["tensor_scale"]) - float(res["tensor_scale"])) <= 2.5e-7 * float(res["tensor_scale"])
+
+
+@pytest.mark.parametrize("b", [1, 16, 128])
+def test_signed_amax_and_quant_error(F, b):
+    import gpu_util as gu
+    from test_quant_error import assert_energies, run_qe
+    M, K = 300, 1024
+    x = make_input(M, K, seed=40 + b, adversarial=False)
+    plan, s = signed_plan(F, (o.NVFP4, 16, b, o.SCALE_NV_STATIC), K, seed=7)
+    ours = gu.run_amax(F, plan, x)
+    ref = o.nv_tensor_scale(o.rotated_amax(x, b, signs=s))
+    assert abs(float(ours) - float(ref)) <= 2.5e-7 * float(ref)
+    assert ref != o.nv_tensor_scale(o.rotated_amax(x, b)) or b == 1
+    qe_ref = o.quant_error(x, o.NVFP4, 16, b, o.SCALE_NV_STATIC, tensor_scale=ref, signs=s)
+    assert_energies(run_qe(F, plan, x, tensor_scale=ref), qe_ref, f"b{b} signed")
+    mplan, ms = signed_plan(F, (o.MXFP4, 32, b, o.SCALE_OAS), K, seed=8)
+    assert_energies(run_qe(F, mplan, x), o.quant_error(x, o.MXFP4, 32, b, o.SCALE_OAS, signs=ms), f"mx b{b} signed")
+
+
+@pytest.mark.parametrize("b", [2, 32, 128])
+def test_signed_dequantize_rotates_back(F, b):
+    import gpu_util as gu
+    M, K = 64, 512
+    x = make_input(M, K, seed=3 + b, adversarial=False)
+    plan, s = signed_plan(F, (o.MXFP4, 32, b, o.SCALE_FLOOR_OCP), K, seed=11)
+    out = gu.run_rotate_quantize(F, plan, x)
+    back = gu.run_dequantize(F, plan, out["codes"], out["scales"], None, unrotate=True)
+    ref = o.dequantize(out["codes"], out["scales"], o.MXFP4, 32, b, unrotate_back=True, signs=s)
+    scale = np.abs(ref).max()
+    assert np.max(np.abs(back - ref)) <= 1e-6 * scale
+
+
+def test_weight_path_gemm_identity(F):
+    """Weights rotated and quantized with the same signs as the activations: the GEMM of the
+    rotated dequantized operands equals the GEMM of the operands rotated back (Q is
+    orthogonal), and it approximates X W^T with the quantization error that the error pass
+    reports for each side."""
+    import gpu_util as gu
+    K, M, N = 2048, 256, 192
+    b = 128
+    X = W.NV_4K.with_rows(M).generate()[:, :K].copy()
+    Wt = W.synthetic_weights(N, K, seed=2)
+    mask = W.random_sign_mask(K, 21)
+    md = torch.from_numpy(mask.view(np.int32)).cuda()
+    plan = F.fp4q_plan_create(o.MXFP4, 32, b, o.SCALE_OAS)
+    F.fp4q_plan_set_signs(plan, md, K)
+    xq = gu.run_rotate_quantize(F, plan, X)
+    wq = gu.run_rotate_quantize(F, plan, Wt)
+    Xr = gu.run_dequantize(F, plan, xq["codes"], xq["scales"], None, unrotate=False).astype(np.float64)
+    Wr = gu.run_dequantize(F, plan, wq["codes"], wq["scales"], None, unrotate=False).astype(np.float64)
+    Xb = gu.run_dequantize(F, plan, xq["codes"], xq["scales"], None, unrotate=True).astype(np.float64)
+    Wb = gu.run_dequantize(F, plan, wq["codes"], wq["scales"], None, unrotate=True).astype(np.float64)
+    G_rot = Xr @ Wr.T
+    G_back = Xb @ Wb.T
+    assert np.max(np.abs(G_rot - G_back)) <= 1e-5 * np.abs(G_rot).max()
+    ref = o.bf16_to_f64(X) @ o.bf16_to_f64(Wt).T
+    rel = np.linalg.norm(G_rot - ref) / np.linalg.norm(ref)
+    assert rel < 0.2, rel
+    # the codes are those of the oracle with the same signs
+    s = o.sign_vector(mask, K)
+    for A, q in ((X, xq), (Wt, wq)):
+        res = o.rotate_quantize(A, o.MXFP4, 32, b, o.SCALE_OAS, signs=s)
+        assert_parity(res, q["codes"], q["scales"], "weight path")
