@@ -60,6 +60,8 @@ import numpy as np
 
 MXFP4 = 0
 NVFP4 = 1
+MXFP4_MBS = 2          # MXFP4 under an MBS-Static macro-block scale ([UP] Methodologie 2)
+MBS_MACRO = 128        # elements per macro block
 
 SCALE_FLOOR_OCP = 0
 SCALE_CEIL_NOCLIP = 1
@@ -267,7 +269,7 @@ def nv_tensor_scale(A_tensor: float) -> np.float32:
 # ----------------------------------------------------------------------------------
 
 def check_plan(fmt: int, group: int, block: int, rule: int) -> None:
-    if fmt == MXFP4:
+    if fmt in (MXFP4, MXFP4_MBS):
         if group != 32 or rule not in (SCALE_FLOOR_OCP, SCALE_CEIL_NOCLIP, SCALE_OAS):
             raise ValueError("MXFP4 uses groups of 32 and an MX scale rule")
     elif fmt == NVFP4:
@@ -345,6 +347,84 @@ def rotate_quantize(x_bits: np.ndarray, fmt: int, group: int, block: int, rule: 
     }
 
 
+# ----------------------------------------------------------------------------------
+# MBS-Static ([UP] Technische samenvatting, Methodologie 2, "Macro Block Scaling"): every
+# macro block of 128 elements gets one extra scale factor with 8 mantissa bits, computed
+# directly from the macro block's maximum; the values are divided by it before the
+# standard MXFP4 quantization of their 32-element groups.
+# ----------------------------------------------------------------------------------
+
+def mbs_macro_byte(A_M32: np.ndarray) -> np.ndarray:
+    """Macro-scale byte m8 from the fp32 macro-block maximum A_M.
+
+    With fp32(A_M / 6) = 2^E (1 + f), f in [0, 1): m8 = ceil(256 f) mod 256 and the macro
+    scale is s_M = 1 + m8 / 256.  s_M is the mantissa of A_M / 6 rounded up to 8 bits, so
+    A_M / s_M <= 6 * 2^E: the block maximum lands on (or just under) the top E2M1 value
+    under its power-of-two group scale and never above it.  ceil(256 f) = 256 means
+    s_M = 2, which is s_M = 1 with every group exponent one higher: byte 0.  A_M = 0 gives
+    byte 0."""
+    r = (np.asarray(A_M32, np.float32) / np.float32(6.0)).astype(np.float32)   # fp32 IEEE division
+    m, _ = np.frexp(r.astype(np.float64))                                       # r = m 2^E', m in [0.5, 1)
+    f = np.where(r > 0, 2.0 * m - 1.0, 0.0)                                     # exact
+    return (np.ceil(f * 256.0).astype(np.int64) % 256).astype(np.uint8)
+
+
+def mbs_macro_scale(m8: np.ndarray) -> np.ndarray:
+    """s_M = 1 + m8 / 256 (exact in fp32)."""
+    return (1.0 + np.asarray(m8, np.float64) / 256.0).astype(np.float32)
+
+
+def rotate_quantize_mbs(x_bits: np.ndarray, group: int, block: int, rule: int, signs=None) -> dict:
+    """Rotate, then MXFP4 (groups of 32, E8M0 by ``rule``) under MBS-Static macro scales.
+
+    y' = fp32(y32 / s_M) (IEEE division) for the 128 elements of each macro block; the
+    group amax, the E8M0 exponent e and the E2M1 codes are taken on y' exactly as for
+    MXFP4.  The dequantized value is q * 2^e * s_M.  Returns the keys of
+    ``rotate_quantize`` plus ``macro`` (M, K/128) uint8 and ``yp32``."""
+    check_plan(MXFP4_MBS, group, block, rule)
+    x_bits = np.asarray(x_bits, np.uint16)
+    M, K = x_bits.shape
+    if K % MBS_MACRO or K % block:
+        raise ValueError("K must be a multiple of the macro block (128) and of the Hadamard block")
+    y64 = rotate(x_bits, block, signs)
+    y32 = y64.astype(np.float32)
+    ym = y32.reshape(M, K // MBS_MACRO, MBS_MACRO)
+    AM = np.max(np.abs(ym), axis=2) if K else np.zeros((M, 0), np.float32)
+    m8 = mbs_macro_byte(AM)
+    sM = mbs_macro_scale(m8)
+    yp = (ym / sM[..., None]).astype(np.float32).reshape(M, K)      # fp32 IEEE division
+    yg = yp.reshape(M, K // group, group)
+    A32 = np.max(np.abs(yg), axis=2) if K else np.zeros((M, 0), np.float32)
+    e = mx_scale_exponent(A32, rule)
+    v = (yg.astype(np.float64) / np.ldexp(1.0, e)[..., None]).astype(np.float32)   # exact: power of two
+    q = e2m1_encode(v)
+    sM_g = np.repeat(sM.astype(np.float64), MBS_MACRO // group, axis=1)
+    return {
+        "codes": pack_nibbles(q.reshape(M, K)),
+        "scales": (e + 127).astype(np.uint8).reshape(M, K // group),
+        "macro": m8.reshape(M, K // MBS_MACRO),
+        "y64": y64, "y32": y32, "yp32": yp,
+        "amax32": A32,
+        "S64": np.ldexp(1.0, e) * sM_g,
+        "tensor_scale": None,
+        "fmt": MXFP4_MBS, "group": group, "block": block, "rule": rule,
+    }
+
+
+def dequantize_mbs(codes: np.ndarray, scales: np.ndarray, macro: np.ndarray, group: int, block: int,
+                   unrotate_back: bool = False, signs=None) -> np.ndarray:
+    """q * 2^(byte - 127) * s_M (exact in fp32: 2 + 9 significant bits), optionally rotated back."""
+    q = e2m1_decode(unpack_nibbles(codes))
+    M, K = q.shape
+    S = np.ldexp(1.0, np.asarray(scales, np.int64).reshape(M, K // group) - 127)
+    sM = np.repeat(mbs_macro_scale(np.asarray(macro, np.uint8).reshape(M, K // MBS_MACRO)).astype(np.float64),
+                   MBS_MACRO // group, axis=1)
+    x = (q.reshape(M, K // group, group) * (S * sM)[..., None]).astype(np.float32).reshape(M, K)
+    if unrotate_back:
+        return unrotate(x.astype(np.float64), block, signs)
+    return x
+
+
 def dequantize(codes: np.ndarray, scales: np.ndarray, fmt: int, group: int, block: int,
                tensor_scale=None, unrotate_back: bool = False, signs=None) -> np.ndarray:
     """codes x block scale (x tensor scale), optionally rotated back.
@@ -403,11 +483,23 @@ def flags(res: dict, tol: float = 1e-5):
     for mp in E2M1_MIDPOINTS:
         el |= np.abs(a - mp) <= tol * mp
     rule = res["rule"]
-    if res["fmt"] == MXFP4:
+    if res["fmt"] in (MXFP4, MXFP4_MBS):
+        if res["fmt"] == MXFP4_MBS:
+            # the group rule sees A / s_M; a macro block whose exact 256 f lies within tol of an
+            # integer (where the ceil can step) flags all of its groups
+            sM = np.repeat(mbs_macro_scale(res["macro"]).astype(np.float64), MBS_MACRO // g, axis=1)
+            A64 = A64 / sM
+            ym = np.abs(y64.reshape(M, K // MBS_MACRO, MBS_MACRO))
+            r = ym.max(axis=2) / 6.0 if K else np.zeros((M, 0))
+            mm, _ = np.frexp(r)
+            t = np.where(r > 0, (2.0 * mm - 1.0) * 256.0, 0.0)
+            near_m = (np.abs(t - np.round(t)) <= tol * 256.0) & (r > 0)
         base = {SCALE_FLOOR_OCP: 1.0, SCALE_CEIL_NOCLIP: 1.5, SCALE_OAS: 1.75}[rule]
         gr = _near_scaled_power(A64, base, tol)
         if rule == SCALE_OAS:
             gr |= _near_scaled_power(A64, 1.5, tol)
+        if res["fmt"] == MXFP4_MBS:
+            gr |= np.repeat(near_m, MBS_MACRO // g, axis=1)
     else:
         s_b = A64 / (6.0 * np.float64(res["tensor_scale"]))
         T = e4m3_table()
@@ -446,7 +538,10 @@ def quant_error(x_bits: np.ndarray, fmt: int, group: int, block: int, rule: int,
     signal = 0.0
     noise = 0.0
     for r in range(0, M, chunk_rows):
-        res = rotate_quantize(x_bits[r:r + chunk_rows], fmt, group, block, rule, tensor_scale, signs)
+        if fmt == MXFP4_MBS:
+            res = rotate_quantize_mbs(x_bits[r:r + chunk_rows], group, block, rule, signs)
+        else:
+            res = rotate_quantize(x_bits[r:r + chunk_rows], fmt, group, block, rule, tensor_scale, signs)
         y = res["y64"]
         m = y.shape[0]
         q = e2m1_decode(unpack_nibbles(res["codes"])).reshape(m, K // group, group)

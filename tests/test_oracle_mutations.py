@@ -240,3 +240,56 @@ def test_sign_pins_catch_planted_mistake(monkeypatch, name, fn, catchers):
     patch(monkeypatch, name, fn)
     for catcher in catchers:
         assert fails(catcher), f"{catcher.__name__} missed {fn.__name__}"
+
+
+# ---- MBS-Static (pins in test_oracle_mbs.py)
+
+import test_oracle_mbs as mpins  # noqa: E402
+
+_orig_macro_byte = core.mbs_macro_byte
+_orig_rq_mbs = core.rotate_quantize_mbs
+
+
+def macro_byte_nearest(A_M32):
+    """Rounds the mantissa to nearest instead of up."""
+    r = (np.asarray(A_M32, np.float32) / np.float32(6.0)).astype(np.float32)
+    m, _ = np.frexp(r.astype(np.float64))
+    f = np.where(r > 0, 2.0 * m - 1.0, 0.0)
+    return (np.rint(f * 256.0).astype(np.int64) % 256).astype(np.uint8)
+
+
+def macro_byte_amax_not_divided(A_M32):
+    """Takes the mantissa of A_M instead of A_M / 6."""
+    return _orig_macro_byte(np.asarray(A_M32, np.float32) * np.float32(6.0))
+
+
+def rq_mbs_macro_64(x_bits, group, block, rule, signs=None):
+    """Macro blocks of 64 elements: quantizes each half of a 128-element block on its own."""
+    x = np.asarray(x_bits, np.uint16)
+    M, K = x.shape
+    if K % 128 == 0 and block <= 64:
+        halves = x.reshape(M, K // 64, 64)
+        pad = np.concatenate([halves, np.zeros_like(halves)], axis=2).reshape(M * K // 64, 128)
+        r = _orig_rq_mbs(pad, group, block, rule, signs=None)
+        q = o.unpack_nibbles(r["codes"]).reshape(M, K // 64, 128)[:, :, :64].reshape(M, K)
+        r["codes"] = o.pack_nibbles(q)
+        r["scales"] = r["scales"].reshape(M, K // 64, 4)[:, :, :2].reshape(M, K // 32)
+        r["macro"] = r["macro"].reshape(M, K // 64)[:, ::2]
+        return r
+    return _orig_rq_mbs(x_bits, group, block, rule, signs)
+
+
+MBS_MUTATIONS = [
+    ("mbs_macro_byte", macro_byte_nearest, [mpins.test_macro_byte_brute_force,
+                                            mpins.test_block_maximum_takes_the_top_code_under_the_ceil_rule]),
+    ("mbs_macro_byte", macro_byte_amax_not_divided, [mpins.test_hand_worked_macro_block,
+                                                     mpins.test_macro_byte_brute_force]),
+    ("rotate_quantize_mbs", rq_mbs_macro_64, [mpins.test_hand_worked_macro_block]),
+]
+
+
+@pytest.mark.parametrize("name,fn,catchers", MBS_MUTATIONS, ids=[m[1].__name__ for m in MBS_MUTATIONS])
+def test_mbs_pins_catch_planted_mistake(monkeypatch, name, fn, catchers):
+    patch(monkeypatch, name, fn)
+    for catcher in catchers:
+        assert fails(catcher), f"{catcher.__name__} missed {fn.__name__}"
