@@ -350,6 +350,8 @@ def run_gpu(args):
             if ow.block >= 16 and ow.block >= ow.group:
                 alt = "butterfly" if kernel_name(ow, "auto") == "tensor_core" else "tensor_core"
                 others[ow.name + f" [{alt} kernel]"] = time_other(torch, F, ow, dev, stream, peak, kernel=alt)
+        for ow in (W.MX_8K_FLOOR, W.PREFILL_MX):
+            others[ow.name + " [MBS-Static]"] = time_mbs(torch, F, ow, dev, stream, peak)
 
     if rank == 0:
         cpu = cpu_baseline(w, args) if world == 1 and not args.no_cpu_baseline else None
@@ -488,6 +490,49 @@ def time_quant_error(torch, F, w, plan, xs, ts, stream, peak, steps):
     return {"us_per_call": round(us, 3), "GBps": round(gbs, 1), "pct_of_hbm_peak": round(100 * gbs / peak, 2),
             "bytes_per_call": nbytes, "launches_per_call": 1, "qsnr_db": round(q, 4), "signal": sig, "error": err,
             "mse": err / (M * K)}
+
+
+def time_mbs(torch, F, w, dev, stream, peak):
+    """MBS-Static (MXFP4 with 128-element macro scales) on an MX workload's input: GB/s on its
+    algorithmic bytes (bf16 in; codes, E8M0 group scales and macro bytes out), and the QSNR
+    against plain MXFP4 with the same rule."""
+    M, K = w.M, w.K
+    plan = F.fp4q_plan_create(F.FP4Q_MXFP4_MBS, 32, w.block, w.rule)
+    x_np = w.generate()
+    nbytes = M * K * 2 + M * K // 2 + M * K // 32 + M * K // 128
+    n_buf = max(1, math.ceil(3 * L2_BYTES / nbytes)) if nbytes < 2 * L2_BYTES else 1
+    xh = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16)
+    xs = [xh.to(dev) for _ in range(n_buf)]
+    del x_np, xh
+    codes = [torch.empty((M, K // 2), dtype=torch.uint8, device=dev) for _ in range(n_buf)]
+    scales = [torch.empty((M, K // 32), dtype=torch.uint8, device=dev) for _ in range(n_buf)]
+    macro = [torch.empty((M, K // 128), dtype=torch.uint8, device=dev) for _ in range(n_buf)]
+
+    def launch(i):
+        F.fp4q_rotate_quantize_mbs(plan, xs[i], M, K, codes[i], scales[i], macro[i], stream=torch.cuda.current_stream())
+
+    steps = 200 if nbytes > 1e8 else 2000
+    with torch.cuda.stream(stream):
+        g, g_rem, reps = time_graph_steps(torch, launch, n_buf, steps, 5, stream)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        a1.record(stream)
+    torch.cuda.synchronize()
+    us = a0.elapsed_time(a1) * 1e3 / steps
+    gbs = nbytes / us / 1e3
+    qe_mbs = time_quant_error(torch, F, w, plan, xs, None, stream, peak, 20)
+    plain = F.fp4q_plan_create(w.fmt, w.group, w.block, w.rule)
+    qe_plain = time_quant_error(torch, F, w, plain, xs, None, stream, peak, 20)
+    out = {"GBps": round(gbs, 1), "pct_of_hbm_peak": round(100 * gbs / peak, 2), "us_per_call": round(us, 3),
+           "bytes_per_call": nbytes, "buffers": n_buf, "kernel": "butterfly",
+           "qsnr_db": qe_mbs["qsnr_db"], "qsnr_db_plain_mxfp4": qe_plain["qsnr_db"]}
+    del xs, codes, scales, macro
+    torch.cuda.empty_cache()
+    return out
 
 
 def time_other(torch, F, w, dev, stream, peak, kernel="auto"):

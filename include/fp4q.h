@@ -43,15 +43,18 @@
  * Shape rules: M >= 0, K >= 0, K a multiple of lcm(g, b), M*K < 2^40.  M*K = 0 is a valid
  * empty call that launches nothing.
  *
- * Ownership.  The caller owns every buffer passed in.  A plan owns nothing on the device
- * except, for FP4Q_SCALE_NV_DYNAMIC and for fp4q_amax, a small device array of per-CTA
- * partial maxima that fp4q_plan_create allocates and fp4q_plan_destroy frees.  Calls
+ * Ownership.  The caller owns every buffer passed in.  A plan owns two small device
+ * arrays that fp4q_plan_create allocates and fp4q_plan_destroy frees: the per-CTA partial
+ * maxima of NV plans (for FP4Q_SCALE_NV_DYNAMIC and fp4q_amax), and the per-CTA partial
+ * sums of fp4q_quant_error (every plan made on a machine with a CUDA device).  Calls
  * allocate nothing.
  *
  * Streams.  Every call is asynchronous and stream-ordered on the given stream (a
- * cudaStream_t passed as void*; NULL is the legacy default stream).  A plan is immutable
- * after creation; two calls that share a DYNAMIC plan must be ordered on one stream
- * (they share the plan's partial-maximum array).
+ * cudaStream_t passed as void*; NULL is the legacy default stream).  A plan's format, group,
+ * block and rule are fixed at creation; fp4q_plan_set_kernel and fp4q_plan_set_signs change
+ * its kernel choice and channel signs for later calls and must not race with calls in
+ * flight on it.  Two calls that share a DYNAMIC plan, or two fp4q_quant_error calls on one
+ * plan, must be ordered on one stream (they share the plan's scratch arrays).
  *
  * Errors.  Argument problems are found on the host before anything is launched and
  * return FP4Q_ERR_ARG / _SHAPE / _ALIGN / _UNSUPPORTED.  A CUDA launch failure returns
@@ -78,7 +81,17 @@ typedef enum {
   FP4Q_ERR_TIMEOUT = 6       /* a bounded wait inside a kernel ran out                */
 } fp4q_status;
 
-typedef enum { FP4Q_MXFP4 = 0, FP4Q_NVFP4 = 1 } fp4q_format;
+/* FP4Q_MXFP4_MBS: MXFP4 under MBS-Static macro-block scales ("Unveiling the Potential of
+ * Quantization with MXFP4", Methodologie 2, Macro Block Scaling).  Every 128-element macro
+ * block of a row gets one extra scale with 8 mantissa bits, taken directly from the block's
+ * maximum A_M: with fp32(A_M / 6) = 2^E (1 + f), the byte m8 = ceil(256 f) mod 256 and
+ * s_M = 1 + m8 / 256 (so the block maximum lands on the top E2M1 value, never above it;
+ * 256 wraps to 0, the same quantization with every group exponent one higher).  The rotated
+ * values are divided by s_M (fp32, correctly rounded) and then quantized as MXFP4 with the
+ * plan's MX rule; a value decodes as E2M1 * 2^(byte - 127) * s_M.  Group 32, K a multiple of
+ * 128.  Served by fp4q_rotate_quantize_mbs, fp4q_dequantize_mbs and fp4q_quant_error (the
+ * butterfly kernel). */
+typedef enum { FP4Q_MXFP4 = 0, FP4Q_NVFP4 = 1, FP4Q_MXFP4_MBS = 2 } fp4q_format;
 
 typedef enum {
   FP4Q_SCALE_FLOOR_OCP = 0,   /* MX: e = floor(log2 A) - 2; values above 6 X saturate  */
@@ -143,6 +156,13 @@ fp4q_status fp4q_rotate_quantize(fp4q_plan plan, const void* x_bf16, int64_t M, 
                                  void* codes_out, void* scales_out, float* tensor_scale,
                                  void* stream);
 
+/* Rotate and quantize X under an FP4Q_MXFP4_MBS plan: codes_out uint8 [M][K/2] and
+ * scales_out uint8 [M][K/32] (E8M0 bytes of the scaled groups) as for MXFP4, and macro_out
+ * uint8 [M][K/128] (the macro-scale bytes m8; any alignment).  Returns FP4Q_ERR_UNSUPPORTED
+ * for a plan of another format; fp4q_rotate_quantize(_dump) return it for an MBS plan. */
+fp4q_status fp4q_rotate_quantize_mbs(fp4q_plan plan, const void* x_bf16, int64_t M, int64_t K,
+                                     void* codes_out, void* scales_out, void* macro_out, void* stream);
+
 /* Same as fp4q_rotate_quantize, and also stores the fp32 rotated values y (before any
  * scaling) to y_out (device fp32 [M][K]).  A debugging and testing aid: the same kernel
  * body with one extra store. */
@@ -184,6 +204,12 @@ fp4q_status fp4q_dequantize(fp4q_plan plan, const void* codes, const void* scale
  * fp4q_rotate_quantize, and out must be 8-byte aligned. */
 fp4q_status fp4q_quant_error(fp4q_plan plan, const void* x_bf16, int64_t M, int64_t K,
                              float* tensor_scale, double* out, void* stream);
+
+/* Decode an FP4Q_MXFP4_MBS result: out[r][k] = E2M1(code) * 2^(byte - 127) * s_M (exact in
+ * fp32), rotated back when unrotate != 0.  macro: the bytes fp4q_rotate_quantize_mbs wrote.
+ * Returns FP4Q_ERR_UNSUPPORTED for other plans; fp4q_dequantize returns it for MBS plans. */
+fp4q_status fp4q_dequantize_mbs(fp4q_plan plan, const void* codes, const void* scales, const void* macro,
+                                int64_t M, int64_t K, int unrotate, float* out_f32, void* stream);
 
 /* No-allocation NVFP4 dynamic-scale path.  The paper has no counterpart: this exists for
  * callers that cannot allocate device memory themselves — for example a library loaded into

@@ -9,6 +9,7 @@ import os
 import shutil
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
@@ -17,8 +18,11 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_DIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIB_DIR, "libfp4q.so")
 
-SOURCES = ["fp4q.cu"]
-DEPS = ["fp4q.cu", "fp4q_kernels.cuh", "fp4q_device.cuh", "fp4q_mma.cuh"]
+# The C ABI and its dispatch, then one unit per kernel family (compiled in parallel).
+SOURCES = ["fp4q.cu", "fp4q_inst_rq_mx.cu", "fp4q_inst_rq_nv.cu", "fp4q_inst_mbs.cu", "fp4q_inst_qe.cu",
+           "fp4q_inst_mma.cu", "fp4q_inst_dequant.cu"]
+DEPS = SOURCES + ["fp4q_kernels.cuh", "fp4q_device.cuh", "fp4q_mma.cuh", "fp4q_host.cuh", "fp4q_launch.cuh"]
+OBJ_DIR = os.path.join(PKG, "lib", "obj")
 
 
 def nvcc() -> str:
@@ -41,20 +45,33 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(d) <= t for d in deps)
 
 
+def _compile(src: str, obj: str, verbose: bool) -> str:
+    cmd = [nvcc(), *flags(), "-c", "-o", obj, os.path.join(CSRC, src)]
+    if verbose:
+        cmd.insert(1, "-Xptxas=-v")
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError(f"nvcc failed on {src} ({r.returncode}):\n{r.stdout}\n{r.stderr}")
+    return r.stdout + r.stderr
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
-    os.makedirs(LIB_DIR, exist_ok=True)
-    tmp = LIB + ".tmp"
-    cmd = [nvcc(), *flags(), "-shared", "-o", tmp] + [os.path.join(CSRC, s) for s in SOURCES]
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    objs = [os.path.join(OBJ_DIR, os.path.splitext(src)[0] + ".o") for src in SOURCES]
+    jobs = max(1, min(len(SOURCES), os.cpu_count() or 1))
+    with ThreadPoolExecutor(max_workers=jobs) as pool:
+        logs = list(pool.map(lambda so: _compile(so[0], so[1], verbose), zip(SOURCES, objs)))
     if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-        print(" ".join(cmd))
+        print("".join(logs))
+    tmp = LIB + ".tmp"
+    # every symbol must resolve inside the library: a launcher instantiated nowhere fails here
+    cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-Xlinker", "--no-undefined",
+           "-o", tmp] + objs
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
-        raise RuntimeError(f"nvcc failed ({r.returncode}):\n{r.stdout}\n{r.stderr}")
-    if verbose:
-        print(r.stdout + r.stderr)
+        raise RuntimeError(f"link failed ({r.returncode}):\n{r.stdout}\n{r.stderr}")
     os.replace(tmp, LIB)
     return LIB
 

@@ -7,60 +7,36 @@
 #include <mutex>
 #include <new>
 #include <unordered_map>
-#include <utility>
 
-#include "fp4q.h"
-#include "fp4q_kernels.cuh"
-#include "fp4q_mma.cuh"
+#include "fp4q_host.cuh"
 
 using namespace fp4q;
+using namespace fp4q::host;
 
-struct fp4q_plan_s {
-  uint32_t magic;
-  int format, group, block, rule;
-  int unit;        // E = max(block, group)
-  int device;
-  float* partials; // NV plans: per-CTA rotated amaxima (device)
-  int n_partials;
-  int kernel;      // fp4q_kernel
-  const uint32_t* signs; // per-channel random signs (device, borrowed; null: none)
-  int64_t signs_K;       // the row length K the signs are for
-  double* err_partials;  // fp4q_quant_error scratch (device; null without a device): per-CTA signal and
-                         // error energy, then a ticket counter
-  int n_err_partials;    // CTAs those hold room for
-};
+namespace fp4q {
+namespace host {
 
 namespace {
+thread_local char g_last_cuda_error[kLastErrorBytes] = "";
+std::mutex g_info_mu;
+std::unordered_map<uint64_t, KernelInfo> g_info;
+std::mutex g_encode_mu;
+EncodeTiledFn g_encode = nullptr;
+}  // namespace
 
-constexpr uint32_t kPlanMagic = 0xF4F4A11Cu;
-thread_local char g_last_cuda_error[512] = "";
+char* last_error_buffer() { return g_last_cuda_error; }
 
 fp4q_status cuda_fail(cudaError_t e, const char* what) {
-  std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s (%s)", what, cudaGetErrorString(e),
+  std::snprintf(last_error_buffer(), kLastErrorBytes, "%s: %s (%s)", what, cudaGetErrorString(e),
                 cudaGetErrorName(e));
   return FP4Q_ERR_CUDA;
 }
 
-bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
-
-bool valid_plan(fp4q_plan p) { return p != nullptr && p->magic == kPlanMagic; }
-
-// Per (kernel, device) one-time set-up: opt in to the dynamic shared memory the kernel
-// needs and record how many CTAs fit on one SM.
-struct KernelInfo {
-  int ctas_per_sm = 0;
-  int sm_count = 0;
-};
-
-std::mutex g_info_mu;
-std::unordered_map<uint64_t, KernelInfo> g_info;
-
-template <class K>
-fp4q_status kernel_info(K kernel, int smem_bytes, int threads, KernelInfo* out) {
+fp4q_status kernel_info_impl(const void* kernel, int smem_bytes, int threads, KernelInfo* out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  const uint64_t key = (reinterpret_cast<uint64_t>(reinterpret_cast<const void*>(kernel)) << 8) ^ static_cast<uint64_t>(dev);
+  const uint64_t key = (reinterpret_cast<uint64_t>(kernel) << 8) ^ static_cast<uint64_t>(dev);
   std::lock_guard<std::mutex> lk(g_info_mu);
   auto it = g_info.find(key);
   if (it != g_info.end()) {
@@ -83,75 +59,6 @@ fp4q_status kernel_info(K kernel, int smem_bytes, int threads, KernelInfo* out) 
   return FP4Q_OK;
 }
 
-// Launch with programmatic stream serialization, so the kernel's start overlaps the tail of
-// the previous kernel on the stream (the kernels wait on the dependency before touching
-// global memory).
-template <class... KArgs, class... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                       Args&&... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
-}
-
-// Call f.template operator()<B>() for the runtime Hadamard block b.
-template <class F>
-fp4q_status with_block(int b, F&& f) {
-  switch (b) {
-    case 1: return f.template operator()<1>();
-    case 2: return f.template operator()<2>();
-    case 4: return f.template operator()<4>();
-    case 8: return f.template operator()<8>();
-    case 16: return f.template operator()<16>();
-    case 32: return f.template operator()<32>();
-    case 64: return f.template operator()<64>();
-    case 128: return f.template operator()<128>();
-    default: return FP4Q_ERR_UNSUPPORTED;
-  }
-}
-
-// The kernels' view of the plan's channel signs for a configuration with E-element units.
-template <class Cfg>
-ChannelSigns channel_signs(const uint32_t* mask, int64_t K) {
-  if (!mask) return ChannelSigns{nullptr, 1, 0};
-  const int upr = static_cast<int>(K / Cfg::kE);
-  return ChannelSigns{mask, upr, static_cast<int>(Cfg::kUnitsPerStage % upr)};
-}
-
-template <class Cfg>
-fp4q_status launch_rq(RQArgs a, int64_t n_elems, cudaStream_t stream, int64_t K = 0) {
-  a.n_units = n_elems / Cfg::kE;
-  a.signs = channel_signs<Cfg>(a.signs.mask, K);
-  auto kernel = rotate_quantize_kernel<Cfg>;
-  KernelInfo ki;
-  fp4q_status st = kernel_info(kernel, Cfg::kSmemBytes, Cfg::kThreads, &ki);
-  if (st != FP4Q_OK) return st;
-  const int64_t warps_needed = (a.n_units + Cfg::kUnitsPerStage - 1) / Cfg::kUnitsPerStage;
-  int64_t ctas = (warps_needed + Cfg::kWarps - 1) / Cfg::kWarps;
-  const int64_t max_ctas = static_cast<int64_t>(ki.sm_count) * ki.ctas_per_sm;
-  if (ctas > max_ctas) ctas = max_ctas;
-  cudaError_t e = launch_pdl(kernel, dim3(static_cast<unsigned>(ctas)), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, a);
-  if (e != cudaSuccess) return cuda_fail(e, "rotate_quantize launch");
-  return FP4Q_OK;
-}
-
-// ---- tensor-core kernel: TMA tensor map over the rows of one Hadamard block each
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-std::mutex g_encode_mu;
-EncodeTiledFn g_encode = nullptr;
-
 fp4q_status encode_fn(EncodeTiledFn* out) {
   std::lock_guard<std::mutex> lk(g_encode_mu);
   if (!g_encode) {
@@ -166,94 +73,49 @@ fp4q_status encode_fn(EncodeTiledFn* out) {
   return FP4Q_OK;
 }
 
-template <class Cfg>
-fp4q_status launch_mma(const uint16_t* x, int64_t n_elems, const RQArgs& ra, cudaStream_t stream) {
-  EncodeTiledFn enc;
-  fp4q_status st = encode_fn(&enc);
-  if (st != FP4Q_OK) return st;
-  MmaArgs a;
-  a.x = x;
-  a.n_rows = n_elems / Cfg::kBlock;
-  a.n_super = (a.n_rows + Cfg::kRowsPerTile - 1) / Cfg::kRowsPerTile;
-  a.codes = ra.codes;
-  a.scales = ra.scales;
-  a.tensor_scale = ra.tensor_scale;
-  a.partials = ra.partials;
-  a.n_partials = ra.n_partials;
-  a.y_dump = ra.y_dump;
-  CUtensorMap map;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(Cfg::kBlock), static_cast<cuuint64_t>(a.n_rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(Cfg::kBlock) * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(Cfg::kKB), static_cast<cuuint32_t>(Cfg::kBoxRows)};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUtensorMapSwizzle sw = Cfg::kRB == 32   ? CU_TENSOR_MAP_SWIZZLE_32B
-                                : Cfg::kRB == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                                 : CU_TENSOR_MAP_SWIZZLE_128B;
-  CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(x), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) {
-    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
-    return FP4Q_ERR_CUDA;
-  }
-  auto kernel = rotate_quantize_mma_kernel<Cfg>;
-  KernelInfo ki;
-  st = kernel_info(kernel, Cfg::kSmemBytes, Cfg::kThreads, &ki);
-  if (st != FP4Q_OK) return st;
-  // CTAs per SM from measurement (the kernel's CTAs are independent, so a CTA that does not
-  // fit next to the others simply starts later); tensor memory holds 512 columns per SM
-  int per_sm = Cfg::kCtasPerSm;
-  if (per_sm > 512 / Cfg::kTmemCols) per_sm = 512 / Cfg::kTmemCols;
-  int64_t ctas = static_cast<int64_t>(ki.sm_count) * per_sm;
-  if (ctas > a.n_super) ctas = a.n_super;
-  cudaError_t e = launch_pdl(kernel, dim3(static_cast<unsigned>(ctas)), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream,
-                             map, a);
-  if (e != cudaSuccess) return cuda_fail(e, "rotate_quantize (tensor core) launch");
-  return FP4Q_OK;
-}
+}  // namespace host
+}  // namespace fp4q
+
+namespace {
+
+constexpr uint32_t kPlanMagic = 0xF4F4A11Cu;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool valid_plan(fp4q_plan p) { return p != nullptr && p->magic == kPlanMagic; }
 
 // Whether the tensor-core kernel serves this plan.  AUTO takes it for tensors of at least
 // kMmaMinElems elements: below that its fixed start-up (TMEM allocation, H_b, filling a
 // three-stage pipeline) costs more than the butterfly kernel's extra instructions.
 constexpr int64_t kMmaMinElems = int64_t(1) << 22;
-bool mma_capable(fp4q_plan p) { return p->block >= 16 && p->block >= p->group; }
+bool mma_capable(fp4q_plan p) { return p->format != FP4Q_MXFP4_MBS && p->block >= 16 && p->block >= p->group; }
 bool use_mma(fp4q_plan p, int64_t n_elems) {
   if (!mma_capable(p) || p->signs) return false;   // channel signs: butterfly kernel only
   if (p->kernel == FP4Q_KERNEL_TENSOR_CORE) return true;
   return p->kernel == FP4Q_KERNEL_AUTO && n_elems >= kMmaMinElems;
 }
 
-template <int B, int MINU>
-using AmaxCfg = RQConfig<kNV, B, kRuleNvStatic, false, MINU>;
-
 // Number of CTAs the amax pass always launches (and of partial maxima a plan holds): one
 // full wave of the larger of its two instances.
 fp4q_status amax_grid(int b, int* n) {
   return with_block(b, [&]<int B>() -> fp4q_status {
-    KernelInfo k16, k32;
-    fp4q_status st = kernel_info(rotated_amax_kernel<AmaxCfg<B, 16>>, AmaxCfg<B, 16>::kSmemBytes,
-                                 AmaxCfg<B, 16>::kThreads, &k16);
+    int a = 0, c = 0;
+    fp4q_status st = amax_wave<AmaxCfg<B, 16>>(&a);
     if (st != FP4Q_OK) return st;
-    st = kernel_info(rotated_amax_kernel<AmaxCfg<B, 32>>, AmaxCfg<B, 32>::kSmemBytes, AmaxCfg<B, 32>::kThreads, &k32);
+    st = amax_wave<AmaxCfg<B, 32>>(&c);
     if (st != FP4Q_OK) return st;
-    const int a = k16.sm_count * k16.ctas_per_sm, c = k32.sm_count * k32.ctas_per_sm;
     *n = a > c ? a : c;
     return FP4Q_OK;
   });
 }
 
-template <class Cfg>
-fp4q_status launch_amax_cfg(fp4q_plan p, const uint16_t* x, int64_t n_elems, cudaStream_t stream) {
-  cudaError_t e = launch_pdl(rotated_amax_kernel<Cfg>, dim3(p->n_partials), dim3(Cfg::kThreads), Cfg::kSmemBytes,
-                             stream, x, n_elems / Cfg::kE, p->partials, channel_signs<Cfg>(p->signs, p->signs_K));
-  if (e != cudaSuccess) return cuda_fail(e, "amax launch");
-  return FP4Q_OK;
-}
-
 fp4q_status launch_amax(fp4q_plan p, const uint16_t* x, int64_t n_elems, cudaStream_t stream) {
   return with_block(p->block, [&]<int B>() -> fp4q_status {
-    if (n_elems % AmaxCfg<B, 32>::kE == 0) return launch_amax_cfg<AmaxCfg<B, 32>>(p, x, n_elems, stream);
-    return launch_amax_cfg<AmaxCfg<B, 16>>(p, x, n_elems, stream);
+    if (n_elems % AmaxCfg<B, 32>::kE == 0)
+      return launch_amax_cfg<AmaxCfg<B, 32>>(x, n_elems, p->partials, p->n_partials,
+                                             channel_signs<AmaxCfg<B, 32>>(p->signs, p->signs_K), stream, true);
+    return launch_amax_cfg<AmaxCfg<B, 16>>(x, n_elems, p->partials, p->n_partials,
+                                           channel_signs<AmaxCfg<B, 16>>(p->signs, p->signs_K), stream, true);
   });
 }
 
@@ -266,8 +128,10 @@ fp4q_status check_shape(fp4q_plan p, int64_t M, int64_t K) {
 }
 
 fp4q_status rotate_quantize_impl(fp4q_plan p, const void* x, int64_t M, int64_t K, void* codes, void* scales,
-                                 float* tensor_scale, float* y_out, bool dump, void* stream) {
+                                 float* tensor_scale, float* y_out, bool dump, void* stream, void* macro = nullptr) {
   if (!valid_plan(p)) return FP4Q_ERR_ARG;
+  // an MBS plan also stores macro-scale bytes: only fp4q_rotate_quantize_mbs (macro != null) serves it
+  if ((p->format == FP4Q_MXFP4_MBS) != (macro != nullptr)) return FP4Q_ERR_UNSUPPORTED;
   fp4q_status st = check_shape(p, M, K);
   if (st != FP4Q_OK) return st;
   if (M * K == 0) return FP4Q_OK;
@@ -288,6 +152,7 @@ fp4q_status rotate_quantize_impl(fp4q_plan p, const void* x, int64_t M, int64_t 
   a.n_partials = p->n_partials;
   a.y_dump = y_out;
   a.signs = ChannelSigns{p->signs, 1, 0};
+  a.macro = static_cast<uint8_t*>(macro);
   if (p->format == FP4Q_NVFP4 && p->rule == FP4Q_SCALE_NV_DYNAMIC) {
     st = launch_amax(p, a.x, n, s);
     if (st != FP4Q_OK) return st;
@@ -322,6 +187,14 @@ fp4q_status rotate_quantize_impl(fp4q_plan p, const void* x, int64_t M, int64_t 
     });
   }
   return with_block(p->block, [&]<int B>() -> fp4q_status {
+    if (p->format == FP4Q_MXFP4_MBS) {
+      switch (p->rule) {
+        case FP4Q_SCALE_FLOOR_OCP: return launch_rq<RQConfig<kMBS, B, kRuleFloor, false, 128>>(a, n, s, K);
+        case FP4Q_SCALE_CEIL_NOCLIP: return launch_rq<RQConfig<kMBS, B, kRuleCeil, false, 128>>(a, n, s, K);
+        case FP4Q_SCALE_OAS: return launch_rq<RQConfig<kMBS, B, kRuleOas, false, 128>>(a, n, s, K);
+        default: return FP4Q_ERR_UNSUPPORTED;
+      }
+    }
     if (p->format == FP4Q_MXFP4) {
       switch (p->rule) {
         case FP4Q_SCALE_FLOOR_OCP:
@@ -360,6 +233,14 @@ fp4q_status rotate_quantize_impl(fp4q_plan p, const void* x, int64_t M, int64_t 
 template <class F>
 fp4q_status with_rq_cfg(int format, int block, int rule, bool u32, F&& f) {
   return with_block(block, [&]<int B>() -> fp4q_status {
+    if (format == FP4Q_MXFP4_MBS) {
+      switch (rule) {
+        case FP4Q_SCALE_FLOOR_OCP: return f.template operator()<RQConfig<kMBS, B, kRuleFloor, false, 128>>();
+        case FP4Q_SCALE_CEIL_NOCLIP: return f.template operator()<RQConfig<kMBS, B, kRuleCeil, false, 128>>();
+        case FP4Q_SCALE_OAS: return f.template operator()<RQConfig<kMBS, B, kRuleOas, false, 128>>();
+        default: return FP4Q_ERR_UNSUPPORTED;
+      }
+    }
     if (format == FP4Q_MXFP4) {
       switch (rule) {
         case FP4Q_SCALE_FLOOR_OCP: return f.template operator()<RQConfig<kMX, B, kRuleFloor, false>>();
@@ -381,9 +262,9 @@ fp4q_status qe_grid(int format, int block, int rule, int* n) {
   *n = 0;
   for (int u32 = 0; u32 < 2; ++u32) {
     fp4q_status st = with_rq_cfg(format, block, rule, u32 != 0, [&]<class Cfg>() -> fp4q_status {
-      KernelInfo ki;
-      fp4q_status r = kernel_info(quant_error_kernel<Cfg>, Cfg::kSmemBytes, Cfg::kThreads, &ki);
-      if (r == FP4Q_OK && ki.sm_count * ki.ctas_per_sm > *n) *n = ki.sm_count * ki.ctas_per_sm;
+      int w = 0;
+      fp4q_status r = qe_wave<Cfg>(&w);
+      if (r == FP4Q_OK && w > *n) *n = w;
       return r;
     });
     if (st != FP4Q_OK) return st;
@@ -391,41 +272,13 @@ fp4q_status qe_grid(int format, int block, int rule, int* n) {
   return FP4Q_OK;
 }
 
-template <class Cfg>
-fp4q_status launch_qe(fp4q_plan p, QEArgs a, int64_t n_elems, double* out, cudaStream_t stream) {
-  a.n_units = n_elems / Cfg::kE;
-  a.signs = channel_signs<Cfg>(p->signs, p->signs_K);
-  auto kernel = quant_error_kernel<Cfg>;
-  KernelInfo ki;
-  fp4q_status st = kernel_info(kernel, Cfg::kSmemBytes, Cfg::kThreads, &ki);
-  if (st != FP4Q_OK) return st;
-  const int64_t warps_needed = (a.n_units + Cfg::kUnitsPerStage - 1) / Cfg::kUnitsPerStage;
-  int64_t ctas = (warps_needed + Cfg::kWarps - 1) / Cfg::kWarps;
-  const int64_t max_ctas = static_cast<int64_t>(ki.sm_count) * ki.ctas_per_sm;
-  if (ctas > max_ctas) ctas = max_ctas;
-  if (ctas > p->n_err_partials) ctas = p->n_err_partials;
-  a.out = out;
-  cudaError_t e = launch_pdl(kernel, dim3(static_cast<unsigned>(ctas)), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, a);
-  if (e != cudaSuccess) return cuda_fail(e, "quant_error launch");
-  return FP4Q_OK;
-}
-
 // ---- no-allocation NVFP4 dynamic path: partial maxima in a fixed device array
 
-constexpr int kNoAllocMaxPartials = 4096;
 constexpr int kNoAllocMaxDevices = 64;
 std::mutex g_noalloc_mu;
 float* g_noalloc_ptr[kNoAllocMaxDevices] = {};
 
-}  // namespace
-
-// Scratch of the no-allocation entry point (the host name below is only a stand-in; kernels
-// get the device address from cudaGetSymbolAddress).
-static __device__ __align__(256) float g_noalloc_partials[kNoAllocMaxPartials];
-
-namespace {
-
-// Device address of g_noalloc_partials on the current device, looked up once per device.
+// Device address of the no-allocation scratch on the current device, looked up once per device.
 fp4q_status noalloc_scratch(float** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -434,21 +287,11 @@ fp4q_status noalloc_scratch(float** out) {
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
   if (!g_noalloc_ptr[dev]) {
     float* ptr = nullptr;
-    e = cudaGetSymbolAddress(reinterpret_cast<void**>(&ptr), g_noalloc_partials);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+    fp4q_status st = noalloc_partials_symbol(&ptr);
+    if (st != FP4Q_OK) return st;
     g_noalloc_ptr[dev] = ptr;
   }
   *out = g_noalloc_ptr[dev];
-  return FP4Q_OK;
-}
-
-template <class Cfg>
-fp4q_status noalloc_amax_launch(const uint16_t* x, int64_t n_elems, float* partials, int n_partials,
-                                cudaStream_t stream) {
-  rotated_amax_kernel<Cfg><<<n_partials, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(x, n_elems / Cfg::kE, partials,
-                                                                                  ChannelSigns{nullptr, 1, 0});
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "amax launch");
   return FP4Q_OK;
 }
 
@@ -476,7 +319,7 @@ fp4q_status fp4q_rotate_quantize_nvfp4_dynamic_noalloc(const void* x_bf16, int64
   st = amax_grid(hadamard_block, &n_partials);
   if (st != FP4Q_OK) return st;
   if (n_partials > kNoAllocMaxPartials) {
-    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+    std::snprintf(last_error_buffer(), kLastErrorBytes,
                   "fp4q_rotate_quantize_nvfp4_dynamic_noalloc: the amax pass needs %d partial maxima, "
                   "the fixed scratch holds %d",
                   n_partials, kNoAllocMaxPartials);
@@ -495,13 +338,14 @@ fp4q_status fp4q_rotate_quantize_nvfp4_dynamic_noalloc(const void* x_bf16, int64
   a.n_partials = n_partials;
   a.y_dump = nullptr;
   a.signs = ChannelSigns{nullptr, 1, 0};
+  a.macro = nullptr;
   return with_block(hadamard_block, [&]<int B>() -> fp4q_status {
     if (n % 32 == 0) {
-      fp4q_status r = noalloc_amax_launch<AmaxCfg<B, 32>>(x, n, partials, n_partials, s);
+      fp4q_status r = launch_amax_cfg<AmaxCfg<B, 32>>(x, n, partials, n_partials, ChannelSigns{nullptr, 1, 0}, s, false);
       if (r != FP4Q_OK) return r;
       return launch_rq<RQConfig<kNV, B, kRuleNvDynamic, false, 32>>(a, n, s);
     }
-    fp4q_status r = noalloc_amax_launch<AmaxCfg<B, 16>>(x, n, partials, n_partials, s);
+    fp4q_status r = launch_amax_cfg<AmaxCfg<B, 16>>(x, n, partials, n_partials, ChannelSigns{nullptr, 1, 0}, s, false);
     if (r != FP4Q_OK) return r;
     return launch_rq<RQConfig<kNV, B, kRuleNvDynamic, false, 16>>(a, n, s);
   });
@@ -510,7 +354,7 @@ fp4q_status fp4q_rotate_quantize_nvfp4_dynamic_noalloc(const void* x_bf16, int64
 fp4q_status fp4q_plan_create(fp4q_plan* out, int format, int group, int hadamard_block, int scale_rule) {
   if (!out) return FP4Q_ERR_ARG;
   *out = nullptr;
-  if (format == FP4Q_MXFP4) {
+  if (format == FP4Q_MXFP4 || format == FP4Q_MXFP4_MBS) {
     if (group != 32) return FP4Q_ERR_UNSUPPORTED;
     if (scale_rule != FP4Q_SCALE_FLOOR_OCP && scale_rule != FP4Q_SCALE_CEIL_NOCLIP && scale_rule != FP4Q_SCALE_OAS)
       return FP4Q_ERR_UNSUPPORTED;
@@ -530,6 +374,7 @@ fp4q_status fp4q_plan_create(fp4q_plan* out, int format, int group, int hadamard
   p->block = hadamard_block;
   p->rule = scale_rule;
   p->unit = group > hadamard_block ? group : hadamard_block;
+  if (format == FP4Q_MXFP4_MBS) p->unit = 128;   // one macro block per unit (b <= 128)
   p->device = -1;
   p->partials = nullptr;
   p->n_partials = 0;
@@ -621,6 +466,14 @@ fp4q_status fp4q_rotate_quantize(fp4q_plan plan, const void* x_bf16, int64_t M, 
   return rotate_quantize_impl(plan, x_bf16, M, K, codes_out, scales_out, tensor_scale, nullptr, false, stream);
 }
 
+fp4q_status fp4q_rotate_quantize_mbs(fp4q_plan plan, const void* x_bf16, int64_t M, int64_t K, void* codes_out,
+                                     void* scales_out, void* macro_out, void* stream) {
+  if (!valid_plan(plan)) return FP4Q_ERR_ARG;
+  if (plan->format != FP4Q_MXFP4_MBS) return FP4Q_ERR_UNSUPPORTED;
+  if (!macro_out) return M * K == 0 && M >= 0 && K >= 0 ? FP4Q_OK : FP4Q_ERR_ARG;
+  return rotate_quantize_impl(plan, x_bf16, M, K, codes_out, scales_out, nullptr, nullptr, false, stream, macro_out);
+}
+
 fp4q_status fp4q_rotate_quantize_dump(fp4q_plan plan, const void* x_bf16, int64_t M, int64_t K, void* codes_out,
                                       void* scales_out, float* tensor_scale, float* y_out, void* stream) {
   return rotate_quantize_impl(plan, x_bf16, M, K, codes_out, scales_out, tensor_scale, y_out, true, stream);
@@ -638,11 +491,7 @@ fp4q_status fp4q_amax(fp4q_plan plan, const void* x_bf16, int64_t M, int64_t K, 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   st = launch_amax(plan, static_cast<const uint16_t*>(x_bf16), M * K, s);
   if (st != FP4Q_OK) return st;
-  const float* partials = plan->partials;
-  cudaError_t e = launch_pdl(tensor_scale_finalize_kernel, dim3(1), dim3(32), 0, s, partials, plan->n_partials,
-                             tensor_scale_out);
-  if (e != cudaSuccess) return cuda_fail(e, "finalize launch");
-  return FP4Q_OK;
+  return launch_tensor_scale_finalize(plan->partials, plan->n_partials, tensor_scale_out, s);
 }
 
 fp4q_status fp4q_quant_error(fp4q_plan plan, const void* x_bf16, int64_t M, int64_t K, float* tensor_scale,
@@ -656,16 +505,14 @@ fp4q_status fp4q_quant_error(fp4q_plan plan, const void* x_bf16, int64_t M, int6
   if ((x_bf16 && !aligned(x_bf16, 16)) || !aligned(out, 8) || (tensor_scale && !aligned(tensor_scale, 4)))
     return FP4Q_ERR_ALIGN;
   if (!plan->err_partials) {
-    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+    std::snprintf(last_error_buffer(), kLastErrorBytes,
                   "fp4q_quant_error: the plan was made without a CUDA device, so it holds no scratch");
     return FP4Q_ERR_UNSUPPORTED;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t n = M * K;
   if (n == 0) {
-    cudaError_t e = launch_pdl(quant_error_empty_kernel, dim3(1), dim3(32), 0, s,
-                               static_cast<const double*>(plan->err_partials), out);
-    return e == cudaSuccess ? FP4Q_OK : cuda_fail(e, "quant_error finalize launch");
+    return launch_quant_error_empty(plan->err_partials, out, s);
   }
   QEArgs a;
   a.x = static_cast<const uint16_t*>(x_bf16);
@@ -684,9 +531,10 @@ fp4q_status fp4q_quant_error(fp4q_plan plan, const void* x_bf16, int64_t M, int6
                      [&]<class Cfg>() -> fp4q_status { return launch_qe<Cfg>(plan, a, n, out, s); });
 }
 
-fp4q_status fp4q_dequantize(fp4q_plan plan, const void* codes, const void* scales, const float* tensor_scale,
-                            int64_t M, int64_t K, int unrotate, float* out_f32, void* stream) {
-  if (!valid_plan(plan)) return FP4Q_ERR_ARG;
+namespace {
+fp4q_status dequantize_impl(fp4q_plan plan, const void* codes, const void* scales, const void* macro,
+                            const float* tensor_scale, int64_t M, int64_t K, int unrotate, float* out_f32,
+                            void* stream) {
   fp4q_status st = check_shape(plan, M, K);
   if (st != FP4Q_OK) return st;
   if (M * K == 0) return FP4Q_OK;
@@ -696,35 +544,52 @@ fp4q_status fp4q_dequantize(fp4q_plan plan, const void* codes, const void* scale
     return FP4Q_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t n_units = (M * K) / plan->unit;
-  const unsigned grid = static_cast<unsigned>((n_units + 127) / 128);
   const uint8_t* c = static_cast<const uint8_t*>(codes);
   const uint8_t* sc = static_cast<const uint8_t*>(scales);
   st = with_block(plan->block, [&]<int B>() -> fp4q_status {
     // the dequantize kernel's unit is the plan's, E = max(g, b)
     const ChannelSigns dsg = plan->signs ? ChannelSigns{plan->signs, static_cast<int>(plan->signs_K / plan->unit), 0}
                                          : ChannelSigns{nullptr, 1, 0};
-    if (plan->format == FP4Q_MXFP4) {
-      if (unrotate) dequantize_kernel<kMX, B, true><<<grid, 128, 0, s>>>(c, sc, tensor_scale, n_units, out_f32, dsg);
-      else dequantize_kernel<kMX, B, false><<<grid, 128, 0, s>>>(c, sc, tensor_scale, n_units, out_f32, dsg);
+    const uint8_t* mc = static_cast<const uint8_t*>(macro);
+    if (plan->format == FP4Q_MXFP4_MBS) {
+      if (unrotate) return launch_dequantize<kMBS, B, true>(c, sc, tensor_scale, n_units, out_f32, dsg, mc, s);
+      else return launch_dequantize<kMBS, B, false>(c, sc, tensor_scale, n_units, out_f32, dsg, mc, s);
+    } else if (plan->format == FP4Q_MXFP4) {
+      if (unrotate) return launch_dequantize<kMX, B, true>(c, sc, tensor_scale, n_units, out_f32, dsg, mc, s);
+      else return launch_dequantize<kMX, B, false>(c, sc, tensor_scale, n_units, out_f32, dsg, mc, s);
     } else {
-      if (unrotate) dequantize_kernel<kNV, B, true><<<grid, 128, 0, s>>>(c, sc, tensor_scale, n_units, out_f32, dsg);
-      else dequantize_kernel<kNV, B, false><<<grid, 128, 0, s>>>(c, sc, tensor_scale, n_units, out_f32, dsg);
+      if (unrotate) return launch_dequantize<kNV, B, true>(c, sc, tensor_scale, n_units, out_f32, dsg, mc, s);
+      else return launch_dequantize<kNV, B, false>(c, sc, tensor_scale, n_units, out_f32, dsg, mc, s);
     }
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");
-    return FP4Q_OK;
   });
   return st;
+}
+}  // namespace
+
+fp4q_status fp4q_dequantize(fp4q_plan plan, const void* codes, const void* scales, const float* tensor_scale,
+                            int64_t M, int64_t K, int unrotate, float* out_f32, void* stream) {
+  if (!valid_plan(plan)) return FP4Q_ERR_ARG;
+  if (plan->format == FP4Q_MXFP4_MBS) return FP4Q_ERR_UNSUPPORTED;   // needs the macro scales
+  return dequantize_impl(plan, codes, scales, nullptr, tensor_scale, M, K, unrotate, out_f32, stream);
+}
+
+fp4q_status fp4q_dequantize_mbs(fp4q_plan plan, const void* codes, const void* scales, const void* macro, int64_t M,
+                                int64_t K, int unrotate, float* out_f32, void* stream) {
+  if (!valid_plan(plan)) return FP4Q_ERR_ARG;
+  if (plan->format != FP4Q_MXFP4_MBS) return FP4Q_ERR_UNSUPPORTED;
+  if (M * K > 0 && !macro) return FP4Q_ERR_ARG;
+  return dequantize_impl(plan, codes, scales, macro, nullptr, M, K, unrotate, out_f32, stream);
 }
 
 fp4q_status fp4q_device_status(void) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
-  unsigned int v = 0, zero = 0;
-  e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v));
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyFromSymbol");
-  e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero));
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol");
+  unsigned int v = 0;
+  for (fp4q_status (*reader)(unsigned int*) : {status_rq_mx, status_rq_nv, status_mbs, status_qe, status_mma,
+                                               status_dequant}) {
+    fp4q_status st = reader(&v);
+    if (st != FP4Q_OK) return st;
+  }
   return (v & kStatusTimeout) ? FP4Q_ERR_TIMEOUT : FP4Q_OK;
 }
 
@@ -741,7 +606,7 @@ const char* fp4q_status_string(fp4q_status status) {
   return "unknown status";
 }
 
-const char* fp4q_last_cuda_error(void) { return g_last_cuda_error; }
+const char* fp4q_last_cuda_error(void) { return last_error_buffer(); }
 
 int fp4q_version(void) { return 100; }
 

@@ -8,7 +8,8 @@
 namespace fp4q {
 
 // Device-side status word, read back by fp4q_device_status().  Bit 0: a bounded wait ran out.
-__device__ unsigned int g_device_status;
+// One per translation unit (each unit's kernels are a module of their own).
+static __device__ unsigned int g_device_status;
 constexpr unsigned int kStatusTimeout = 1u;
 
 // A wait on an mbarrier gives up after this many nanoseconds (about one second).

@@ -1,0 +1,143 @@
+// Host-side internals shared by the translation units of the library: the plan object,
+// launch helpers, and the declarations of the per-configuration launchers.  The launchers
+// are defined in fp4q_launch.cuh and explicitly instantiated, one kernel family per
+// translation unit (fp4q_inst_*.cu), so that the kernels compile in parallel; the C ABI and
+// its dispatch (fp4q.cu) only call them.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <utility>
+
+#include "fp4q.h"
+#include "fp4q_kernels.cuh"
+#include "fp4q_mma.cuh"
+
+struct fp4q_plan_s {
+  uint32_t magic;
+  int format, group, block, rule;
+  int unit;        // elements per butterfly unit: max(block, group), 128 for MBS
+  int device;
+  float* partials; // NV plans: per-CTA rotated amaxima (device)
+  int n_partials;
+  int kernel;      // fp4q_kernel
+  const uint32_t* signs; // per-channel random signs (device, borrowed; null: none)
+  int64_t signs_K;       // the row length K the signs are for
+  double* err_partials;  // fp4q_quant_error scratch (device; null without a device): per-CTA signal and
+                         // error energy, then a ticket counter
+  int n_err_partials;    // CTAs those hold room for
+};
+
+namespace fp4q {
+namespace host {
+
+// Records the CUDA error message (fp4q_last_cuda_error) and returns FP4Q_ERR_CUDA.
+fp4q_status cuda_fail(cudaError_t e, const char* what);
+// The thread's message buffer behind fp4q_last_cuda_error.
+char* last_error_buffer();
+constexpr int kLastErrorBytes = 512;
+
+// Per (kernel, device) one-time set-up: opt in to the dynamic shared memory the kernel
+// needs and record how many CTAs fit on one SM.
+struct KernelInfo {
+  int ctas_per_sm = 0;
+  int sm_count = 0;
+};
+fp4q_status kernel_info_impl(const void* kernel, int smem_bytes, int threads, KernelInfo* out);
+
+template <class K>
+fp4q_status kernel_info(K kernel, int smem_bytes, int threads, KernelInfo* out) {
+  return kernel_info_impl(reinterpret_cast<const void*>(kernel), smem_bytes, threads, out);
+}
+
+// Launch with programmatic stream serialization, so the kernel's start overlaps the tail of
+// the previous kernel on the stream (the kernels wait on the dependency before touching
+// global memory).
+template <class... KArgs, class... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Call f.template operator()<B>() for the runtime Hadamard block b.
+template <class F>
+fp4q_status with_block(int b, F&& f) {
+  switch (b) {
+    case 1: return f.template operator()<1>();
+    case 2: return f.template operator()<2>();
+    case 4: return f.template operator()<4>();
+    case 8: return f.template operator()<8>();
+    case 16: return f.template operator()<16>();
+    case 32: return f.template operator()<32>();
+    case 64: return f.template operator()<64>();
+    case 128: return f.template operator()<128>();
+    default: return FP4Q_ERR_UNSUPPORTED;
+  }
+}
+
+// The kernels' view of the plan's channel signs for a configuration with E-element units.
+template <class Cfg>
+ChannelSigns channel_signs(const uint32_t* mask, int64_t K) {
+  if (!mask) return ChannelSigns{nullptr, 1, 0};
+  const int upr = static_cast<int>(K / Cfg::kE);
+  return ChannelSigns{mask, upr, static_cast<int>(Cfg::kUnitsPerStage % upr)};
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+// cuTensorMapEncodeTiled from the driver, looked up once.
+fp4q_status encode_fn(EncodeTiledFn* out);
+
+template <int B, int MINU>
+using AmaxCfg = RQConfig<kNV, B, kRuleNvStatic, false, MINU>;
+
+// ---- launchers (fp4q_launch.cuh), instantiated per kernel family
+
+template <class Cfg>
+fp4q_status launch_rq(RQArgs a, int64_t n_elems, cudaStream_t stream, int64_t K = 0);
+template <class Cfg>
+fp4q_status launch_mma(const uint16_t* x, int64_t n_elems, const RQArgs& ra, cudaStream_t stream);
+template <class Cfg>
+fp4q_status launch_qe(fp4q_plan p, QEArgs a, int64_t n_elems, double* out, cudaStream_t stream);
+// CTAs of one full wave of a configuration's error kernel / amax kernel.
+template <class Cfg>
+fp4q_status qe_wave(int* n);
+template <class Cfg>
+fp4q_status amax_wave(int* n);
+// The amax pass over n_partials CTAs (pdl: with programmatic dependent launch).
+template <class Cfg>
+fp4q_status launch_amax_cfg(const uint16_t* x, int64_t n_elems, float* partials, int n_partials, ChannelSigns sg,
+                            cudaStream_t stream, bool pdl);
+template <int FMT, int B, bool UNROTATE>
+fp4q_status launch_dequantize(const uint8_t* codes, const uint8_t* scales, const float* tensor_scale, int64_t n_units,
+                              float* out, ChannelSigns sg, const uint8_t* macro, cudaStream_t stream);
+fp4q_status launch_tensor_scale_finalize(const float* partials, int n, float* out, cudaStream_t stream);
+fp4q_status launch_quant_error_empty(const double* partials, double* out, cudaStream_t stream);
+// Device address of the no-allocation path's fixed scratch (kNoAllocMaxPartials floats).
+constexpr int kNoAllocMaxPartials = 4096;
+fp4q_status noalloc_partials_symbol(float** out);
+
+// Each translation unit with kernels has its own copy of the device status word; these read
+// and clear it, OR-ing the flags into *v.
+fp4q_status status_rq_mx(unsigned int* v);
+fp4q_status status_rq_nv(unsigned int* v);
+fp4q_status status_mbs(unsigned int* v);
+fp4q_status status_qe(unsigned int* v);
+fp4q_status status_mma(unsigned int* v);
+fp4q_status status_dequant(unsigned int* v);
+
+}  // namespace host
+}  // namespace fp4q

@@ -35,7 +35,7 @@
 
 namespace fp4q {
 
-enum : int { kMX = 0, kNV = 1 };
+enum : int { kMX = 0, kNV = 1, kMBS = 2 };   // kMBS: MXFP4 under MBS-Static macro-block scales
 enum : int { kRuleFloor = 0, kRuleCeil = 1, kRuleOas = 2, kRuleNvStatic = 3, kRuleNvDynamic = 4 };
 
 constexpr int ilog2(int v) { return v <= 1 ? 0 : 1 + ilog2(v / 2); }
@@ -109,8 +109,9 @@ struct RQConfig {
   static constexpr int kBlock = B;
   static constexpr int kRule = RULE;
   static constexpr bool kDump = DUMP;
-  static constexpr int kGroup = FMT == kMX ? 32 : 16;
+  static constexpr int kGroup = FMT == kNV ? 16 : 32;
   static constexpr int kE = cmax(cmax(B, kGroup), MINU);  // elements per unit
+  static_assert(FMT != kMBS || kE == 128, "an MBS unit is one 128-element macro block");
   static constexpr int kPairs = kE / 2;                   // packed fp32 pairs per unit
   static constexpr int kChunks = kE / 8;                  // 16-byte chunks per unit
   static constexpr int kGroupsPerUnit = kE / kGroup;
@@ -150,6 +151,7 @@ struct RQArgs {
   int n_partials;
   float* y_dump;           // [n_units * E] when dumping
   ChannelSigns signs;      // per-channel random signs (mask nullptr: none)
+  uint8_t* macro;          // MBS: [n_units] macro-scale bytes
 };
 
 // Per-lane constants of the chunk XOR: tau, and for each of tau's (at most three) bits the
@@ -373,6 +375,21 @@ __device__ __forceinline__ uint32_t e2m1x8_pairs(const f32x2 (&v)[4]) {
   return e2m1x8(e[0], e[1], e[2], e[3], e[4], e[5], e[6], e[7]);
 }
 
+// MBS-Static macro-scale byte from the fp32 macro-block maximum A_M: with
+// fp32(A_M / 6) = 2^E (1 + f), m8 = ceil(256 f) mod 256 (the mantissa rounded up to 8 bits;
+// 256 wraps to 0, which is s_M = 2 with every group exponent one higher).  A_M = 0 gives 0.
+__device__ __forceinline__ uint32_t mbs_macro_byte(float A_M) {
+  const float r = __fdiv_rn(A_M, 6.0f);
+  if (r == 0.0f) return 0u;
+  uint32_t bits = __float_as_uint(r);
+  if (bits < 0x00800000u) bits = __float_as_uint(r * 0x1p64f);   // subnormal: the same mantissa, normalised
+  const uint32_t F = bits & 0x7FFFFFu;                            // f = F / 2^23
+  return ((F + 0x7FFFu) >> 15) & 0xFFu;
+}
+
+// s_M = 1 + m8 / 256 (exact).
+__device__ __forceinline__ float mbs_macro_scale(uint32_t m8) { return 1.0f + static_cast<float>(m8) * (1.0f / 256.0f); }
+
 // Quantize one rotated unit (pairs p, unnormalised butterfly sums) and store its codes and
 // scales.  `lx` undoes the chunk XOR's sign flips.
 template <class Cfg>
@@ -382,6 +399,26 @@ __device__ __forceinline__ void quantize_store_unit(const f32x2 (&p)[Cfg::kPairs
   constexpr float c = Cfg::kC;
   uint32_t words[E / 8];
   uint32_t sbytes[NG];
+  if constexpr (Cfg::kFmt == kMBS) {
+    // the unit is one macro block: y' = RN(y / s_M), then MXFP4 groups on y'
+    const float AM = scale_by_inv_sqrt<Cfg::kBlock>(pairs_amax<E / 2>(p));
+    const uint32_t m8 = mbs_macro_byte(AM);
+    a.macro[unit] = static_cast<uint8_t>(m8);
+    f32x2 yq[E / 2];
+    nv_quotients<Cfg::kBlock, E / 2>(p, nv_divisor<Cfg::kBlock>(mbs_macro_scale(m8)), yq);
+#pragma unroll
+    for (int q = 0; q < NG; ++q) {
+      const int byte = mx_scale_byte<Cfg::kRule>(pairs_amax<G / 2>(&yq[q * G / 2]));
+      sbytes[q] = static_cast<uint32_t>(byte);
+#pragma unroll
+      for (int j = 0; j < G / 8; ++j) {
+        const int chunk = q * (G / 8) + j;
+        f32x2 v[4];
+        mx_quotients<4>(&yq[4 * chunk], byte, 1.0f, v);
+        words[chunk] = e2m1x8_pairs(v) ^ chunk_sign_mask<Cfg::kBlock>(lx, chunk);
+      }
+    }
+  } else {
 #pragma unroll
   for (int q = 0; q < NG; ++q) {
     // group amax of the fp32 rotated values: RN(max |s| / sqrt(b)) = max |RN(s / sqrt(b))|
@@ -411,6 +448,7 @@ __device__ __forceinline__ void quantize_store_unit(const f32x2 (&p)[Cfg::kPairs
         words[chunk] = (e2m1x8_pairs(v) ^ chunk_sign_mask<Cfg::kBlock>(lx, chunk)) & keep;
       }
     }
+  }
   }
   // codes: E/2 bytes per unit
   uint8_t* cp = a.codes + unit * (E / 2);
@@ -659,6 +697,26 @@ __device__ __forceinline__ void unit_energies(const f32x2 (&p)[Cfg::kPairs], flo
                                               double& sig, double& err) {
   constexpr int G = Cfg::kGroup, NG = Cfg::kGroupsPerUnit;
   constexpr float c = Cfg::kC;
+  if constexpr (Cfg::kFmt == kMBS) {
+    constexpr int E = Cfg::kE;
+    const uint32_t m8 = mbs_macro_byte(scale_by_inv_sqrt<Cfg::kBlock>(pairs_amax<E / 2>(p)));
+    const float sM = mbs_macro_scale(m8);
+    const double sM2 = static_cast<double>(sM) * static_cast<double>(sM);
+    f32x2 yq[E / 2];
+    nv_quotients<Cfg::kBlock, E / 2>(p, nv_divisor<Cfg::kBlock>(sM), yq);
+#pragma unroll
+    for (int q = 0; q < NG; ++q) {
+      const int byte = mx_scale_byte<Cfg::kRule>(pairs_amax<G / 2>(&yq[q * G / 2]));
+      f32x2 v[G / 2];
+      mx_quotients<G / 2>(&yq[q * G / 2], byte, 1.0f, v);
+      float gs, ge;
+      group_energies<G / 2>(v, gs, ge);
+      const double X2 = mx_scale_sq(byte) * sM2;
+      sig = fma(static_cast<double>(gs), X2, sig);
+      err = fma(static_cast<double>(ge), X2, err);
+    }
+    return;
+  }
 #pragma unroll
   for (int q = 0; q < NG; ++q) {
     const f32x2* pg = &p[q * G / 2];
@@ -785,7 +843,7 @@ __global__ void __launch_bounds__(Cfg::kThreads) quant_error_kernel(QEArgs a) {
 }
 
 // The same result for an empty X (no CTA to finish): {0, 0, +inf}.  One warp.
-__global__ void quant_error_empty_kernel(const double* __restrict__ partials, double* __restrict__ out) {
+static __global__ void quant_error_empty_kernel(const double* __restrict__ partials, double* __restrict__ out) {
   pdl_launch_dependents();
   pdl_wait();
   qe_final_sum(partials, 0, out);
@@ -819,7 +877,7 @@ __global__ void __launch_bounds__(Cfg::kThreads) rotated_amax_kernel(const uint1
 }
 
 // s_g = fp32(max(partials) / 2688), 1 for an all-zero tensor.  One warp.
-__global__ void tensor_scale_finalize_kernel(const float* __restrict__ partials, int n, float* __restrict__ out) {
+static __global__ void tensor_scale_finalize_kernel(const float* __restrict__ partials, int n, float* __restrict__ out) {
   pdl_launch_dependents();
   pdl_wait();
   float m = 0.0f;
@@ -834,9 +892,10 @@ template <int FMT, int B, bool UNROTATE>
 __global__ void __launch_bounds__(128) dequantize_kernel(const uint8_t* __restrict__ codes,
                                                          const uint8_t* __restrict__ scales,
                                                          const float* __restrict__ tensor_scale, int64_t n_units,
-                                                         float* __restrict__ out, ChannelSigns signs) {
-  constexpr int G = FMT == kMX ? 32 : 16;
-  constexpr int E = cmax(B, G);
+                                                         float* __restrict__ out, ChannelSigns signs,
+                                                         const uint8_t* __restrict__ macro) {
+  constexpr int G = FMT == kNV ? 16 : 32;
+  constexpr int E = FMT == kMBS ? 128 : cmax(B, G);   // MBS: one macro block per unit
   const int64_t unit = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (unit >= n_units) return;
   const float s_g = FMT == kNV ? *tensor_scale : 1.0f;
@@ -846,8 +905,9 @@ __global__ void __launch_bounds__(128) dequantize_kernel(const uint8_t* __restri
   for (int q = 0; q < E / G; ++q) {
     const uint32_t byte = scales[unit * (E / G) + q];
     float S;
-    if (FMT == kMX) {
+    if (FMT != kNV) {
       S = byte == 0 ? __uint_as_float(0x00400000u) : __uint_as_float(byte << 23);   // 2^(byte - 127)
+      if (FMT == kMBS) S *= mbs_macro_scale(macro[unit]);                             // exact: 9-bit s_M
     } else {
       S = e4m3_decode(byte) * s_g;
     }

@@ -22,7 +22,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 FP4Q_OK, FP4Q_ERR_ARG, FP4Q_ERR_SHAPE, FP4Q_ERR_ALIGN, FP4Q_ERR_UNSUPPORTED, FP4Q_ERR_CUDA, FP4Q_ERR_TIMEOUT = range(7)
-FP4Q_MXFP4, FP4Q_NVFP4 = 0, 1
+FP4Q_MXFP4, FP4Q_NVFP4, FP4Q_MXFP4_MBS = 0, 1, 2
 FP4Q_KERNEL_AUTO, FP4Q_KERNEL_BUTTERFLY, FP4Q_KERNEL_TENSOR_CORE = 0, 1, 2
 (FP4Q_SCALE_FLOOR_OCP, FP4Q_SCALE_CEIL_NOCLIP, FP4Q_SCALE_OAS,
  FP4Q_SCALE_NV_STATIC, FP4Q_SCALE_NV_DYNAMIC) = range(5)
@@ -42,6 +42,8 @@ _SIGS = {
     "fp4q_dequantize": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _int, _vp, _vp]),
     "fp4q_rotate_quantize_nvfp4_dynamic_noalloc": (_int, [_vp, _i64, _i64, _int, _vp, _vp, _vp, _vp]),
     "fp4q_quant_error": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp]),
+    "fp4q_rotate_quantize_mbs": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "fp4q_dequantize_mbs": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _int, _vp, _vp]),
     "fp4q_device_status": (_int, []),
     "fp4q_status_string": (ctypes.c_char_p, [_int]),
     "fp4q_last_cuda_error": (ctypes.c_char_p, []),
@@ -169,6 +171,17 @@ def fp4q_quant_error(plan: Plan, x, M: int, K: int, tensor_scale, out_f64, strea
     """out_f64: device float64 [3] <- {signal energy, error energy, QSNR dB}."""
     _check(_lib.fp4q_quant_error(plan.handle, _ptr(x), M, K, _ptr(tensor_scale), _ptr(out_f64), _stream(stream)),
            "fp4q_quant_error")
+
+
+def fp4q_rotate_quantize_mbs(plan: Plan, x, M: int, K: int, codes_out, scales_out, macro_out, stream=None) -> None:
+    _check(_lib.fp4q_rotate_quantize_mbs(plan.handle, _ptr(x), M, K, _ptr(codes_out), _ptr(scales_out),
+                                         _ptr(macro_out), _stream(stream)), "fp4q_rotate_quantize_mbs")
+
+
+def fp4q_dequantize_mbs(plan: Plan, codes, scales, macro, M: int, K: int, unrotate: bool, out_f32,
+                        stream=None) -> None:
+    _check(_lib.fp4q_dequantize_mbs(plan.handle, _ptr(codes), _ptr(scales), _ptr(macro), M, K, int(bool(unrotate)),
+                                    _ptr(out_f32), _stream(stream)), "fp4q_dequantize_mbs")
 
 
 def fp4q_device_status() -> int:

@@ -86,3 +86,32 @@ def run_dequantize(F, plan, codes: np.ndarray, scales: np.ndarray, tensor_scale,
     torch.cuda.synchronize()
     out.check("dequantize out")
     return out.numpy().view(np.float32).reshape(M, K)
+
+
+def run_rotate_quantize_mbs(F, plan, x_bits: np.ndarray):
+    """MBS-Static rotate + quantize: dict(codes (M, K/2), scales (M, K/32), macro (M, K/128))."""
+    M, K = x_bits.shape
+    xd = to_device_bf16(x_bits)
+    codes = Guarded(M * K // 2)
+    scales = Guarded(M * K // 32)
+    macro = Guarded(M * K // 128)
+    F.fp4q_rotate_quantize_mbs(plan, xd, M, K, codes.view, scales.view, macro.view)
+    torch.cuda.synchronize()
+    assert F.fp4q_device_status() == F.FP4Q_OK
+    for g, n in ((codes, "codes"), (scales, "scales"), (macro, "macro")):
+        g.check(n)
+    return {"codes": codes.numpy().reshape(M, K // 2), "scales": scales.numpy().reshape(M, K // 32),
+            "macro": macro.numpy().reshape(M, K // 128)}
+
+
+def run_dequantize_mbs(F, plan, codes: np.ndarray, scales: np.ndarray, macro: np.ndarray, unrotate: bool):
+    M = codes.shape[0]
+    K = codes.shape[1] * 2
+    cd = torch.from_numpy(np.ascontiguousarray(codes)).cuda()
+    sd = torch.from_numpy(np.ascontiguousarray(scales)).cuda()
+    md = torch.from_numpy(np.ascontiguousarray(macro)).cuda()
+    out = Guarded(M * K * 4)
+    F.fp4q_dequantize_mbs(plan, cd, sd, md, M, K, unrotate, out.view)
+    torch.cuda.synchronize()
+    out.check("dequantize_mbs out")
+    return out.numpy().view(np.float32).reshape(M, K)

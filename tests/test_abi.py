@@ -45,7 +45,7 @@ def test_version_and_strings(F):
 
 def test_plan_validation_without_gpu(F):
     for args in [(0, 16, 32, 0), (1, 32, 16, 3), (0, 32, 3, 0), (0, 32, 256, 0), (0, 32, 32, 3), (1, 16, 16, 0),
-                 (2, 32, 32, 0), (0, 32, 0, 0)]:
+                 (3, 32, 32, 0), (0, 32, 0, 0), (2, 16, 32, 0), (2, 32, 32, 3)]:
         with pytest.raises(F.Fp4qError) as e:
             F.fp4q_plan_create(*args)
         assert e.value.status == F.FP4Q_ERR_UNSUPPORTED, args
@@ -82,6 +82,26 @@ def test_sign_validation_without_gpu(F):
     assert ss(p.handle, None, 0) == F.FP4Q_OK                   # cleared
     F.fp4q_plan_set_kernel(p, F.FP4Q_KERNEL_TENSOR_CORE)
     assert ss(p.handle, A, 256) == F.FP4Q_ERR_UNSUPPORTED       # forced tensor-core kernel
+    F.fp4q_plan_destroy(p)
+
+
+def test_mbs_validation_without_gpu(F):
+    p = F.fp4q_plan_create(F.FP4Q_MXFP4_MBS, 32, 32, F.FP4Q_SCALE_OAS)
+    A = 1 << 20
+    mq = lambda *a: F.raw_call("fp4q_rotate_quantize_mbs", *a)
+    assert mq(p.handle, A, 4, 96, A, A, A, None) == F.FP4Q_ERR_SHAPE          # K % 128 (the macro block)
+    assert mq(p.handle, A, 4, 256, A, A, None, None) == F.FP4Q_ERR_ARG        # no macro output
+    assert mq(p.handle, A + 8, 4, 256, A, A, A, None) == F.FP4Q_ERR_ALIGN
+    assert mq(p.handle, A, 0, 256, None, None, None, None) == F.FP4Q_OK       # empty call
+    rq = lambda *a: F.raw_call("fp4q_rotate_quantize", *a)
+    assert rq(p.handle, A, 4, 256, A, A, None, None) == F.FP4Q_ERR_UNSUPPORTED
+    dq = lambda *a: F.raw_call("fp4q_dequantize", *a)
+    assert dq(p.handle, A, A, None, 4, 256, 0, A, None) == F.FP4Q_ERR_UNSUPPORTED
+    dm = lambda *a: F.raw_call("fp4q_dequantize_mbs", *a)
+    assert dm(p.handle, A, A, None, 4, 256, 0, A, None) == F.FP4Q_ERR_ARG
+    mx = F.fp4q_plan_create(F.FP4Q_MXFP4, 32, 32, F.FP4Q_SCALE_OAS)
+    assert mq(mx.handle, A, 4, 256, A, A, A, None) == F.FP4Q_ERR_UNSUPPORTED
+    assert dm(mx.handle, A, A, A, 4, 256, 0, A, None) == F.FP4Q_ERR_UNSUPPORTED
     F.fp4q_plan_destroy(p)
 
 
