@@ -551,3 +551,30 @@ def quant_error(x_bits: np.ndarray, fmt: int, group: int, block: int, rule: int,
     qsnr = math.inf if noise == 0.0 else 10.0 * math.log10(signal / noise) if signal > 0 else -math.inf
     return {"signal": signal, "noise": noise, "qsnr_db": qsnr,
             "mse": noise / (M * K) if M * K else 0.0, "tensor_scale": tensor_scale}
+
+
+# ----------------------------------------------------------------------------------
+# The FP4 GEMM that consumes the codes ([BG] Technische Zusammenfassung, 2. Methodik,
+# GPU-Kernel-Unterstützung: block-scaled FP4 matrix multiplication of the rotated, quantized
+# activations and weights; [BG-en]: the weights absorb the rotation, so the product of the
+# rotated operands is the layer's product)
+# ----------------------------------------------------------------------------------
+
+def gemm_fp4(a_codes: np.ndarray, a_scales: np.ndarray, b_codes: np.ndarray, b_scales: np.ndarray, fmt: int,
+             a_tensor_scale=None, b_tensor_scale=None) -> np.ndarray:
+    """D = A_hat B_hat^T in fp64, with A_hat (M x K) and B_hat (N x K) the exact dequantized
+    operands: q * 2^(byte - 127) for MXFP4, q * E4M3(byte) * s_g for NVFP4 (the product of the
+    two tensor scales is applied once to the result, which is the same number)."""
+    group = 32 if fmt == MXFP4 else 16
+
+    def exact(codes, scales):
+        q = e2m1_decode(unpack_nibbles(codes))
+        R, K = q.shape
+        sc = np.asarray(scales, np.uint8).reshape(R, K // group)
+        S = np.ldexp(1.0, sc.astype(np.int64) - 127) if fmt == MXFP4 else e4m3_decode(sc)
+        return (q.reshape(R, K // group, group) * S[..., None]).reshape(R, K)
+
+    D = exact(a_codes, a_scales) @ exact(b_codes, b_scales).T
+    if fmt == NVFP4:
+        D = D * (float(np.float32(a_tensor_scale)) * float(np.float32(b_tensor_scale)))
+    return D

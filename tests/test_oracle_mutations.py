@@ -293,3 +293,40 @@ def test_mbs_pins_catch_planted_mistake(monkeypatch, name, fn, catchers):
     patch(monkeypatch, name, fn)
     for catcher in catchers:
         assert fails(catcher), f"{catcher.__name__} missed {fn.__name__}"
+
+
+# ---- FP4 GEMM (pins in test_oracle_gemm.py)
+
+import test_oracle_gemm as gpins  # noqa: E402
+
+_orig_gemm = core.gemm_fp4
+
+
+def gemm_no_tensor_scale(a_codes, a_scales, b_codes, b_scales, fmt, a_tensor_scale=None, b_tensor_scale=None):
+    return _orig_gemm(a_codes, a_scales, b_codes, b_scales, fmt, 1.0, 1.0)
+
+
+def gemm_scale_off_by_one(a_codes, a_scales, b_codes, b_scales, fmt, a_tensor_scale=None, b_tensor_scale=None):
+    """Reads the E8M0 byte as 2^(byte - 126)."""
+    if fmt == o.MXFP4:
+        return 4.0 * _orig_gemm(a_codes, a_scales, b_codes, b_scales, fmt)
+    return _orig_gemm(a_codes, a_scales, b_codes, b_scales, fmt, a_tensor_scale, b_tensor_scale)
+
+
+def gemm_b_not_transposed(a_codes, a_scales, b_codes, b_scales, fmt, a_tensor_scale=None, b_tensor_scale=None):
+    D = _orig_gemm(a_codes, a_scales, b_codes, b_scales, fmt, a_tensor_scale, b_tensor_scale)
+    return D.T if D.shape[0] == D.shape[1] else D[:, ::-1]
+
+
+GEMM_MUTATIONS = [
+    (gemm_no_tensor_scale, [gpins.test_hand_worked_nv_dot_product]),
+    (gemm_scale_off_by_one, [gpins.test_hand_worked_mx_dot_product]),
+    (gemm_b_not_transposed, [lambda: gpins.test_gemm_equals_dequantize_then_product(o.MXFP4, 32, 32, 0)]),
+]
+
+
+@pytest.mark.parametrize("fn,catchers", GEMM_MUTATIONS, ids=[m[0].__name__ for m in GEMM_MUTATIONS])
+def test_gemm_pins_catch_planted_mistake(monkeypatch, fn, catchers):
+    patch(monkeypatch, "gemm_fp4", fn)
+    for catcher in catchers:
+        assert fails(catcher), f"pin missed {fn.__name__}"
