@@ -352,6 +352,12 @@ def run_gpu(args):
                 others[ow.name + f" [{alt} kernel]"] = time_other(torch, F, ow, dev, stream, peak, kernel=alt)
         for ow in (W.MX_8K_FLOOR, W.PREFILL_MX):
             others[ow.name + " [MBS-Static]"] = time_mbs(torch, F, ow, dev, stream, peak)
+        gemms = {}
+        for fmt, name in ((W.MXFP4, "mxfp4"), (W.NVFP4, "nvfp4")):
+            for (M, N, K) in ((8192, 8192, 8192), (4096, 14336, 4096), (4096, 4096, 14336)):
+                gemms[f"{name}_{M}x{N}x{K}"] = time_gemm(torch, F, fmt, M, N, K, stream)
+        line_extra_gemm = gemms
+        extra["fp4_gemm"] = line_extra_gemm
 
     if rank == 0:
         cpu = cpu_baseline(w, args) if world == 1 and not args.no_cpu_baseline else None
@@ -432,6 +438,66 @@ def run_kernel_only(args):
     torch.cuda.synchronize()
     assert F.fp4q_device_status() == F.FP4Q_OK
     print(f"kernel-only: {w.name} M={w.M} K={w.K} launches={args.warmup + args.steps}", flush=True)
+
+
+def tensor_peak_fp4():
+    """Dense FP4 tensor peak for a kernel timed alone: the measured bf16 burst figure times
+    the nominal fp4 / bf16 ratio (9 / 2.25 = 4)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return 4.0 * float(json.load(f)["bf16_tflops"]), "measured bf16 burst x 4 (nominal fp4/bf16)"
+    except Exception:
+        return 4.0 * 1590.0, "fallback 1.59 PFLOP/s bf16 x 4"
+
+
+def time_gemm(torch, F, fmt, M, N, K, stream, steps=50):
+    """fp4q_gemm on operands quantized by the library (activations N(0,1) rows, Laplace
+    weights), two rotating operand / output sets (more than L2 in total): TFLOP/s against the
+    FP4 tensor peak."""
+    g = 32 if fmt == W.MXFP4 else 16
+    rule = W.SCALE_FLOOR_OCP if fmt == W.MXFP4 else W.SCALE_NV_DYNAMIC
+    blk = 32 if fmt == W.MXFP4 else 16
+    rng = np.random.default_rng(M + N + K)
+    sets = []
+    for i in range(2):
+        xs_ = []
+        for R, data in ((M, None), (N, None)):
+            plan = F.fp4q_plan_create(fmt, g, blk, rule)
+            x = torch.randn((R, K), dtype=torch.float32, device="cuda", generator=None).to(torch.bfloat16)
+            c = torch.empty((R, K // 2), dtype=torch.uint8, device="cuda")
+            sc = torch.empty((R, K // g), dtype=torch.uint8, device="cuda")
+            ts_ = torch.empty(1, dtype=torch.float32, device="cuda")
+            F.fp4q_rotate_quantize(plan, x, R, K, c, sc, ts_ if fmt == W.NVFP4 else None)
+            del x
+            xs_.append((c, sc, ts_))
+        d = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        sets.append((xs_[0], xs_[1], d))
+    torch.cuda.synchronize()
+    nv = fmt == W.NVFP4
+
+    def launch(i):
+        a, bb, d = sets[i]
+        F.fp4q_gemm(fmt, a[0], a[1], a[2] if nv else None, bb[0], bb[1], bb[2] if nv else None, M, N, K, d,
+                    stream=torch.cuda.current_stream())
+
+    with torch.cuda.stream(stream):
+        gph, g_rem, reps = time_graph_steps(torch, launch, 2, steps, 3, stream)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(reps):
+            gph.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        a1.record(stream)
+    torch.cuda.synchronize()
+    us = a0.elapsed_time(a1) * 1e3 / steps
+    tflops = 2.0 * M * N * K / (us * 1e-6) / 1e12
+    peak, kind = tensor_peak_fp4()
+    del sets
+    torch.cuda.empty_cache()
+    return {"M": M, "N": N, "K": K, "us_per_call": round(us, 2), "TFLOPs": round(tflops, 1),
+            "frac_of_fp4_peak": round(tflops / peak, 4), "fp4_peak_TFLOPs": round(peak, 1), "peak_source": kind,
+            "bound": "tensor"}
 
 
 def time_signed(torch, F, w, xs, codes, scales, ts, stream, peak, steps):

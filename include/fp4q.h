@@ -211,6 +211,24 @@ fp4q_status fp4q_quant_error(fp4q_plan plan, const void* x_bf16, int64_t M, int6
 fp4q_status fp4q_dequantize_mbs(fp4q_plan plan, const void* codes, const void* scales, const void* macro,
                                 int64_t M, int64_t K, int unrotate, float* out_f32, void* stream);
 
+/* Block-scaled FP4 GEMM on the tensor cores: D = alpha * A * B^T, the product the rotated,
+ * quantized activations and weights meet in ("Bridging the Gap Between Promise and Performance
+ * for Microscaling FP4 Quantization", Technische Zusammenfassung, 2. Methodik,
+ * GPU-Kernel-Unterstützung; the weights absorb the rotation, so no inverse rotation is needed).
+ *
+ * format: FP4Q_MXFP4 (E8M0 scales per 32) or FP4Q_NVFP4 (E4M3 scales per 16).  A: the output of
+ * fp4q_rotate_quantize on an activation X [M][K]: a_codes uint8 [M][K/2], a_scales uint8
+ * [M][K/g]; B: the same for the weights W [N][K] (quantized with the same block and signs, so
+ * that (X Q)(W Q)^T = X W^T): b_codes uint8 [N][K/2], b_scales uint8 [N][K/g].  NVFP4: alpha =
+ * *a_tensor_scale * *b_tensor_scale (device fp32); MXFP4: alpha = 1 (the pointers are
+ * ignored).  d_bf16: device bf16 [M][N], row-major, the fp32 accumulator times alpha rounded
+ * to nearest even.  Shapes: M >= 0 any; N a multiple of 32; K a positive multiple of 256 (an
+ * empty M or N launches nothing).  Arrays 16-byte aligned, tensor scales 4-byte aligned.  The
+ * MMA is tcgen05 kind::mxf4 / kind::mxf4nvf4 with fp32 accumulation in tensor memory. */
+fp4q_status fp4q_gemm(int format, const void* a_codes, const void* a_scales, const float* a_tensor_scale,
+                      const void* b_codes, const void* b_scales, const float* b_tensor_scale, int64_t M,
+                      int64_t N, int64_t K, void* d_bf16, void* stream);
+
 /* No-allocation NVFP4 dynamic-scale path.  The paper has no counterpart: this exists for
  * callers that cannot allocate device memory themselves — for example a library loaded into
  * a framework or serving runtime whose own allocator owns all device memory, or a service that

@@ -581,12 +581,38 @@ fp4q_status fp4q_dequantize_mbs(fp4q_plan plan, const void* codes, const void* s
   return dequantize_impl(plan, codes, scales, macro, nullptr, M, K, unrotate, out_f32, stream);
 }
 
+fp4q_status fp4q_gemm(int format, const void* a_codes, const void* a_scales, const float* a_tensor_scale,
+                      const void* b_codes, const void* b_scales, const float* b_tensor_scale, int64_t M, int64_t N,
+                      int64_t K, void* d_bf16, void* stream) {
+  if (format != FP4Q_MXFP4 && format != FP4Q_NVFP4) return FP4Q_ERR_UNSUPPORTED;
+  if (M < 0 || N < 0 || K < 0 || N % 32 != 0 || K % 256 != 0) return FP4Q_ERR_SHAPE;
+  if (M > (int64_t(1) << 31) || N > (int64_t(1) << 31) || (K > 0 && (M > (int64_t(1) << 40) / K ||
+                                                                        N > (int64_t(1) << 40) / K)))
+    return FP4Q_ERR_SHAPE;
+  if (M == 0 || N == 0) return FP4Q_OK;
+  if (K == 0) return FP4Q_ERR_SHAPE;   // an empty reduction: no MMA would write the accumulator
+  if (!a_codes || !a_scales || !b_codes || !b_scales || !d_bf16) return FP4Q_ERR_ARG;
+  if (format == FP4Q_NVFP4 && (!a_tensor_scale || !b_tensor_scale)) return FP4Q_ERR_ARG;
+  if (!aligned(a_codes, 16) || !aligned(a_scales, 16) || !aligned(b_codes, 16) || !aligned(b_scales, 16) ||
+      !aligned(d_bf16, 16) || (a_tensor_scale && !aligned(a_tensor_scale, 4)) ||
+      (b_tensor_scale && !aligned(b_tensor_scale, 4)))
+    return FP4Q_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const auto* ac = static_cast<const uint8_t*>(a_codes);
+  const auto* as = static_cast<const uint8_t*>(a_scales);
+  const auto* bc = static_cast<const uint8_t*>(b_codes);
+  const auto* bs = static_cast<const uint8_t*>(b_scales);
+  auto* d = static_cast<uint16_t*>(d_bf16);
+  if (format == FP4Q_MXFP4) return launch_gemm<kMX>(ac, as, a_tensor_scale, bc, bs, b_tensor_scale, M, N, K, d, s);
+  return launch_gemm<kNV>(ac, as, a_tensor_scale, bc, bs, b_tensor_scale, M, N, K, d, s);
+}
+
 fp4q_status fp4q_device_status(void) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
   unsigned int v = 0;
   for (fp4q_status (*reader)(unsigned int*) : {status_rq_mx, status_rq_nv, status_mbs, status_qe, status_mma,
-                                               status_dequant}) {
+                                               status_dequant, status_gemm}) {
     fp4q_status st = reader(&v);
     if (st != FP4Q_OK) return st;
   }

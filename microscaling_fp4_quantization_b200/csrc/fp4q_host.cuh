@@ -14,6 +14,7 @@
 #include "fp4q.h"
 #include "fp4q_kernels.cuh"
 #include "fp4q_mma.cuh"
+#include "fp4q_gemm.cuh"
 
 struct fp4q_plan_s {
   uint32_t magic;
@@ -124,6 +125,11 @@ fp4q_status launch_amax_cfg(const uint16_t* x, int64_t n_elems, float* partials,
 template <int FMT, int B, bool UNROTATE>
 fp4q_status launch_dequantize(const uint8_t* codes, const uint8_t* scales, const float* tensor_scale, int64_t n_units,
                               float* out, ChannelSigns sg, const uint8_t* macro, cudaStream_t stream);
+// The block-scaled FP4 GEMM D = alpha A B^T (bf16 D [M][N]); arguments validated by the caller.
+template <int FMT>
+fp4q_status launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_ts, const uint8_t* b_codes,
+                        const uint8_t* b_scales, const float* b_ts, int64_t M, int64_t N, int64_t K, uint16_t* d,
+                        cudaStream_t stream);
 fp4q_status launch_tensor_scale_finalize(const float* partials, int n, float* out, cudaStream_t stream);
 fp4q_status launch_quant_error_empty(const double* partials, double* out, cudaStream_t stream);
 // Device address of the no-allocation path's fixed scratch (kNoAllocMaxPartials floats).
@@ -138,6 +144,7 @@ fp4q_status status_mbs(unsigned int* v);
 fp4q_status status_qe(unsigned int* v);
 fp4q_status status_mma(unsigned int* v);
 fp4q_status status_dequant(unsigned int* v);
+fp4q_status status_gemm(unsigned int* v);
 
 }  // namespace host
 }  // namespace fp4q

@@ -134,6 +134,57 @@ fp4q_status launch_dequantize(const uint8_t* codes, const uint8_t* scales, const
   return FP4Q_OK;
 }
 
+template <int FMT>
+fp4q_status launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_ts, const uint8_t* b_codes,
+                        const uint8_t* b_scales, const float* b_ts, int64_t M, int64_t N, int64_t K, uint16_t* d,
+                        cudaStream_t stream) {
+  using Cfg = GemmConfig<FMT>;
+  EncodeTiledFn enc;
+  fp4q_status st = encode_fn(&enc);
+  if (st != FP4Q_OK) return st;
+  // code tiles: bytes [rows][K/2], boxes of 128 bytes (256 E2M1 values) x 128 or 256 rows,
+  // 128-byte swizzled; rows past the end read as zeros
+  CUtensorMap maps[2];
+  const uint8_t* srcs[2] = {a_codes, b_codes};
+  const int64_t rows[2] = {M, N};
+  const cuuint32_t box_rows[2] = {static_cast<cuuint32_t>(Cfg::kBM), static_cast<cuuint32_t>(Cfg::kBN)};
+  for (int i = 0; i < 2; ++i) {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows[i])};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(Cfg::kBK / 2), box_rows[i]};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(&maps[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(srcs[i]), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+      std::snprintf(last_error_buffer(), kLastErrorBytes, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+      return FP4Q_ERR_CUDA;
+    }
+  }
+  GemmArgs a;
+  a.a_scales = a_scales;
+  a.b_scales = b_scales;
+  a.a_tensor_scale = a_ts;
+  a.b_tensor_scale = b_ts;
+  a.d = d;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.tiles_m = static_cast<int>((M + Cfg::kBM - 1) / Cfg::kBM);
+  a.tiles_n = static_cast<int>((N + Cfg::kBN - 1) / Cfg::kBN);
+  a.k_stages = static_cast<int>(K / Cfg::kBK);
+  auto kernel = gemm_fp4_kernel<Cfg>;
+  KernelInfo ki;
+  st = kernel_info(kernel, Cfg::kSmemBytes, Cfg::kThreads, &ki);
+  if (st != FP4Q_OK) return st;
+  int64_t ctas = static_cast<int64_t>(a.tiles_m) * a.tiles_n;
+  if (ctas > ki.sm_count) ctas = ki.sm_count;   // one persistent CTA per SM (its shared memory fills the SM)
+  cudaError_t e = launch_pdl(kernel, dim3(static_cast<unsigned>(ctas)), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream,
+                             maps[0], maps[1], a);
+  if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
+  return FP4Q_OK;
+}
+
 }  // namespace host
 }  // namespace fp4q
 

@@ -44,6 +44,7 @@ _SIGS = {
     "fp4q_quant_error": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp]),
     "fp4q_rotate_quantize_mbs": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp]),
     "fp4q_dequantize_mbs": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _int, _vp, _vp]),
+    "fp4q_gemm": (_int, [_int, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp]),
     "fp4q_device_status": (_int, []),
     "fp4q_status_string": (ctypes.c_char_p, [_int]),
     "fp4q_last_cuda_error": (ctypes.c_char_p, []),
@@ -182,6 +183,13 @@ def fp4q_dequantize_mbs(plan: Plan, codes, scales, macro, M: int, K: int, unrota
                         stream=None) -> None:
     _check(_lib.fp4q_dequantize_mbs(plan.handle, _ptr(codes), _ptr(scales), _ptr(macro), M, K, int(bool(unrotate)),
                                     _ptr(out_f32), _stream(stream)), "fp4q_dequantize_mbs")
+
+
+def fp4q_gemm(fmt: int, a_codes, a_scales, a_tensor_scale, b_codes, b_scales, b_tensor_scale, M: int, N: int,
+              K: int, d_bf16, stream=None) -> None:
+    """D [M, N] bf16 = alpha * A B^T from the quantizer's codes and scales of A [M, K] and B [N, K]."""
+    _check(_lib.fp4q_gemm(fmt, _ptr(a_codes), _ptr(a_scales), _ptr(a_tensor_scale), _ptr(b_codes), _ptr(b_scales),
+                          _ptr(b_tensor_scale), M, N, K, _ptr(d_bf16), _stream(stream)), "fp4q_gemm")
 
 
 def fp4q_device_status() -> int:

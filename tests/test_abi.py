@@ -105,6 +105,20 @@ def test_mbs_validation_without_gpu(F):
     F.fp4q_plan_destroy(p)
 
 
+def test_gemm_validation_without_gpu(F):
+    gm = lambda *a: F.raw_call("fp4q_gemm", *a)
+    A = 1 << 20
+    assert gm(5, A, A, None, A, A, None, 128, 256, 256, A, None) == F.FP4Q_ERR_UNSUPPORTED
+    assert gm(F.FP4Q_MXFP4, A, A, None, A, A, None, 128, 250, 256, A, None) == F.FP4Q_ERR_SHAPE   # N % 32
+    assert gm(F.FP4Q_MXFP4, A, A, None, A, A, None, 128, 256, 300, A, None) == F.FP4Q_ERR_SHAPE   # K % 256
+    assert gm(F.FP4Q_MXFP4, A, A, None, A, A, None, 128, 256, 0, A, None) == F.FP4Q_ERR_SHAPE     # empty K
+    assert gm(F.FP4Q_MXFP4, A, A, None, A, A, None, 0, 256, 256, None, None) == F.FP4Q_OK         # empty M
+    assert gm(F.FP4Q_MXFP4, None, A, None, A, A, None, 128, 256, 256, A, None) == F.FP4Q_ERR_ARG
+    assert gm(F.FP4Q_NVFP4, A, A, None, A, A, A, 128, 256, 256, A, None) == F.FP4Q_ERR_ARG       # tensor scale
+    assert gm(F.FP4Q_MXFP4, A + 8, A, None, A, A, None, 128, 256, 256, A, None) == F.FP4Q_ERR_ALIGN
+    assert gm(F.FP4Q_MXFP4, A, A, None, A, A, None, 128, 256, 256, A + 2, None) == F.FP4Q_ERR_ALIGN
+
+
 def test_call_validation_without_gpu(F):
     p = F.fp4q_plan_create(F.FP4Q_MXFP4, 32, 128, F.FP4Q_SCALE_FLOOR_OCP)
     rq = lambda *a: F.raw_call("fp4q_rotate_quantize", *a)
