@@ -32,9 +32,10 @@
 //               waits for the slot, so four stages of scale loads are in flight.
 // In tensor memory, the scale factor of row r (r < 128) and scale j of one MMA sits in lane
 // r mod 32 (and its copies in the other lane quarters), column r / 32, byte j; B's 256 rows
-// take 8 columns.  MXFP4's two scales per MMA take bytes 0 and
-// 1 of their cells (scale-factor id 0 throughout).  Every wait is bounded in time; a wait that runs out records
-// kStatusTimeout and the CTA lets its issued copies and MMAs land before it frees TMEM.
+// take 8 columns.  MXFP4's two scales per MMA take half a cell: MMA 2q uses bytes 0-1 of
+// cell q (scale-factor id 0) and MMA 2q + 1 bytes 2-3 (id 2).  Every wait is bounded in time;
+// a wait that runs out records kStatusTimeout and the CTA lets its issued copies and MMAs land
+// before it frees TMEM.
 #pragma once
 
 #include <cuda.h>
@@ -55,13 +56,18 @@ struct GemmConfig {
   static constexpr int kStages = 4;
   static constexpr int kABytes = kBM * kBK / 2;            // 16 KB of codes
   static constexpr int kBBytes = kBN * kBK / 2;            // 32 KB of codes
-  static constexpr int kSfaBytes = kKSteps * 512;          // one 32 x 16 B block per MMA
-  static constexpr int kSfbBytes = kKSteps * 1024;         // two per MMA (up to 256 rows)
-  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+  // MXFP4's two scales per MMA share a 32-bit cell with the next MMA's (bytes 0-1 and 2-3,
+  // told apart by the scale-factor id), so a cell column serves two MMAs; NVFP4's four fill it
+  static constexpr int kMmasPerCell = FMT == kMX ? 2 : 1;
+  static constexpr int kCellSteps = kKSteps / kMmasPerCell;   // cell columns per stage and row group
+  static constexpr int kSfaBytes = kCellSteps * 512;       // one 32 x 16 B block per cell step
+  static constexpr int kSfbBytes = kCellSteps * 1024;      // two per cell step (up to 256 rows)
+  static constexpr int kSfPad = (1024 - (kABytes + kBBytes + kSfaBytes + kSfbBytes) % 1024) % 1024;
+  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes + kSfPad;
   static_assert(kStageBytes % 1024 == 0, "stages stay 1024-byte aligned (128-byte swizzle atoms)");
   static constexpr int kBarOffset = kStages * kStageBytes;
   static constexpr int kSmemBytes = 1024 + kBarOffset + 256;
-  static constexpr int kSfColsPerStage = kKSteps * (4 + 8);
+  static constexpr int kSfColsPerStage = kCellSteps * (4 + 8);
   static constexpr int kSfCol0 = 0;                        // two scale-factor buffers, then
   static constexpr int kAccCol0 = 2 * kSfColsPerStage;     // the fp32 accumulator(s) of kBN columns
   static constexpr int kTmemCols = 512;
@@ -121,8 +127,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
-// The four 4-byte scale words of one row for the stage's four MMAs (word kk: the scales of
-// K elements 64 kk .. 64 kk + 63 of the stage, low bytes first); zero for rows past the end.
+// The 4-byte scale cells of one row for the stage (NVFP4: cell kk = the scales of K elements
+// 64 kk .. 64 kk + 63 of the stage; MXFP4: cells 0 and 1, two MMAs each); zero for rows past
+// the end.
 template <int FMT>
 __device__ __forceinline__ uint4 stage_scale_words(const uint8_t* scales, int64_t row, int64_t rows, int64_t K,
                                                    int ks) {
@@ -131,9 +138,9 @@ __device__ __forceinline__ uint4 stage_scale_words(const uint8_t* scales, int64_
     // 16 scale bytes: 4 per MMA
     return __ldg(reinterpret_cast<const uint4*>(scales + row * (K / 16) + static_cast<int64_t>(ks) * 16));
   } else {
-    // 8 scale bytes: 2 per MMA, in bytes 0 and 1 of each word
+    // 8 scale bytes: 2 per MMA; word q holds MMAs 2q (bytes 0-1) and 2q + 1 (bytes 2-3)
     const uint2 v = __ldg(reinterpret_cast<const uint2*>(scales + row * (K / 32) + static_cast<int64_t>(ks) * 8));
-    return make_uint4(v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16);
+    return make_uint4(v.x, v.y, 0u, 0u);
   }
 }
 
@@ -239,16 +246,18 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
       const uint32_t la = sfa_blk(slot) + lane * 16, lb = sfb_blk(slot) + lane * 16;
       sts128(la + 0 * 512, wa[0].x, wa[1].x, wa[2].x, wa[3].x);
       sts128(la + 1 * 512, wa[0].y, wa[1].y, wa[2].y, wa[3].y);
-      sts128(la + 2 * 512, wa[0].z, wa[1].z, wa[2].z, wa[3].z);
-      sts128(la + 3 * 512, wa[0].w, wa[1].w, wa[2].w, wa[3].w);
       sts128(lb + 0 * 1024, wb[0].x, wb[1].x, wb[2].x, wb[3].x);
       sts128(lb + 0 * 1024 + 512, wb[4].x, wb[5].x, wb[6].x, wb[7].x);
       sts128(lb + 1 * 1024, wb[0].y, wb[1].y, wb[2].y, wb[3].y);
       sts128(lb + 1 * 1024 + 512, wb[4].y, wb[5].y, wb[6].y, wb[7].y);
-      sts128(lb + 2 * 1024, wb[0].z, wb[1].z, wb[2].z, wb[3].z);
-      sts128(lb + 2 * 1024 + 512, wb[4].z, wb[5].z, wb[6].z, wb[7].z);
-      sts128(lb + 3 * 1024, wb[0].w, wb[1].w, wb[2].w, wb[3].w);
-      sts128(lb + 3 * 1024 + 512, wb[4].w, wb[5].w, wb[6].w, wb[7].w);
+      if constexpr (Cfg::kCellSteps == 4) {
+        sts128(la + 2 * 512, wa[0].z, wa[1].z, wa[2].z, wa[3].z);
+        sts128(la + 3 * 512, wa[0].w, wa[1].w, wa[2].w, wa[3].w);
+        sts128(lb + 2 * 1024, wb[0].z, wb[1].z, wb[2].z, wb[3].z);
+        sts128(lb + 2 * 1024 + 512, wb[4].z, wb[5].z, wb[6].z, wb[7].z);
+        sts128(lb + 3 * 1024, wb[0].w, wb[1].w, wb[2].w, wb[3].w);
+        sts128(lb + 3 * 1024 + 512, wb[4].w, wb[5].w, wb[6].w, wb[7].w);
+      }
       fence_proxy_async_smem();   // the tensor core's copy reads these bytes through the async proxy
       __syncwarp();
       if (lane == 0) mbar_arrive(sfull_bar(slot));
@@ -275,17 +284,24 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
           }
           tc_fence_after();
           const uint32_t sf = tmem_base + Cfg::kSfCol0 + static_cast<uint32_t>(it & 1) * Cfg::kSfColsPerStage;
+          constexpr int CS = Cfg::kCellSteps;
 #pragma unroll
-          for (int kk = 0; kk < KS; ++kk) {
-            utccp_32x128b_x4(sf + kk * 4, umma_smem_desc(sfa_blk(s) + kk * 512, 128, 0));
-            utccp_32x128b_x4(sf + 4 * KS + kk * 8, umma_smem_desc(sfb_blk(s) + kk * 1024, 128, 0));
-            utccp_32x128b_x4(sf + 4 * KS + kk * 8 + 4, umma_smem_desc(sfb_blk(s) + kk * 1024 + 512, 128, 0));
+          for (int c = 0; c < CS; ++c) {
+            utccp_32x128b_x4(sf + c * 4, umma_smem_desc(sfa_blk(s) + c * 512, 128, 0));
+            utccp_32x128b_x4(sf + 4 * CS + c * 8, umma_smem_desc(sfb_blk(s) + c * 1024, 128, 0));
+            utccp_32x128b_x4(sf + 4 * CS + c * 8 + 4, umma_smem_desc(sfb_blk(s) + c * 1024 + 512, 128, 0));
           }
 #pragma unroll
           for (int kk = 0; kk < KS; ++kk) {
+            // the MMA's scales start at byte `id` of their cells: the id goes in the instruction
+            // descriptor and in the top two bits of the TMEM addresses
+            const int c = kk / Cfg::kMmasPerCell;
+            const uint32_t id = static_cast<uint32_t>((kk % Cfg::kMmasPerCell) * 2);
+            const uint32_t idesc = Cfg::kIdesc | (id << 4) | (id << 29);
             umma_fp4_block_scaled<Cfg::kFmt>(acc, umma_smem_desc(a_tile(s) + kk * 32, 1024, 2),
-                                             umma_smem_desc(b_tile(s) + kk * 32, 1024, 2), Cfg::kIdesc, sf + kk * 4,
-                                             sf + 4 * KS + kk * 8, (ks | kk) != 0 ? 1u : 0u);
+                                             umma_smem_desc(b_tile(s) + kk * 32, 1024, 2), idesc,
+                                             (sf + c * 4) | (id << 30), (sf + 4 * CS + c * 8) | (id << 30),
+                                             (ks | kk) != 0 ? 1u : 0u);
           }
           umma_commit(empty_bar(s));
         }
