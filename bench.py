@@ -53,7 +53,7 @@ L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 SPEC_HBM_GBS = 8000.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "rotate_quantize_nvfp4_b16_4096x4096.md")
-KERNEL_SOURCES = ["fp4q.cu", "fp4q_kernels.cuh", "fp4q_device.cuh", "fp4q_mma.cuh"]
+KERNEL_SOURCES = ["fp4q.cu", "fp4q_kernels.cuh", "fp4q_device.cuh", "fp4q_mma.cuh", "fp4q_launch.cuh"]
 
 
 def kernel_source_hash() -> str:
@@ -528,6 +528,35 @@ def time_signed(torch, F, w, xs, codes, scales, ts, stream, peak, steps):
             "bytes_per_call": nbytes, "kernel": "butterfly"}
 
 
+def run_gemm_only(args):
+    """W + K launches of fp4q_gemm (a case for profilers): N(0, 1) activations [M][K] and weights
+    [N][K] quantized by the library (block 32 floor for MXFP4, 16 dynamic for NVFP4)."""
+    import torch
+    from microscaling_fp4_quantization_b200 import fp4q as F
+    torch.cuda.set_device(0)
+    M, N, K = args.gemm
+    fmt = W.MXFP4 if args.gemm_format == "mxfp4" else W.NVFP4
+    g = 32 if fmt == W.MXFP4 else 16
+    rule = W.SCALE_FLOOR_OCP if fmt == W.MXFP4 else W.SCALE_NV_DYNAMIC
+    ops = []
+    for R in (M, N):
+        plan = F.fp4q_plan_create(fmt, g, g, rule)
+        x = torch.randn((R, K), device="cuda").to(torch.bfloat16)
+        c = torch.empty((R, K // 2), dtype=torch.uint8, device="cuda")
+        sc = torch.empty((R, K // g), dtype=torch.uint8, device="cuda")
+        t = torch.empty(1, dtype=torch.float32, device="cuda")
+        F.fp4q_rotate_quantize(plan, x, R, K, c, sc, t if fmt == W.NVFP4 else None)
+        ops.append((c, sc, t))
+    d = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    nv = fmt == W.NVFP4
+    for _ in range(args.warmup + args.steps):
+        F.fp4q_gemm(fmt, ops[0][0], ops[0][1], ops[0][2] if nv else None, ops[1][0], ops[1][1],
+                    ops[1][2] if nv else None, M, N, K, d)
+    torch.cuda.synchronize()
+    assert F.fp4q_device_status() == F.FP4Q_OK
+    print(f"gemm-only: {args.gemm_format} {M}x{N}x{K} launches={args.warmup + args.steps}", flush=True)
+
+
 def time_quant_error(torch, F, w, plan, xs, ts, stream, peak, steps):
     """fp4q_quant_error on the workload's rotating inputs: device time per call (one kernel),
     GB/s on its algorithmic bytes (X read once, 24 bytes out) and the QSNR."""
@@ -721,11 +750,16 @@ def main():
                     help="which rotate + quantize kernel the plan uses")
     ap.add_argument("--kernel-only", action="store_true",
                     help="only W + K plain launches of the workload (a case for profilers), no JSON line")
+    ap.add_argument("--gemm", type=int, nargs=3, metavar=("M", "N", "K"), default=None,
+                    help="with --kernel-only: W + K launches of fp4q_gemm on operands the library quantized")
+    ap.add_argument("--gemm-format", default="nvfp4", choices=["mxfp4", "nvfp4"])
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.kernel_only and args.gemm:
+        run_gemm_only(args)
     elif args.kernel_only:
         run_kernel_only(args)
     else:
