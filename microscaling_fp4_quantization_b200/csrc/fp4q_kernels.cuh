@@ -519,8 +519,16 @@ __device__ __forceinline__ bool stream_units(const uint16_t* __restrict__ x, int
     for (int s = 0; s < S; ++s) mbar_init(bar0 + 8u * s, 1);
     fence_mbar_init();
   }
-  // Nothing below reads or writes global memory before the kernels this one depends on
-  // (for example the producer of x) have finished.
+  // Before the grid dependency only a hint: ask L2 for this warp's first S stages, so their
+  // DRAM traffic overlaps the end of the kernel this one follows.  Nothing below reads or writes
+  // global memory before the kernels this one depends on (for example the producer of x) have
+  // finished.
+  if (lane == 0)
+    for (int64_t t = 0; t < S && t < n_stages; ++t) {
+      const int64_t us = u0 + t * SU;
+      const int64_t cnt = (u1 - us) < SU ? (u1 - us) : SU;
+      bulk_prefetch_l2(x + us * E, static_cast<uint32_t>(cnt) * (E * 2));
+    }
   pdl_wait();
   if (lane == 0)
     for (int64_t t = 0; t < S && t < n_stages; ++t) issue(t);

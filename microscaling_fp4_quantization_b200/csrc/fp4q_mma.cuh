@@ -19,7 +19,8 @@
 //                 block, or a part of one) and does the amax, scale, E2M1 rounding, packing and
 //                 stores of it in its registers; it frees the buffer as soon as its slice is read.
 // All roles wait on the grid dependency (programmatic dependent launch) before touching global
-// memory, so the set-up overlaps the end of the kernel this one follows.
+// memory, so the set-up overlaps the end of the kernel this one follows; before it the producer
+// only asks L2 to prefetch its first stages.
 // H_b is written into shared memory once per CTA, in the same swizzled layout.
 // Every wait is bounded in time; a wait that runs out records kStatusTimeout, and the CTA
 // lets its issued copies and MMAs land before it frees TMEM and leaves.
@@ -116,6 +117,11 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
           dst),
       "l"(map), "r"(x), "r"(y), "r"(bar)
       : "memory");
+}
+
+// The box at (x, y) of a 2-D tensor map into L2 (a hint, as bulk_prefetch_l2).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y) : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
@@ -246,6 +252,26 @@ __global__ void __launch_bounds__(Cfg::kThreads, 2)
   if (warp == 0) {
     // ---------------- producer
     if (lane == 0) {
+      // Before the grid dependency: ask L2 for this CTA's first S super-tiles, so their DRAM
+      // traffic overlaps the end of the kernel this one follows.  Only a hint: the copies below
+      // still wait on the dependency, and L2 holds any write that kernel makes meanwhile.
+      {
+        int64_t i = 0;
+        for (int64_t t = blockIdx.x; t < n_super && i < S; t += gridDim.x, ++i) {
+          const int64_t row0 = t * Cfg::kRowsPerTile;
+          if constexpr (Cfg::kBulk) {
+            const int64_t rows = (a.n_rows - row0) < Cfg::kRowsPerTile ? (a.n_rows - row0) : Cfg::kRowsPerTile;
+            bulk_prefetch_l2(a.x + row0 * B, static_cast<uint32_t>(rows) * (2 * B));
+          } else if constexpr (B >= 128) {
+            tma_prefetch_2d(&xmap, 0, static_cast<int>(row0));
+            tma_prefetch_2d(&xmap, 64, static_cast<int>(row0));
+          } else {
+#pragma unroll
+            for (int k = 0; k < Cfg::kBoxes; ++k)
+              if (row0 + k * Cfg::kBoxRows < a.n_rows) tma_prefetch_2d(&xmap, 0, static_cast<int>(row0 + k * Cfg::kBoxRows));
+          }
+        }
+      }
       pdl_wait();   // x may come from the kernel this one depends on
       int64_t i = 0;
       bool ok = true;
