@@ -161,6 +161,22 @@ def dist_setup():
     return world, rank, local
 
 
+def max_over_ranks(torch, ms: float, world: int, device) -> float:
+    """The slowest rank's time.  Every rank calls it, in the same order (one all-reduce)."""
+    if world == 1:
+        return ms
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world: int, bytes_per_step: int, steps: int, ms: float) -> float:
+    """Weak scaling: every rank processes its own replica, so the job moves world x the bytes
+    of one replica in the slowest rank's time."""
+    return world * bytes_per_step * steps / (ms * 1e-3) / 1e9
+
+
 def time_graph_steps(torch, launch, n_buf: int, steps: int, warmup: int, stream):
     """Capture `launch(i)` for i in 0..G-1 into a CUDA graph (i cycles the buffers) and time
     `steps` steps.  Returns (ms total, n_graph_launches)."""
@@ -256,14 +272,9 @@ def run_gpu(args):
         import torch.distributed as dist
         dist.barrier()
     sampler.stop()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(torch, e0.elapsed_time(e1), world, dev)
     ms_step = ms / args.steps
-    value = world * bytes_call * args.steps / (ms * 1e-3) / 1e9
+    value = whole_job_gbs(world, bytes_call, args.steps, ms)
     kernel_us = ms_step * 1e3
     peak, peak_kind = measured_peak()
 
@@ -329,13 +340,8 @@ def run_gpu(args):
             e2e_step()
         b1.record(cur)
         torch.cuda.synchronize()
-        e_ms = b0.elapsed_time(b1)
-        if world > 1:
-            import torch.distributed as dist
-            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": round(world * bytes_call * n_e2e / (e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+        e_ms = max_over_ranks(torch, b0.elapsed_time(b1), world, dev)
+        e2e = {"value": round(whole_job_gbs(world, bytes_call, n_e2e, e_ms), 2), "unit": "GB/s",
                "h2d_bytes_per_step": int(x_host.numel() * 2),
                "d2h_bytes_per_step": int(codes_h.numel() + scales_h.numel()), "steps": n_e2e}
 
