@@ -306,7 +306,7 @@ def run_gpu(args):
                            "bytes_per_call": nbytes}
         extra["dynamic_mode"]["note"] = "reads X twice (amax pass, then quantize); bytes are the algorithmic ones"
 
-    # the randomised rotation (per-channel random signs; butterfly kernel) on the same workload
+    # the randomised rotation (per-channel random signs) on the same workload, on the kernel the plan picks
     if rank == 0:
         extra["signed_rotation"] = time_signed(torch, F, w, xs, codes, scales, ts if is_nv else None, stream, peak,
                                                max(50, min(args.steps, 400)))
@@ -433,6 +433,9 @@ def run_kernel_only(args):
     w = workload_for(args)
     plan = F.fp4q_plan_create(w.fmt, w.group, w.block, w.rule)
     F.fp4q_plan_set_kernel(plan, KERNELS[args.kernel])
+    if args.signs:
+        mask = torch.from_numpy(W.random_sign_mask(w.K, 1234).view(np.int32)).cuda()
+        F.fp4q_plan_set_signs(plan, mask, w.K)
     x = torch.from_numpy(w.generate().view(np.int16)).view(torch.bfloat16).cuda()
     codes = torch.empty((w.M, w.K // 2), dtype=torch.uint8, device="cuda")
     scales = torch.empty((w.M, w.K // w.group), dtype=torch.uint8, device="cuda")
@@ -443,7 +446,8 @@ def run_kernel_only(args):
         F.fp4q_rotate_quantize(plan, x, w.M, w.K, codes, scales, ts if w.fmt == W.NVFP4 else None)
     torch.cuda.synchronize()
     assert F.fp4q_device_status() == F.FP4Q_OK
-    print(f"kernel-only: {w.name} M={w.M} K={w.K} launches={args.warmup + args.steps}", flush=True)
+    print(f"kernel-only: {w.name} M={w.M} K={w.K} signs={args.signs} launches={args.warmup + args.steps}",
+          flush=True)
 
 
 def tensor_peak_fp4():
@@ -506,13 +510,10 @@ def time_gemm(torch, F, fmt, M, N, K, stream, steps=50):
             "bound": "tensor"}
 
 
-def time_signed(torch, F, w, xs, codes, scales, ts, stream, peak, steps):
-    """fp4q_rotate_quantize with a plan carrying per-channel random signs (seeded mask): the
-    same bytes as the plain call, on the butterfly kernel."""
+def time_plan(torch, F, plan, w, xs, codes, scales, ts, stream, steps):
+    """Device microseconds per fp4q_rotate_quantize call of `plan` over the buffers in turn
+    (CUDA graph replays, CUDA events on the launching stream)."""
     M, K = w.M, w.K
-    plan = F.fp4q_plan_create(w.fmt, w.group, w.block, w.rule)
-    mask = torch.from_numpy(W.random_sign_mask(K, 1234).view(np.int32)).to(xs[0].device)
-    F.fp4q_plan_set_signs(plan, mask, K)
 
     def launch(i):
         F.fp4q_rotate_quantize(plan, xs[i], M, K, codes[i], scales[i], ts, stream=torch.cuda.current_stream())
@@ -527,11 +528,22 @@ def time_signed(torch, F, w, xs, codes, scales, ts, stream, peak, steps):
             g_rem.replay()
         a1.record(stream)
     torch.cuda.synchronize()
-    us = a0.elapsed_time(a1) * 1e3 / steps
+    return a0.elapsed_time(a1) * 1e3 / steps
+
+
+def time_signed(torch, F, w, xs, codes, scales, ts, stream, peak, steps, kernel="auto"):
+    """fp4q_rotate_quantize with a plan carrying per-channel random signs (seeded mask): the
+    same bytes as the plain call, on the kernel the plan picks."""
+    K = w.K
+    plan = F.fp4q_plan_create(w.fmt, w.group, w.block, w.rule)
+    F.fp4q_plan_set_kernel(plan, KERNELS[kernel])
+    mask = torch.from_numpy(W.random_sign_mask(K, 1234).view(np.int32)).to(xs[0].device)
+    F.fp4q_plan_set_signs(plan, mask, K)
+    us = time_plan(torch, F, plan, w, xs, codes, scales, ts, stream, steps)
     nbytes = w.bytes_per_call()
     gbs = nbytes / us / 1e3
     return {"us_per_call": round(us, 3), "GBps": round(gbs, 1), "pct_of_hbm_peak": round(100 * gbs / peak, 2),
-            "bytes_per_call": nbytes, "kernel": "butterfly"}
+            "bytes_per_call": nbytes, "kernel": kernel_name(w, kernel)}
 
 
 def run_gemm_only(args):
@@ -672,6 +684,8 @@ def time_other(torch, F, w, dev, stream, peak, kernel="auto"):
     gbs = bytes_call / us / 1e3
     out = {"GBps": round(gbs, 1), "pct_of_hbm_peak": round(100 * gbs / peak, 2), "us_per_call": round(us, 3),
            "bytes_per_call": bytes_call, "buffers": n_buf, "kernel": kernel_name(w, kernel)}
+    out["signed"] = time_signed(torch, F, w, xs, codes, scales, ts if w.fmt == W.NVFP4 else None, stream, peak,
+                                steps, kernel)
     if kernel == "auto":
         out["quant_error"] = time_quant_error(torch, F, w, plan, xs, ts if w.fmt == W.NVFP4 else None, stream, peak,
                                               steps // 2)
@@ -756,6 +770,8 @@ def main():
                     help="which rotate + quantize kernel the plan uses")
     ap.add_argument("--kernel-only", action="store_true",
                     help="only W + K plain launches of the workload (a case for profilers), no JSON line")
+    ap.add_argument("--signs", action="store_true",
+                    help="with --kernel-only: the plan carries per-channel random signs (seeded mask)")
     ap.add_argument("--gemm", type=int, nargs=3, metavar=("M", "N", "K"), default=None,
                     help="with --kernel-only: W + K launches of fp4q_gemm on operands the library quantized")
     ap.add_argument("--gemm-format", default="nvfp4", choices=["mxfp4", "nvfp4"])

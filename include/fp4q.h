@@ -142,10 +142,9 @@ fp4q_status fp4q_plan_destroy(fp4q_plan plan);
  * clears the signs.  K: the row length the signs are for; a multiple of max(g, b), at most
  * 2^34.  Afterwards every call on the plan must have this K (FP4Q_ERR_SHAPE otherwise), and
  * fp4q_rotate_quantize(_dump), fp4q_amax, fp4q_quant_error and fp4q_dequantize (with
- * unrotate) all use the signs.  A plan with signs runs the butterfly kernel: it returns
- * FP4Q_ERR_UNSUPPORTED when the plan is forced to FP4Q_KERNEL_TENSOR_CORE, and
- * fp4q_plan_set_kernel refuses TENSOR_CORE while signs are set.  signs must be 4-byte
- * aligned. */
+ * unrotate) all use the signs, on either rotate + quantize kernel (the tensor-core kernel
+ * flips the signs in shared memory before its product; the butterfly kernel as it loads).
+ * signs must be 4-byte aligned. */
 fp4q_status fp4q_plan_set_signs(fp4q_plan plan, const uint32_t* signs, int64_t K);
 
 /* Rotate and quantize X in one pass over HBM (steps 1-5 above).

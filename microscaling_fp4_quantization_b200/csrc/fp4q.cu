@@ -90,7 +90,7 @@ bool valid_plan(fp4q_plan p) { return p != nullptr && p->magic == kPlanMagic; }
 constexpr int64_t kMmaMinElems = int64_t(1) << 22;
 bool mma_capable(fp4q_plan p) { return p->format != FP4Q_MXFP4_MBS && p->block >= 16 && p->block >= p->group; }
 bool use_mma(fp4q_plan p, int64_t n_elems) {
-  if (!mma_capable(p) || p->signs) return false;   // channel signs: butterfly kernel only
+  if (!mma_capable(p)) return false;
   if (p->kernel == FP4Q_KERNEL_TENSOR_CORE) return true;
   return p->kernel == FP4Q_KERNEL_AUTO && n_elems >= kMmaMinElems;
 }
@@ -164,24 +164,24 @@ fp4q_status rotate_quantize_impl(fp4q_plan p, const void* x, int64_t M, int64_t 
           if constexpr (B >= 32) {
             switch (p->rule) {
               case FP4Q_SCALE_FLOOR_OCP:
-                return dump ? launch_mma<MmaConfig<kMX, B, kRuleFloor, true>>(a.x, n, a, s)
-                            : launch_mma<MmaConfig<kMX, B, kRuleFloor, false>>(a.x, n, a, s);
+                return dump ? launch_mma<MmaConfig<kMX, B, kRuleFloor, true>>(a.x, n, a, s, K)
+                            : launch_mma<MmaConfig<kMX, B, kRuleFloor, false>>(a.x, n, a, s, K);
               case FP4Q_SCALE_CEIL_NOCLIP:
-                return dump ? launch_mma<MmaConfig<kMX, B, kRuleCeil, true>>(a.x, n, a, s)
-                            : launch_mma<MmaConfig<kMX, B, kRuleCeil, false>>(a.x, n, a, s);
+                return dump ? launch_mma<MmaConfig<kMX, B, kRuleCeil, true>>(a.x, n, a, s, K)
+                            : launch_mma<MmaConfig<kMX, B, kRuleCeil, false>>(a.x, n, a, s, K);
               case FP4Q_SCALE_OAS:
-                return dump ? launch_mma<MmaConfig<kMX, B, kRuleOas, true>>(a.x, n, a, s)
-                            : launch_mma<MmaConfig<kMX, B, kRuleOas, false>>(a.x, n, a, s);
+                return dump ? launch_mma<MmaConfig<kMX, B, kRuleOas, true>>(a.x, n, a, s, K)
+                            : launch_mma<MmaConfig<kMX, B, kRuleOas, false>>(a.x, n, a, s, K);
               default: return FP4Q_ERR_UNSUPPORTED;
             }
           }
           return FP4Q_ERR_UNSUPPORTED;
         }
         if (p->rule == FP4Q_SCALE_NV_DYNAMIC)
-          return dump ? launch_mma<MmaConfig<kNV, B, kRuleNvDynamic, true>>(a.x, n, a, s)
-                      : launch_mma<MmaConfig<kNV, B, kRuleNvDynamic, false>>(a.x, n, a, s);
-        return dump ? launch_mma<MmaConfig<kNV, B, kRuleNvStatic, true>>(a.x, n, a, s)
-                    : launch_mma<MmaConfig<kNV, B, kRuleNvStatic, false>>(a.x, n, a, s);
+          return dump ? launch_mma<MmaConfig<kNV, B, kRuleNvDynamic, true>>(a.x, n, a, s, K)
+                      : launch_mma<MmaConfig<kNV, B, kRuleNvDynamic, false>>(a.x, n, a, s, K);
+        return dump ? launch_mma<MmaConfig<kNV, B, kRuleNvStatic, true>>(a.x, n, a, s, K)
+                    : launch_mma<MmaConfig<kNV, B, kRuleNvStatic, false>>(a.x, n, a, s, K);
       }
       return FP4Q_ERR_UNSUPPORTED;
     });
@@ -424,7 +424,7 @@ fp4q_status fp4q_plan_set_kernel(fp4q_plan plan, int kernel) {
   if (!valid_plan(plan)) return FP4Q_ERR_ARG;
   if (kernel != FP4Q_KERNEL_AUTO && kernel != FP4Q_KERNEL_BUTTERFLY && kernel != FP4Q_KERNEL_TENSOR_CORE)
     return FP4Q_ERR_ARG;
-  if (kernel == FP4Q_KERNEL_TENSOR_CORE && (!mma_capable(plan) || plan->signs)) return FP4Q_ERR_UNSUPPORTED;
+  if (kernel == FP4Q_KERNEL_TENSOR_CORE && !mma_capable(plan)) return FP4Q_ERR_UNSUPPORTED;
   plan->kernel = kernel;
   return FP4Q_OK;
 }
@@ -438,7 +438,6 @@ fp4q_status fp4q_plan_set_signs(fp4q_plan plan, const uint32_t* signs, int64_t K
   }
   if (K <= 0 || K % plan->unit != 0 || K > (int64_t(1) << 34)) return FP4Q_ERR_SHAPE;
   if (!aligned(signs, 4)) return FP4Q_ERR_ALIGN;
-  if (plan->kernel == FP4Q_KERNEL_TENSOR_CORE) return FP4Q_ERR_UNSUPPORTED;
   plan->signs = signs;
   plan->signs_K = K;
   return FP4Q_OK;

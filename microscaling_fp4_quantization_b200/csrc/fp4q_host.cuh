@@ -110,7 +110,7 @@ using AmaxCfg = RQConfig<kNV, B, kRuleNvStatic, false, MINU>;
 template <class Cfg>
 fp4q_status launch_rq(RQArgs a, int64_t n_elems, cudaStream_t stream, int64_t K = 0);
 template <class Cfg>
-fp4q_status launch_mma(const uint16_t* x, int64_t n_elems, const RQArgs& ra, cudaStream_t stream);
+fp4q_status launch_mma(const uint16_t* x, int64_t n_elems, const RQArgs& ra, cudaStream_t stream, int64_t K);
 template <class Cfg>
 fp4q_status launch_qe(fp4q_plan p, QEArgs a, int64_t n_elems, double* out, cudaStream_t stream);
 // CTAs of one full wave of a configuration's error kernel / amax kernel.

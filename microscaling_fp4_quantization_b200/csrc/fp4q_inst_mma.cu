@@ -7,8 +7,9 @@ namespace host {
 
 #define FP4Q_MMA_ONE(F, B, R)                                                                                  \
   template fp4q_status launch_mma<MmaConfig<F, B, R, false>>(const uint16_t*, int64_t, const RQArgs&,         \
-                                                             cudaStream_t);                                   \
-  template fp4q_status launch_mma<MmaConfig<F, B, R, true>>(const uint16_t*, int64_t, const RQArgs&, cudaStream_t);
+                                                             cudaStream_t, int64_t);                          \
+  template fp4q_status launch_mma<MmaConfig<F, B, R, true>>(const uint16_t*, int64_t, const RQArgs&, cudaStream_t, \
+                                                            int64_t);
 #define FP4Q_MMA_MX(B) FP4Q_MMA_ONE(kMX, B, kRuleFloor) FP4Q_MMA_ONE(kMX, B, kRuleCeil) FP4Q_MMA_ONE(kMX, B, kRuleOas)
 #define FP4Q_MMA_NV(B) FP4Q_MMA_ONE(kNV, B, kRuleNvStatic) FP4Q_MMA_ONE(kNV, B, kRuleNvDynamic)
 FP4Q_MMA_MX(32) FP4Q_MMA_MX(64) FP4Q_MMA_MX(128)

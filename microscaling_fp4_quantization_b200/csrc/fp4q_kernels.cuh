@@ -204,12 +204,16 @@ __device__ __forceinline__ UnitSigns<E> unit_signs(const uint32_t* mask, int cu)
 
 // XOR masks that negate the bf16 elements of one 16-byte chunk (8 elements, word i holding
 // elements 2i and 2i+1) whose sign bits are set in byte `mb`.
+// One multiply places two copies of the byte so that bits 2i and 2i+1 land on bits 15 and 31
+// (the two shifted copies occupy disjoint bit ranges, so the sum carries nowhere), and one AND
+// keeps those two bits.
 __device__ __forceinline__ uint4 chunk_sign_xor(uint32_t mb) {
+  const uint32_t b = mb & 0xFFu;
   uint4 r;
-  r.x = ((mb & 0x01u) << 15) | ((mb & 0x02u) << 30);
-  r.y = ((mb & 0x04u) << 13) | ((mb & 0x08u) << 28);
-  r.z = ((mb & 0x10u) << 11) | ((mb & 0x20u) << 26);
-  r.w = ((mb & 0x40u) << 9) | ((mb & 0x80u) << 24);
+  r.x = (b * 0x40008000u) & 0x80008000u;   // b << 15 + b << 30
+  r.y = (b * 0x10002000u) & 0x80008000u;   // b << 13 + b << 28
+  r.z = (b * 0x04000800u) & 0x80008000u;   // b << 11 + b << 26
+  r.w = (b * 0x01000200u) & 0x80008000u;   // b << 9 + b << 24
   return r;
 }
 

@@ -29,7 +29,7 @@ fp4q_status launch_rq(RQArgs a, int64_t n_elems, cudaStream_t stream, int64_t K)
 
 // Tensor-core kernel: a TMA tensor map over the rows of one Hadamard block each.
 template <class Cfg>
-fp4q_status launch_mma(const uint16_t* x, int64_t n_elems, const RQArgs& ra, cudaStream_t stream) {
+fp4q_status launch_mma(const uint16_t* x, int64_t n_elems, const RQArgs& ra, cudaStream_t stream, int64_t K) {
   EncodeTiledFn enc;
   fp4q_status st = encode_fn(&enc);
   if (st != FP4Q_OK) return st;
@@ -43,6 +43,11 @@ fp4q_status launch_mma(const uint16_t* x, int64_t n_elems, const RQArgs& ra, cud
   a.partials = ra.partials;
   a.n_partials = ra.n_partials;
   a.y_dump = ra.y_dump;
+  a.sign_bytes = reinterpret_cast<const uint8_t*>(ra.signs.mask);
+  a.sign_upr = ra.signs.mask ? K / Cfg::kBlock : 1;
+  // the mask's words (ceil(K / 32) of them), staged in shared memory when they fit
+  const int64_t mask_bytes = ra.signs.mask ? (K + 127) / 128 * 16 : 0;
+  a.sign_smem = mask_bytes <= Cfg::kMaskSmemMax ? static_cast<int>(mask_bytes) : 0;
   CUtensorMap map;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(Cfg::kBlock), static_cast<cuuint64_t>(a.n_rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(Cfg::kBlock) * 2};
@@ -60,7 +65,7 @@ fp4q_status launch_mma(const uint16_t* x, int64_t n_elems, const RQArgs& ra, cud
   }
   auto kernel = rotate_quantize_mma_kernel<Cfg>;
   KernelInfo ki;
-  st = kernel_info(kernel, Cfg::kSmemBytes, Cfg::kThreads, &ki);
+  st = kernel_info(kernel, Cfg::kSmemBytes + Cfg::kMaskSmemMax, Cfg::kThreads, &ki);
   if (st != FP4Q_OK) return st;
   // CTAs per SM from measurement (the kernel's CTAs are independent, so a CTA that does not
   // fit next to the others simply starts later); tensor memory holds 512 columns per SM
@@ -68,8 +73,8 @@ fp4q_status launch_mma(const uint16_t* x, int64_t n_elems, const RQArgs& ra, cud
   if (per_sm > 512 / Cfg::kTmemCols) per_sm = 512 / Cfg::kTmemCols;
   int64_t ctas = static_cast<int64_t>(ki.sm_count) * per_sm;
   if (ctas > a.n_super) ctas = a.n_super;
-  cudaError_t e = launch_pdl(kernel, dim3(static_cast<unsigned>(ctas)), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream,
-                             map, a);
+  cudaError_t e = launch_pdl(kernel, dim3(static_cast<unsigned>(ctas)), dim3(Cfg::kThreads),
+                             Cfg::kSmemBytes + a.sign_smem, stream, map, a);
   if (e != cudaSuccess) return cuda_fail(e, "rotate_quantize (tensor core) launch");
   return FP4Q_OK;
 }

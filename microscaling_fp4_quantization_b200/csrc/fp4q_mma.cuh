@@ -66,7 +66,10 @@ struct MmaConfig {
   static constexpr int kEpiWarps = 4 * kSlices;
   static constexpr int kEpiCols = kSuperCols / kSlices;   // columns per epilogue warp
   static constexpr int kCtasPerSm = (FMT == kNV && B <= 64) ? 1 : 2;
-  static constexpr int kThreads = 32 * (2 + kEpiWarps);
+  // plans with per-channel signs: these warps flip the signs of each landed stage's elements
+  // (four where one CTA has the SM, two beside a second CTA)
+  static constexpr int kSignWarps = kCtasPerSm == 1 ? 4 : 2;
+  static constexpr int kThreads = 32 * (2 + kEpiWarps + kSignWarps);
   static constexpr int kTmemCols = 2 * kSuperCols;   // two accumulator buffers
   static constexpr float kC = inv_sqrt_block(B);
   // shared memory: [align pad][stages][H][barriers]
@@ -80,7 +83,13 @@ struct MmaConfig {
   static constexpr int kFlipShift = kRB == 32 ? 2 : 1;
   static constexpr int kFlipMask = kRB == 32 ? 1 : 3;
   static constexpr int kBarOffset = kStages * kStageBytes + kHBytes + kTableBytes;
-  static constexpr int kSmemBytes = 1024 + kBarOffset + 128;
+  static constexpr int kMaskOffset = (kBarOffset + 8 * (3 * kStages + 4) + 15) / 16 * 16;
+  static constexpr int kSmemBytes = 1024 + kMaskOffset;   // without the staged sign mask
+  // Plans with channel signs stage the mask (K / 8 bytes) after the barriers when it fits
+  // beside kCtasPerSm CTAs (228 KB of shared memory per SM, 1 KB of it reserved per CTA).
+  static constexpr int kMaskRoom = (233472 / kCtasPerSm - 1024 - kSmemBytes) / 16 * 16;
+  static constexpr int kMaskSmemMax = kMaskRoom < 16384 ? kMaskRoom : 16384;
+  static_assert(kMaskSmemMax >= 1024, "room for the sign mask of K <= 8192");
   static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(B >> 3) << 17) |
                                      (static_cast<uint32_t>(128 >> 4) << 24);
 };
@@ -95,6 +104,9 @@ struct MmaArgs {
   const float* partials;
   int n_partials;
   float* y_dump;
+  const uint8_t* sign_bytes;   // per-channel signs (bit k of byte k / 8 negates channel k), or null
+  int64_t sign_upr;            // Hadamard blocks per matrix row, K / b
+  int sign_smem;               // bytes of the mask staged in shared memory (0: read from global)
 };
 
 // Offset of byte `off` inside a swizzled K-major tile (rows of 32 / 64 / 128 bytes): the
@@ -199,7 +211,7 @@ __device__ __forceinline__ uint32_t quantize_group(const float (&s)[G], uint32_t
 }
 
 template <class Cfg>
-__global__ void __launch_bounds__(Cfg::kThreads, 2)
+__global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
     rotate_quantize_mma_kernel(const __grid_constant__ CUtensorMap xmap, MmaArgs a) {
   constexpr int B = Cfg::kBlock, G = Cfg::kGroup, S = Cfg::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -215,6 +227,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 2)
   auto empty_bar = [&](int s) { return bars + 8u * (S + s); };
   auto tfull_bar = [&](int d) { return bars + 8u * (2 * S + d); };
   auto tempty_bar = [&](int d) { return bars + 8u * (2 * S + 2 + d); };
+  auto signed_bar = [&](int s) { return bars + 8u * (2 * S + 4 + s); };
 
   // H_b, K-major, swizzled like the activation tiles: row n holds H[n][0..b) (H is symmetric)
   uint8_t* hs = smem + S * Cfg::kStageBytes;
@@ -234,6 +247,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 2)
       mbar_init(tfull_bar(d), 1);
       mbar_init(tempty_bar(d), Cfg::kEpiWarps);
     }
+    for (int s = 0; s < S; ++s) mbar_init(signed_bar(s), Cfg::kSignWarps);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -319,7 +333,8 @@ __global__ void __launch_bounds__(Cfg::kThreads, 2)
         const uint32_t ph = static_cast<uint32_t>((i / S) & 1);
         const int d = static_cast<int>(i & 1);
         const uint32_t dph = static_cast<uint32_t>((i >> 1) & 1);
-        if (!mbar_wait_bounded(full_bar(s), ph)) break;
+        // with signs, the sign warps' "signed" barrier follows the stage's "full" one
+        if (!mbar_wait_bounded(a.sign_bytes ? signed_bar(s) : full_bar(s), ph)) break;
         if (!mbar_wait_bounded(tempty_bar(d), dph ^ 1u)) break;
         tc_fence_after();
         const uint32_t a0 = stage0 + s * Cfg::kStageBytes;
@@ -342,6 +357,82 @@ __global__ void __launch_bounds__(Cfg::kThreads, 2)
       if (i > 0) {
         const int64_t j = i - 1;
         mbar_wait_bounded(tfull_bar(static_cast<int>(j & 1)), static_cast<uint32_t>((j >> 1) & 1));
+      }
+    }
+  } else if (warp >= 2 + Cfg::kEpiWarps) {
+    // ---------------- sign warps: x_k -> s_k x_k in the landed stage (plans with channel signs)
+    // The warps walk the stage's 16-byte chunks in physical order (lane-consecutive addresses:
+    // no bank conflicts), kBatch chunks a lane at a time.  A stage region (the whole stage in
+    // the bulk layout, one K-half of swizzled 128-byte rows otherwise) holds kCpr chunks per
+    // row; a lane's chunks sit kRowStep rows apart and, as kRowStep is a multiple of the
+    // 8-row swizzle period, all carry the same logical chunk q of their rows.
+    if (a.sign_bytes != nullptr) {
+      constexpr int kCpr = Cfg::kBulk ? B / 8 : 8;                 // chunks per row of a region
+      constexpr int kRegions = Cfg::kBulk ? 1 : Cfg::kHalves;
+      constexpr int kRegionBytes = Cfg::kStageBytes / kRegions;
+      constexpr int kLaneStride = 32 * Cfg::kSignWarps;            // chunks between a lane's chunks
+      constexpr int kRowStep = kLaneStride / kCpr;
+      constexpr int kPerLane = kRegionBytes / 16 / kLaneStride;    // chunks per lane per region
+      constexpr int kBatch = Cfg::kCtasPerSm == 1 ? 4 : 8;
+      static_assert(kLaneStride % kCpr == 0 && (Cfg::kBulk || kRowStep % 8 == 0), "lane chunk walk");
+      static_assert(kPerLane % kBatch == 0, "whole batches per region");
+      const int sw = warp - (2 + Cfg::kEpiWarps);
+      const int c0 = 32 * sw + lane;                               // lane's first chunk of a region
+      const uint32_t row0 = static_cast<uint32_t>(c0 / kCpr);
+      const uint32_t pq = static_cast<uint32_t>(c0 % kCpr);
+      const uint32_t upr = static_cast<uint32_t>(a.sign_upr);
+      const uint32_t row_step = static_cast<uint32_t>(kRowStep) % upr;
+      pdl_wait();   // the mask belongs to the caller and may come from an earlier kernel
+      const uint8_t* mask = a.sign_bytes;
+      if (a.sign_smem > 0) {
+        // the mask's words, once per CTA, into shared memory (a few hundred bytes to 16 KB)
+        uint32_t* ms = reinterpret_cast<uint32_t*>(smem + Cfg::kMaskOffset);
+        const uint32_t* mg = reinterpret_cast<const uint32_t*>(a.sign_bytes);
+        const int words = static_cast<int>((static_cast<int64_t>(upr) * B + 31) / 32);   // the caller's ceil(K / 32)
+        for (int w = 32 * sw + lane; w < words; w += 32 * Cfg::kSignWarps) ms[w] = __ldg(mg + w);
+        asm volatile("bar.sync 2, %0;" ::"r"(32 * Cfg::kSignWarps) : "memory");
+        mask = smem + Cfg::kMaskOffset;
+      }
+      int64_t i = 0;
+      for (int64_t t = blockIdx.x; t < n_super; t += gridDim.x, ++i) {
+        const int s = static_cast<int>(i % S);
+        const uint32_t ph = static_cast<uint32_t>((i / S) & 1);
+        const bool mine = mbar_wait_bounded(full_bar(s), ph);
+        if (!__all_sync(0xFFFFFFFFu, mine)) break;
+        // Hadamard block (within its matrix row) of the lane's first row
+        const uint32_t kb_first = static_cast<uint32_t>(
+            (static_cast<uint64_t>((t * Cfg::kRowsPerTile) % upr) + row0) % upr);
+#pragma unroll 1
+        for (int h = 0; h < kRegions; ++h) {
+          // logical chunk of the lane's rows: the bulk layout is unswizzled; a swizzled row's
+          // physical chunk is its logical one XOR (row & 7)
+          const uint32_t q = Cfg::kBulk ? pq : 8u * h + (pq ^ (row0 & 7u));
+          const uint8_t* mq = mask + q;
+          uint32_t kb = kb_first;
+          uint32_t addr = stage0 + s * Cfg::kStageBytes + h * kRegionBytes + 16u * c0;
+#pragma unroll 1
+          for (int j = 0; j < kPerLane; j += kBatch) {
+            uint4 w[kBatch];
+            uint32_t m[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+              m[u] = mq[kb * (B / 8)];
+              kb += row_step;
+              if (kb >= upr) kb -= upr;
+              w[u] = lds128(addr + 16u * kLaneStride * u);
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+              const uint4 f = chunk_sign_xor(m[u]);
+              sts128_u4(addr + 16u * kLaneStride * u,
+                        make_uint4(w[u].x ^ f.x, w[u].y ^ f.y, w[u].z ^ f.z, w[u].w ^ f.w));
+            }
+            addr += 16u * kLaneStride * kBatch;
+          }
+        }
+        fence_proxy_async_smem();   // the tensor core reads the stage through the async proxy
+        __syncwarp();
+        if (lane == 0) mbar_arrive(signed_bar(s));
       }
     }
   } else {

@@ -78,10 +78,9 @@ def test_sign_validation_without_gpu(F):
     assert ss(p.handle, A, 256) == F.FP4Q_OK
     rq = lambda *a: F.raw_call("fp4q_rotate_quantize", *a)
     assert rq(p.handle, A, 4, 128, A, A, None, None) == F.FP4Q_ERR_SHAPE      # K differs from the signs'
-    assert F.raw_call("fp4q_plan_set_kernel", p.handle, F.FP4Q_KERNEL_TENSOR_CORE) == F.FP4Q_ERR_UNSUPPORTED
+    F.fp4q_plan_set_kernel(p, F.FP4Q_KERNEL_TENSOR_CORE)       # signs work on both kernels
     assert ss(p.handle, None, 0) == F.FP4Q_OK                   # cleared
-    F.fp4q_plan_set_kernel(p, F.FP4Q_KERNEL_TENSOR_CORE)
-    assert ss(p.handle, A, 256) == F.FP4Q_ERR_UNSUPPORTED       # forced tensor-core kernel
+    assert ss(p.handle, A, 256) == F.FP4Q_OK
     F.fp4q_plan_destroy(p)
 
 

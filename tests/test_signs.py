@@ -34,13 +34,21 @@ def signed_plan(F, combo, K, seed):
     return plan, o.sign_vector(mask, K)
 
 
-@pytest.mark.parametrize("combo", COMBOS, ids=[combo_id(c) for c in COMBOS])
-def test_signed_rotate_quantize_matches_oracle(F, combo):
+SIGN_CASES = ([(c, 1) for c in COMBOS] + [(c, 2) for c in COMBOS if c[2] >= 16 and c[2] >= c[1]])
+
+
+@pytest.mark.parametrize("combo,kernel", SIGN_CASES,
+                         ids=[combo_id(c) + ("-tc" if k == 2 else "-bf") for c, k in SIGN_CASES])
+def test_signed_rotate_quantize_matches_oracle(F, combo, kernel):
+    """kernel 1: the butterfly kernel (signs applied as it loads); 2: the tensor-core kernel
+    (signs flipped in the landed shared-memory stage before the product)."""
     import gpu_util as gu
     fmt, g, b, rule = combo
     unit = max(g, b)
-    for i, (M, K) in enumerate([(3, 2 * unit), (37, 6 * unit), (130, 4096 // unit * unit), (200, 1536)]):
+    for i, (M, K) in enumerate([(3, 2 * unit), (37, 6 * unit), (130, 4096 // unit * unit), (200, 1536),
+                                (1100, 4096)]):
         plan, s = signed_plan(F, combo, K, seed=500 + i)
+        F.fp4q_plan_set_kernel(plan, kernel)
         x = make_input(M, K, seed=9000 + 100 * b + 10 * rule + i, adversarial=M >= 8)
         s_g = o.nv_tensor_scale(o.rotated_amax(x, b, signs=s)) if rule == o.SCALE_NV_STATIC else None
         res = o.rotate_quantize(x, fmt, g, b, rule, tensor_scale=s_g, signs=s)
