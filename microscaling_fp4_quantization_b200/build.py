@@ -20,7 +20,7 @@ LIB = os.path.join(LIB_DIR, "libfp4q.so")
 
 # The C ABI and its dispatch, then one unit per kernel family (compiled in parallel).
 SOURCES = ["fp4q.cu", "fp4q_inst_rq_mx.cu", "fp4q_inst_rq_nv.cu", "fp4q_inst_mbs.cu", "fp4q_inst_qe.cu",
-           "fp4q_inst_mma.cu", "fp4q_inst_dequant.cu", "fp4q_inst_gemm.cu"]
+           "fp4q_inst_mma.cu", "fp4q_inst_mma_qe.cu", "fp4q_inst_dequant.cu", "fp4q_inst_gemm.cu"]
 DEPS = SOURCES + ["fp4q_kernels.cuh", "fp4q_device.cuh", "fp4q_mma.cuh", "fp4q_host.cuh", "fp4q_launch.cuh", "fp4q_gemm.cuh"]
 OBJ_DIR = os.path.join(PKG, "lib", "obj")
 

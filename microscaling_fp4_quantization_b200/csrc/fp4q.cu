@@ -269,6 +269,12 @@ fp4q_status qe_grid(int format, int block, int rule, int* n) {
     });
     if (st != FP4Q_OK) return st;
   }
+  // the tensor-core error pass: at most two persistent CTAs per SM
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  if (2 * sms > *n) *n = 2 * sms;
   return FP4Q_OK;
 }
 
@@ -526,6 +532,33 @@ fp4q_status fp4q_quant_error(fp4q_plan plan, const void* x_bf16, int64_t M, int6
     st = launch_amax(plan, a.x, n, s);
     if (st != FP4Q_OK) return st;
   }
+  if (use_mma(plan, n)) {
+    // the kernel fp4q_rotate_quantize picks for this plan and size, so the same codes
+    a.signs = ChannelSigns{plan->signs, 1, 0};
+    const int slots = plan->n_err_partials;
+    return with_block(plan->block, [&]<int B>() -> fp4q_status {
+      if constexpr (B >= 16) {
+        if (plan->format == FP4Q_MXFP4) {
+          if constexpr (B >= 32) {
+            switch (plan->rule) {
+              case FP4Q_SCALE_FLOOR_OCP:
+                return launch_mma_qe<MmaConfig<kMX, B, kRuleFloor, false, true>>(a, n, s, K, slots);
+              case FP4Q_SCALE_CEIL_NOCLIP:
+                return launch_mma_qe<MmaConfig<kMX, B, kRuleCeil, false, true>>(a, n, s, K, slots);
+              case FP4Q_SCALE_OAS:
+                return launch_mma_qe<MmaConfig<kMX, B, kRuleOas, false, true>>(a, n, s, K, slots);
+              default: return FP4Q_ERR_UNSUPPORTED;
+            }
+          }
+          return FP4Q_ERR_UNSUPPORTED;
+        }
+        if (plan->rule == FP4Q_SCALE_NV_DYNAMIC)
+          return launch_mma_qe<MmaConfig<kNV, B, kRuleNvDynamic, false, true>>(a, n, s, K, slots);
+        return launch_mma_qe<MmaConfig<kNV, B, kRuleNvStatic, false, true>>(a, n, s, K, slots);
+      }
+      return FP4Q_ERR_UNSUPPORTED;
+    });
+  }
   return with_rq_cfg(plan->format, plan->block, plan->rule, n % 32 == 0,
                      [&]<class Cfg>() -> fp4q_status { return launch_qe<Cfg>(plan, a, n, out, s); });
 }
@@ -611,7 +644,7 @@ fp4q_status fp4q_device_status(void) {
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
   unsigned int v = 0;
   for (fp4q_status (*reader)(unsigned int*) : {status_rq_mx, status_rq_nv, status_mbs, status_qe, status_mma,
-                                               status_dequant, status_gemm}) {
+                                               status_mma_qe, status_dequant, status_gemm}) {
     fp4q_status st = reader(&v);
     if (st != FP4Q_OK) return st;
   }

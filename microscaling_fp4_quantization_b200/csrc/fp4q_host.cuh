@@ -112,6 +112,8 @@ fp4q_status launch_rq(RQArgs a, int64_t n_elems, cudaStream_t stream, int64_t K 
 template <class Cfg>
 fp4q_status launch_mma(const uint16_t* x, int64_t n_elems, const RQArgs& ra, cudaStream_t stream, int64_t K);
 template <class Cfg>
+fp4q_status launch_mma_qe(const QEArgs& qa, int64_t n_elems, cudaStream_t stream, int64_t K, int max_ctas);
+template <class Cfg>
 fp4q_status launch_qe(fp4q_plan p, QEArgs a, int64_t n_elems, double* out, cudaStream_t stream);
 // CTAs of one full wave of a configuration's error kernel / amax kernel.
 template <class Cfg>
@@ -143,6 +145,7 @@ fp4q_status status_rq_nv(unsigned int* v);
 fp4q_status status_mbs(unsigned int* v);
 fp4q_status status_qe(unsigned int* v);
 fp4q_status status_mma(unsigned int* v);
+fp4q_status status_mma_qe(unsigned int* v);
 fp4q_status status_dequant(unsigned int* v);
 fp4q_status status_gemm(unsigned int* v);
 

@@ -27,26 +27,22 @@ fp4q_status launch_rq(RQArgs a, int64_t n_elems, cudaStream_t stream, int64_t K)
   return FP4Q_OK;
 }
 
-// Tensor-core kernel: a TMA tensor map over the rows of one Hadamard block each.
+// Tensor-core kernel: a TMA tensor map over the rows of one Hadamard block each.  `a` holds
+// the outputs (codes and scales, or the error pass's sums); the rest is filled in here.
+// max_ctas caps the persistent grid (the error pass's partial-sum slots), 0 for none.
 template <class Cfg>
-fp4q_status launch_mma(const uint16_t* x, int64_t n_elems, const RQArgs& ra, cudaStream_t stream, int64_t K) {
+fp4q_status launch_mma_common(MmaArgs a, const uint16_t* x, int64_t n_elems, const ChannelSigns& signs,
+                              cudaStream_t stream, int64_t K, int64_t max_ctas) {
   EncodeTiledFn enc;
   fp4q_status st = encode_fn(&enc);
   if (st != FP4Q_OK) return st;
-  MmaArgs a;
   a.x = x;
   a.n_rows = n_elems / Cfg::kBlock;
   a.n_super = (a.n_rows + Cfg::kRowsPerTile - 1) / Cfg::kRowsPerTile;
-  a.codes = ra.codes;
-  a.scales = ra.scales;
-  a.tensor_scale = ra.tensor_scale;
-  a.partials = ra.partials;
-  a.n_partials = ra.n_partials;
-  a.y_dump = ra.y_dump;
-  a.sign_bytes = reinterpret_cast<const uint8_t*>(ra.signs.mask);
-  a.sign_upr = ra.signs.mask ? K / Cfg::kBlock : 1;
+  a.sign_bytes = reinterpret_cast<const uint8_t*>(signs.mask);
+  a.sign_upr = signs.mask ? K / Cfg::kBlock : 1;
   // the mask's words (ceil(K / 32) of them), staged in shared memory when they fit
-  const int64_t mask_bytes = ra.signs.mask ? (K + 127) / 128 * 16 : 0;
+  const int64_t mask_bytes = signs.mask ? (K + 127) / 128 * 16 : 0;
   a.sign_smem = mask_bytes <= Cfg::kMaskSmemMax ? static_cast<int>(mask_bytes) : 0;
   CUtensorMap map;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(Cfg::kBlock), static_cast<cuuint64_t>(a.n_rows)};
@@ -73,10 +69,38 @@ fp4q_status launch_mma(const uint16_t* x, int64_t n_elems, const RQArgs& ra, cud
   if (per_sm > 512 / Cfg::kTmemCols) per_sm = 512 / Cfg::kTmemCols;
   int64_t ctas = static_cast<int64_t>(ki.sm_count) * per_sm;
   if (ctas > a.n_super) ctas = a.n_super;
+  if (max_ctas > 0 && ctas > max_ctas) ctas = max_ctas;
   cudaError_t e = launch_pdl(kernel, dim3(static_cast<unsigned>(ctas)), dim3(Cfg::kThreads),
                              Cfg::kSmemBytes + a.sign_smem, stream, map, a);
-  if (e != cudaSuccess) return cuda_fail(e, "rotate_quantize (tensor core) launch");
+  if (e != cudaSuccess) return cuda_fail(e, Cfg::kQE ? "quant_error (tensor core) launch"
+                                                     : "rotate_quantize (tensor core) launch");
   return FP4Q_OK;
+}
+
+template <class Cfg>
+fp4q_status launch_mma(const uint16_t* x, int64_t n_elems, const RQArgs& ra, cudaStream_t stream, int64_t K) {
+  MmaArgs a = {};
+  a.codes = ra.codes;
+  a.scales = ra.scales;
+  a.tensor_scale = ra.tensor_scale;
+  a.partials = ra.partials;
+  a.n_partials = ra.n_partials;
+  a.y_dump = ra.y_dump;
+  return launch_mma_common<Cfg>(a, x, n_elems, ra.signs, stream, K, 0);
+}
+
+// The error pass on the tensor-core kernel: one partial pair per CTA in qa.out_partials,
+// whose slots (max_ctas of them) cap the grid.
+template <class Cfg>
+fp4q_status launch_mma_qe(const QEArgs& qa, int64_t n_elems, cudaStream_t stream, int64_t K, int max_ctas) {
+  MmaArgs a = {};
+  a.tensor_scale = qa.tensor_scale;
+  a.partials = qa.partials;
+  a.n_partials = qa.n_partials;
+  a.qe_partials = qa.out_partials;
+  a.qe_ticket = qa.ticket;
+  a.qe_out = qa.out;
+  return launch_mma_common<Cfg>(a, qa.x, n_elems, qa.signs, stream, K, max_ctas);
 }
 
 template <class Cfg>

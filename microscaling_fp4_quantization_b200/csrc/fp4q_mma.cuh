@@ -35,12 +35,16 @@
 
 namespace fp4q {
 
-template <int FMT, int B, int RULE, bool DUMP>
+// QE: the error pass.  The epilogue makes the same scale decisions and codes as the quantizer
+// and accumulates the signal and error energies instead of storing anything.
+template <int FMT, int B, int RULE, bool DUMP, bool QE = false>
 struct MmaConfig {
   static constexpr int kFmt = FMT;
   static constexpr int kBlock = B;
   static constexpr int kRule = RULE;
   static constexpr bool kDump = DUMP;
+  static constexpr bool kQE = QE;
+  static_assert(!(QE && DUMP), "the error pass stores nothing");
   static constexpr int kGroup = FMT == kMX ? 32 : 16;
   static_assert(B >= 16 && B >= kGroup && B <= 128, "one block holds whole groups");
   static constexpr int kKB = B > 64 ? 64 : B;        // K elements per swizzled row (one TMA box row)
@@ -107,6 +111,11 @@ struct MmaArgs {
   const uint8_t* sign_bytes;   // per-channel signs (bit k of byte k / 8 negates channel k), or null
   int64_t sign_upr;            // Hadamard blocks per matrix row, K / b
   int sign_smem;               // bytes of the mask staged in shared memory (0: read from global)
+  // error pass only: [gridDim.x][2] per-CTA signal, error energies; the ticket counter (0
+  // between calls, reset by the last CTA); out [3] = signal, error, QSNR dB
+  double* qe_partials;
+  unsigned int* qe_ticket;
+  double* qe_out;
 };
 
 // Offset of byte `off` inside a swizzled K-major tile (rows of 32 / 64 / 128 bytes): the
@@ -210,6 +219,52 @@ __device__ __forceinline__ uint32_t quantize_group(const float (&s)[G], uint32_t
   return byte;
 }
 
+// Signal and error energy of one group of G rotated sums s, added to fp64 running sums: the
+// same scale byte and quotients as quantize_group (so the same codes), then sum v^2 and
+// sum (v - q)^2 in units of X^2.  A zero NV block scale zeroes every code: the error is then
+// the whole signal, y = s / sqrt(b) in fp64.
+template <class Cfg, int G>
+__device__ __forceinline__ void group_energy_mma(const float (&s)[G], const float* nv_tab, float s_g, float nv_den,
+                                                 float nv_rden, double& sig, double& err) {
+  constexpr float c = Cfg::kC;
+  f32x2 p[G / 2];
+#pragma unroll
+  for (int k = 0; k < G / 2; ++k) p[k] = f2_pack(s[2 * k], s[2 * k + 1]);
+  const float A = scale_by_inv_sqrt<Cfg::kBlock>(pairs_amax<G / 2>(p));
+  float mult;
+  double X2;
+  if constexpr (Cfg::kFmt == kMX) {
+    const int byte = mx_scale_byte<Cfg::kRule>(A);
+    mult = c * mx_inv_scale(byte);
+    X2 = mx_scale_sq(byte);
+  } else {
+    const uint32_t byte = e4m3_encode(div_rn_markstein(A, nv_den, nv_rden));
+    mult = nv_tab[byte];
+    if (byte == 0u || mult == 0.0f) {
+      constexpr double c64 = inv_sqrt_block_f64(Cfg::kBlock);
+      double e2 = 0.0;
+#pragma unroll
+      for (int k = 0; k < G; ++k) {
+        const double y = static_cast<double>(s[k]) * c64;
+        e2 = fma(y, y, e2);
+      }
+      sig += e2;
+      err += e2;
+      return;
+    }
+    const double S = static_cast<double>(e4m3_decode(byte) * s_g);
+    X2 = S * S;
+  }
+  const f32x2 mm = f2_pack(mult, mult);
+  f32x2 v[G / 2];
+#pragma unroll
+  for (int k = 0; k < G / 2; ++k) v[k] = f2_mul(p[k], mm);
+  float gs, ge;
+  group_energies<G / 2>(v, gs, ge);
+  sig = fma(static_cast<double>(gs), X2, sig);
+  err = fma(static_cast<double>(ge), X2, err);
+}
+
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
     rotate_quantize_mma_kernel(const __grid_constant__ CUtensorMap xmap, MmaArgs a) {
@@ -217,6 +272,8 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ uint32_t s_tmem_base;
   __shared__ float s_tensor_scale;
+  __shared__ double s_qe[Cfg::kQE ? Cfg::kEpiWarps : 1][2];   // error pass: energies per epilogue warp
+  __shared__ bool s_qe_last;
   pdl_launch_dependents();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
@@ -478,6 +535,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
     const float nv_rden = __frcp_rn(nv_den);
     constexpr int EC = Cfg::kEpiCols;                 // 16, 32 or 64 columns
     constexpr int NGW = EC / G;                        // groups per warp slice
+    double qe_sig = 0.0, qe_err = 0.0;                 // error pass: this lane's running energies
     int64_t i = 0;
     for (int64_t t = blockIdx.x; t < n_super; t += gridDim.x, ++i) {
       const int d = static_cast<int>(i & 1);
@@ -503,6 +561,25 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
       // The slice holds whole blocks (b < EC), exactly one block (b == EC) or half of one.
       constexpr int BW = B < EC ? B : EC;              // block elements in one slice piece
       constexpr int PIECES = EC / BW;                  // block pieces in the slice
+      if constexpr (Cfg::kQE) {
+        // energies only; a column's sign flip from the bulk layout changes neither v^2 nor
+        // (v - q)^2 (E2M1 rounds the magnitude)
+#pragma unroll
+        for (int pc = 0; pc < PIECES; ++pc) {
+          const int j = (col0 + pc * BW) / B;
+          const int64_t row = t * Cfg::kRowsPerTile + j * 128 + lane_row;
+          if (row < a.n_rows) {
+#pragma unroll
+            for (int q = 0; q < BW / G; ++q) {
+              float gv[G];
+#pragma unroll
+              for (int e = 0; e < G; ++e) gv[e] = v[pc * BW + q * G + e];
+              group_energy_mma<Cfg, G>(gv, nv_tab, s_g, nv_den, nv_rden, qe_sig, qe_err);
+            }
+          }
+        }
+        continue;
+      }
 #pragma unroll
       for (int pc = 0; pc < PIECES; ++pc) {
         const int col = col0 + pc * BW;                // column within the super-tile
@@ -564,6 +641,39 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
         }
       }
       (void)NGW;
+    }
+    if constexpr (Cfg::kQE) {
+      // the CTA's energies (epilogue warps in order), then the last CTA to finish sums the
+      // per-CTA pairs in CTA order: a fixed order for a fixed grid, so the result is deterministic
+      constexpr int kEpiThreads = 32 * Cfg::kEpiWarps;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        qe_sig += __shfl_xor_sync(0xFFFFFFFFu, qe_sig, o);
+        qe_err += __shfl_xor_sync(0xFFFFFFFFu, qe_err, o);
+      }
+      if (lane == 0) {
+        s_qe[warp - 2][0] = qe_sig;
+        s_qe[warp - 2][1] = qe_err;
+      }
+      asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
+      if (warp == 2 && lane == 0) {
+        double ts = 0.0, te = 0.0;
+#pragma unroll
+        for (int w = 0; w < Cfg::kEpiWarps; ++w) {
+          ts += s_qe[w][0];
+          te += s_qe[w][1];
+        }
+        a.qe_partials[2 * blockIdx.x] = ts;
+        a.qe_partials[2 * blockIdx.x + 1] = te;
+        __threadfence();
+        s_qe_last = atomicAdd(a.qe_ticket, 1u) == gridDim.x - 1;
+      }
+      asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
+      if (s_qe_last && warp == 2) {
+        __threadfence();
+        qe_final_sum(a.qe_partials, static_cast<int>(gridDim.x), a.qe_out);
+        if (lane == 0) *a.qe_ticket = 0u;
+      }
     }
   }
   tc_fence_before();

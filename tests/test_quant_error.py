@@ -52,6 +52,23 @@ def run_qe(F, plan, x_bits=None, tensor_scale=None, x_dev=None):
     return s, e, q, np.float32(ts.item())
 
 
+BUTTERFLY, TENSOR_CORE = 1, 2
+
+
+def tc_capable(fmt, g, b):
+    """The tensor-core kernel serves MXFP4 / NVFP4 plans whose blocks hold whole groups."""
+    return fmt in (o.MXFP4, o.NVFP4) and b >= 16 and b >= g
+
+
+def kernel_cases(combos):
+    return [(c, BUTTERFLY) for c in combos] + [(c, TENSOR_CORE) for c in combos if tc_capable(c[0], c[1], c[2])]
+
+
+def kernel_id(case):
+    c, k = case
+    return combo_id(c) + ("-tc" if k == TENSOR_CORE else "-bf")
+
+
 def static_scale(x, fmt, b, rule):
     if fmt == o.NVFP4 and rule == o.SCALE_NV_STATIC:
         return o.nv_tensor_scale(o.rotated_amax(x, b))
@@ -68,10 +85,15 @@ def assert_energies(ours, ref, label):
         assert abs(q - ref["qsnr_db"]) <= QSNR_ATOL_DB, (label, q, ref["qsnr_db"])
 
 
-@pytest.mark.parametrize("combo", COMBOS, ids=[combo_id(c) for c in COMBOS])
-def test_quant_error_matches_oracle(F, combo):
+QE_CASES = kernel_cases(COMBOS)
+
+
+@pytest.mark.parametrize("case", QE_CASES, ids=[kernel_id(c) for c in QE_CASES])
+def test_quant_error_matches_oracle(F, case):
+    combo, kernel = case
     fmt, g, b, rule = combo
     plan = F.fp4q_plan_create(fmt, g, b, rule)
+    F.fp4q_plan_set_kernel(plan, kernel)
     unit = max(g, b)
     for i, (M, K) in enumerate([(1, unit), (37, 6 * unit), (130, 4096 // unit * unit), (1000, 1536)]):
         x = make_input(M, K, seed=7000 + 100 * b + 10 * rule + i, adversarial=M >= 8)
@@ -83,16 +105,21 @@ def test_quant_error_matches_oracle(F, combo):
             assert abs(float(ours[3]) - float(ref["tensor_scale"])) <= 2.5e-7 * float(ref["tensor_scale"])
 
 
-@pytest.mark.parametrize("combo", [(o.MXFP4, 32, 32, o.SCALE_FLOOR_OCP), (o.MXFP4, 32, 128, o.SCALE_OAS),
-                                   (o.NVFP4, 16, 16, o.SCALE_NV_STATIC), (o.NVFP4, 16, 2, o.SCALE_NV_DYNAMIC)],
-                         ids=combo_id)
-def test_quant_error_measures_the_codes_rotate_quantize_stores(F, combo):
-    """The error pass decides exactly as the butterfly quantize kernel: its error energy is the
-    one of that kernel's stored codes, dequantized on the GPU, against its dumped fp32 y."""
+STORE_CASES = kernel_cases([(o.MXFP4, 32, 32, o.SCALE_FLOOR_OCP), (o.MXFP4, 32, 128, o.SCALE_OAS),
+                            (o.NVFP4, 16, 16, o.SCALE_NV_STATIC), (o.NVFP4, 16, 2, o.SCALE_NV_DYNAMIC),
+                            (o.NVFP4, 16, 64, o.SCALE_NV_DYNAMIC)])
+
+
+@pytest.mark.parametrize("case", STORE_CASES, ids=[kernel_id(c) for c in STORE_CASES])
+def test_quant_error_measures_the_codes_rotate_quantize_stores(F, case):
+    """The error pass decides exactly as the quantize kernel of the same plan: its error
+    energy is the one of that kernel's stored codes, dequantized on the GPU, against its
+    dumped fp32 y (butterfly and tensor-core kernels alike)."""
     import gpu_util as gu
+    combo, kernel = case
     fmt, g, b, rule = combo
     plan = F.fp4q_plan_create(fmt, g, b, rule)
-    F.fp4q_plan_set_kernel(plan, F.FP4Q_KERNEL_BUTTERFLY)
+    F.fp4q_plan_set_kernel(plan, kernel)
     x = make_input(512, 2048, seed=11 + b, adversarial=False)
     s_g = static_scale(x, fmt, b, rule)
     rq = gu.run_rotate_quantize(F, plan, x, tensor_scale=s_g, dump=True)
@@ -105,12 +132,14 @@ def test_quant_error_measures_the_codes_rotate_quantize_stores(F, combo):
     assert e == pytest.approx(noise, rel=ERR_RTOL)
 
 
-def test_quant_error_is_deterministic_and_additive_over_rows(F):
+@pytest.mark.parametrize("kernel", [BUTTERFLY, TENSOR_CORE], ids=["bf", "tc"])
+def test_quant_error_is_deterministic_and_additive_over_rows(F, kernel):
     """Two calls give the same bits; the energies of row blocks add up to the whole
     tensor's (a grid of many waves against one of a few CTAs)."""
     w = W.NV_4K
     x = w.generate()
     plan = F.fp4q_plan_create(w.fmt, w.group, w.block, o.SCALE_NV_STATIC)
+    F.fp4q_plan_set_kernel(plan, kernel)
     import gpu_util as gu
     xd = gu.to_device_bf16(x)
     ts = o.nv_tensor_scale(o.rotated_amax(x, w.block))
@@ -126,9 +155,16 @@ def test_quant_error_is_deterministic_and_additive_over_rows(F):
         assert_energies(parts[r // 512], ref, f"rows {r}..")
 
 
-@pytest.mark.parametrize("name", [W.SMALL_MX.name, W.MX_8K_FLOOR.name, W.MX_8K_CEIL.name, W.PREFILL_NV.name,
-                                  W.PREFILL_MX.name] + [w.name for w in W.DECODE])
-def test_quant_error_on_workloads(F, name):
+WORKLOAD_NAMES = [W.SMALL_MX.name, W.MX_8K_FLOOR.name, W.MX_8K_CEIL.name, W.PREFILL_NV.name,
+                  W.PREFILL_MX.name] + [w.name for w in W.DECODE]
+WORKLOAD_CASES = [(n, BUTTERFLY) for n in WORKLOAD_NAMES] + [
+    (n, TENSOR_CORE) for n in WORKLOAD_NAMES
+    if tc_capable(W.BY_NAME[n].fmt, W.BY_NAME[n].group, W.BY_NAME[n].block)]
+
+
+@pytest.mark.parametrize("name,kernel", WORKLOAD_CASES,
+                         ids=[n + ("-tc" if k == TENSOR_CORE else "-bf") for n, k in WORKLOAD_CASES])
+def test_quant_error_on_workloads(F, name, kernel):
     """Full-size workloads: the GPU over the whole tensor equals the sum of the GPU over row
     blocks, and the oracle agrees with the GPU on sampled blocks."""
     import gpu_util as gu
@@ -136,6 +172,7 @@ def test_quant_error_on_workloads(F, name):
     x = w.generate()
     rule = w.rule
     plan = F.fp4q_plan_create(w.fmt, w.group, w.block, rule)
+    F.fp4q_plan_set_kernel(plan, kernel)
     xd = gu.to_device_bf16(x)
     ts = None
     if w.fmt == o.NVFP4:
