@@ -442,11 +442,15 @@ def run_kernel_only(args):
     ts = torch.ones(1, dtype=torch.float32, device="cuda")
     if w.fmt == W.NVFP4:
         F.fp4q_amax(plan, x, w.M, w.K, ts)
+    out = torch.zeros(3, dtype=torch.float64, device="cuda")
     for _ in range(args.warmup + args.steps):
-        F.fp4q_rotate_quantize(plan, x, w.M, w.K, codes, scales, ts if w.fmt == W.NVFP4 else None)
+        if args.op == "quant_error":
+            F.fp4q_quant_error(plan, x, w.M, w.K, ts if w.fmt == W.NVFP4 else None, out)
+        else:
+            F.fp4q_rotate_quantize(plan, x, w.M, w.K, codes, scales, ts if w.fmt == W.NVFP4 else None)
     torch.cuda.synchronize()
     assert F.fp4q_device_status() == F.FP4Q_OK
-    print(f"kernel-only: {w.name} M={w.M} K={w.K} signs={args.signs} launches={args.warmup + args.steps}",
+    print(f"kernel-only: {args.op} {w.name} M={w.M} K={w.K} signs={args.signs} launches={args.warmup + args.steps}",
           flush=True)
 
 
@@ -770,6 +774,8 @@ def main():
                     help="which rotate + quantize kernel the plan uses")
     ap.add_argument("--kernel-only", action="store_true",
                     help="only W + K plain launches of the workload (a case for profilers), no JSON line")
+    ap.add_argument("--op", default="rotate_quantize", choices=["rotate_quantize", "quant_error"],
+                    help="with --kernel-only: the call to launch")
     ap.add_argument("--signs", action="store_true",
                     help="with --kernel-only: the plan carries per-channel random signs (seeded mask)")
     ap.add_argument("--gemm", type=int, nargs=3, metavar=("M", "N", "K"), default=None,

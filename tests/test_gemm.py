@@ -74,8 +74,10 @@ def check(D, qa, qb, fmt, K, rows=None, label=""):
 
 @pytest.mark.parametrize("fmt,g,b,rule", FORMATS, ids=["mxfp4", "nvfp4"])
 @pytest.mark.parametrize("M,N,K", [(128, 256, 256), (1, 256, 512), (200, 512, 1024), (1000, 768, 2048),
-                                   (300, 32, 256)])
+                                   (300, 32, 256), (257, 512, 512), (384, 288, 768), (129, 1024, 256)])
 def test_gemm_matches_oracle(F, fmt, g, b, rule, M, N, K):
+    """Ragged shapes: a last M tile of one row (257, 129) or of a few rows (200, 300, 1000), and
+    a last N tile of 32 columns (N = 288)."""
     rng = np.random.default_rng(M + N + K)
     X = W.f32_to_bf16_bits((rng.standard_normal((M, K)) * np.exp(rng.normal(0, 1, (M, 1)))).astype(np.float32))
     Wt = W.synthetic_weights(N, K, seed=N + K)
