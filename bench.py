@@ -358,6 +358,8 @@ def run_gpu(args):
                 others[ow.name + f" [{alt} kernel]"] = time_other(torch, F, ow, dev, stream, peak, kernel=alt)
         for ow in (W.MX_8K_FLOOR, W.PREFILL_MX):
             others[ow.name + " [MBS-Static]"] = time_mbs(torch, F, ow, dev, stream, peak)
+            for k in ("butterfly", "tensor_core"):
+                others[ow.name + f" [MBS-Static, {k} kernel]"] = time_mbs(torch, F, ow, dev, stream, peak, kernel=k)
         gemms = {}
         for fmt, name in ((W.MXFP4, "mxfp4"), (W.NVFP4, "nvfp4")):
             for (M, N, K) in ((8192, 8192, 8192), (4096, 14336, 4096), (4096, 4096, 14336)):
@@ -609,12 +611,13 @@ def time_quant_error(torch, F, w, plan, xs, ts, stream, peak, steps):
             "mse": err / (M * K)}
 
 
-def time_mbs(torch, F, w, dev, stream, peak):
+def time_mbs(torch, F, w, dev, stream, peak, kernel="auto"):
     """MBS-Static (MXFP4 with 128-element macro scales) on an MX workload's input: GB/s on its
     algorithmic bytes (bf16 in; codes, E8M0 group scales and macro bytes out), and the QSNR
     against plain MXFP4 with the same rule."""
     M, K = w.M, w.K
     plan = F.fp4q_plan_create(F.FP4Q_MXFP4_MBS, 32, w.block, w.rule)
+    F.fp4q_plan_set_kernel(plan, KERNELS[kernel])
     x_np = w.generate()
     nbytes = M * K * 2 + M * K // 2 + M * K // 32 + M * K // 128
     n_buf = max(1, math.ceil(3 * L2_BYTES / nbytes)) if nbytes < 2 * L2_BYTES else 1
@@ -643,10 +646,13 @@ def time_mbs(torch, F, w, dev, stream, peak):
     gbs = nbytes / us / 1e3
     qe_mbs = time_quant_error(torch, F, w, plan, xs, None, stream, peak, 20)
     plain = F.fp4q_plan_create(w.fmt, w.group, w.block, w.rule)
+    F.fp4q_plan_set_kernel(plain, KERNELS[kernel])
     qe_plain = time_quant_error(torch, F, w, plain, xs, None, stream, peak, 20)
+    used = kernel_name(w, kernel)   # MBS plans choose as MXFP4 plans do (group 32)
     out = {"GBps": round(gbs, 1), "pct_of_hbm_peak": round(100 * gbs / peak, 2), "us_per_call": round(us, 3),
-           "bytes_per_call": nbytes, "buffers": n_buf, "kernel": "butterfly",
-           "qsnr_db": qe_mbs["qsnr_db"], "qsnr_db_plain_mxfp4": qe_plain["qsnr_db"]}
+           "bytes_per_call": nbytes, "buffers": n_buf, "kernel": used,
+           "qsnr_db": qe_mbs["qsnr_db"], "qsnr_db_plain_mxfp4": qe_plain["qsnr_db"],
+           "quant_error": {k: qe_mbs[k] for k in ("us_per_call", "GBps", "pct_of_hbm_peak")}}
     del xs, codes, scales, macro
     torch.cuda.empty_cache()
     return out

@@ -89,8 +89,8 @@ typedef enum {
  * 256 wraps to 0, the same quantization with every group exponent one higher).  The rotated
  * values are divided by s_M (fp32, correctly rounded) and then quantized as MXFP4 with the
  * plan's MX rule; a value decodes as E2M1 * 2^(byte - 127) * s_M.  Group 32, K a multiple of
- * 128.  Served by fp4q_rotate_quantize_mbs, fp4q_dequantize_mbs and fp4q_quant_error (the
- * butterfly kernel). */
+ * 128.  Served by fp4q_rotate_quantize_mbs, fp4q_dequantize_mbs and fp4q_quant_error, on
+ * either rotate + quantize kernel (the tensor-core kernel for b >= 32). */
 typedef enum { FP4Q_MXFP4 = 0, FP4Q_NVFP4 = 1, FP4Q_MXFP4_MBS = 2 } fp4q_format;
 
 typedef enum {

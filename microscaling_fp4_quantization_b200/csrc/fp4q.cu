@@ -88,7 +88,7 @@ bool valid_plan(fp4q_plan p) { return p != nullptr && p->magic == kPlanMagic; }
 // kMmaMinElems elements: below that its fixed start-up (TMEM allocation, H_b, filling a
 // three-stage pipeline) costs more than the butterfly kernel's extra instructions.
 constexpr int64_t kMmaMinElems = int64_t(1) << 22;
-bool mma_capable(fp4q_plan p) { return p->format != FP4Q_MXFP4_MBS && p->block >= 16 && p->block >= p->group; }
+bool mma_capable(fp4q_plan p) { return p->block >= 16 && p->block >= p->group; }
 bool use_mma(fp4q_plan p, int64_t n_elems) {
   if (!mma_capable(p)) return false;
   if (p->kernel == FP4Q_KERNEL_TENSOR_CORE) return true;
@@ -160,6 +160,18 @@ fp4q_status rotate_quantize_impl(fp4q_plan p, const void* x, int64_t M, int64_t 
   if (use_mma(p, n)) {
     return with_block(p->block, [&]<int B>() -> fp4q_status {
       if constexpr (B >= 16) {
+        if (p->format == FP4Q_MXFP4_MBS) {
+          // the MBS entry has no dump form (it was refused above when macro is null)
+          if constexpr (B >= 32) {
+            switch (p->rule) {
+              case FP4Q_SCALE_FLOOR_OCP: return launch_mma<MmaConfig<kMBS, B, kRuleFloor, false>>(a.x, n, a, s, K);
+              case FP4Q_SCALE_CEIL_NOCLIP: return launch_mma<MmaConfig<kMBS, B, kRuleCeil, false>>(a.x, n, a, s, K);
+              case FP4Q_SCALE_OAS: return launch_mma<MmaConfig<kMBS, B, kRuleOas, false>>(a.x, n, a, s, K);
+              default: return FP4Q_ERR_UNSUPPORTED;
+            }
+          }
+          return FP4Q_ERR_UNSUPPORTED;
+        }
         if (p->format == FP4Q_MXFP4) {
           if constexpr (B >= 32) {
             switch (p->rule) {
@@ -538,6 +550,20 @@ fp4q_status fp4q_quant_error(fp4q_plan plan, const void* x_bf16, int64_t M, int6
     const int slots = plan->n_err_partials;
     return with_block(plan->block, [&]<int B>() -> fp4q_status {
       if constexpr (B >= 16) {
+        if (plan->format == FP4Q_MXFP4_MBS) {
+          if constexpr (B >= 32) {
+            switch (plan->rule) {
+              case FP4Q_SCALE_FLOOR_OCP:
+                return launch_mma_qe<MmaConfig<kMBS, B, kRuleFloor, false, true>>(a, n, s, K, slots);
+              case FP4Q_SCALE_CEIL_NOCLIP:
+                return launch_mma_qe<MmaConfig<kMBS, B, kRuleCeil, false, true>>(a, n, s, K, slots);
+              case FP4Q_SCALE_OAS:
+                return launch_mma_qe<MmaConfig<kMBS, B, kRuleOas, false, true>>(a, n, s, K, slots);
+              default: return FP4Q_ERR_UNSUPPORTED;
+            }
+          }
+          return FP4Q_ERR_UNSUPPORTED;
+        }
         if (plan->format == FP4Q_MXFP4) {
           if constexpr (B >= 32) {
             switch (plan->rule) {

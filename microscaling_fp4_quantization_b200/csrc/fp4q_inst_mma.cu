@@ -12,7 +12,13 @@ namespace host {
                                                             int64_t);
 #define FP4Q_MMA_MX(B) FP4Q_MMA_ONE(kMX, B, kRuleFloor) FP4Q_MMA_ONE(kMX, B, kRuleCeil) FP4Q_MMA_ONE(kMX, B, kRuleOas)
 #define FP4Q_MMA_NV(B) FP4Q_MMA_ONE(kNV, B, kRuleNvStatic) FP4Q_MMA_ONE(kNV, B, kRuleNvDynamic)
+// MBS-Static: no dump form
+#define FP4Q_MMA_MBS_ONE(B, R)                                                                              \
+  template fp4q_status launch_mma<MmaConfig<kMBS, B, R, false>>(const uint16_t*, int64_t, const RQArgs&, \
+                                                                cudaStream_t, int64_t);
+#define FP4Q_MMA_MBS(B) FP4Q_MMA_MBS_ONE(B, kRuleFloor) FP4Q_MMA_MBS_ONE(B, kRuleCeil) FP4Q_MMA_MBS_ONE(B, kRuleOas)
 FP4Q_MMA_MX(32) FP4Q_MMA_MX(64) FP4Q_MMA_MX(128)
+FP4Q_MMA_MBS(32) FP4Q_MMA_MBS(64) FP4Q_MMA_MBS(128)
 FP4Q_MMA_NV(16) FP4Q_MMA_NV(32) FP4Q_MMA_NV(64) FP4Q_MMA_NV(128)
 
 }  // namespace host

@@ -10,7 +10,10 @@ namespace host {
   template fp4q_status launch_mma_qe<MmaConfig<F, B, R, false, true>>(const QEArgs&, int64_t, cudaStream_t, int64_t, int);
 #define FP4Q_MMA_QE_MX(B) FP4Q_MMA_QE_ONE(kMX, B, kRuleFloor) FP4Q_MMA_QE_ONE(kMX, B, kRuleCeil) FP4Q_MMA_QE_ONE(kMX, B, kRuleOas)
 #define FP4Q_MMA_QE_NV(B) FP4Q_MMA_QE_ONE(kNV, B, kRuleNvStatic) FP4Q_MMA_QE_ONE(kNV, B, kRuleNvDynamic)
+#define FP4Q_MMA_QE_MBS(B) \
+  FP4Q_MMA_QE_ONE(kMBS, B, kRuleFloor) FP4Q_MMA_QE_ONE(kMBS, B, kRuleCeil) FP4Q_MMA_QE_ONE(kMBS, B, kRuleOas)
 FP4Q_MMA_QE_MX(32) FP4Q_MMA_QE_MX(64) FP4Q_MMA_QE_MX(128)
+FP4Q_MMA_QE_MBS(32) FP4Q_MMA_QE_MBS(64) FP4Q_MMA_QE_MBS(128)
 FP4Q_MMA_QE_NV(16) FP4Q_MMA_QE_NV(32) FP4Q_MMA_QE_NV(64) FP4Q_MMA_QE_NV(128)
 
 }  // namespace host

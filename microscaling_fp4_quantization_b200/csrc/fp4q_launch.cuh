@@ -86,6 +86,7 @@ fp4q_status launch_mma(const uint16_t* x, int64_t n_elems, const RQArgs& ra, cud
   a.partials = ra.partials;
   a.n_partials = ra.n_partials;
   a.y_dump = ra.y_dump;
+  a.macro = ra.macro;
   return launch_mma_common<Cfg>(a, x, n_elems, ra.signs, stream, K, 0);
 }
 

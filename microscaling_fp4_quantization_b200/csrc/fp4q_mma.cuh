@@ -45,8 +45,11 @@ struct MmaConfig {
   static constexpr bool kDump = DUMP;
   static constexpr bool kQE = QE;
   static_assert(!(QE && DUMP), "the error pass stores nothing");
-  static constexpr int kGroup = FMT == kMX ? 32 : 16;
+  static constexpr int kGroup = FMT == kNV ? 16 : 32;   // MXFP4 and MBS-Static: 32
   static_assert(B >= 16 && B >= kGroup && B <= 128, "one block holds whole groups");
+  // MBS-Static: a 128-element macro block is 128 / b consecutive rows (TMEM lanes of one warp)
+  // for b <= 64, and both column halves of one row for b = 128
+  static constexpr int kMacroLanes = FMT == kMBS ? (B < 128 ? 128 / B : 1) : 1;
   static constexpr int kKB = B > 64 ? 64 : B;        // K elements per swizzled row (one TMA box row)
   static constexpr int kRB = 2 * kKB;                // bytes per swizzled row
   static constexpr int kHalves = B / kKB;            // K-halves (2 for b = 128)
@@ -111,6 +114,7 @@ struct MmaArgs {
   const uint8_t* sign_bytes;   // per-channel signs (bit k of byte k / 8 negates channel k), or null
   int64_t sign_upr;            // Hadamard blocks per matrix row, K / b
   int sign_smem;               // bytes of the mask staged in shared memory (0: read from global)
+  uint8_t* macro;              // MBS-Static: the macro-scale bytes [R * b / 128]
   // error pass only: [gridDim.x][2] per-CTA signal, error energies; the ticket counter (0
   // between calls, reset by the last CTA); out [3] = signal, error, QSNR dB
   double* qe_partials;
@@ -219,6 +223,46 @@ __device__ __forceinline__ uint32_t quantize_group(const float (&s)[G], uint32_t
   return byte;
 }
 
+// MBS-Static on G rotated sums s of one group: y' = RN(y / s_M) (dv: the divisor for s_M),
+// then the MXFP4 scale byte of y' under the plan's rule and the E2M1 code words of
+// y' / 2^(byte - 127), as the butterfly kernel's quantizer takes them.
+template <class Cfg, int G>
+__device__ __forceinline__ uint32_t quantize_group_mbs(const float (&s)[G], NvDivisor dv, uint32_t (&words)[G / 8]) {
+  f32x2 p[G / 2];
+#pragma unroll
+  for (int k = 0; k < G / 2; ++k) p[k] = f2_pack(s[2 * k], s[2 * k + 1]);
+  f32x2 yq[G / 2];
+  nv_quotients<Cfg::kBlock, G / 2>(p, dv, yq);
+  const int byte = mx_scale_byte<Cfg::kRule>(pairs_amax<G / 2>(yq));
+#pragma unroll
+  for (int j = 0; j < G / 8; ++j) {
+    f32x2 v[4];
+    mx_quotients<4>(&yq[4 * j], byte, 1.0f, v);
+    words[j] = e2m1x8_pairs(v);
+  }
+  return static_cast<uint32_t>(byte);
+}
+
+// The macro-scale byte of MBS-Static for this lane's macro block, from the largest raw sum
+// magnitude of the lane's piece (am) and, for b = 128, of the other half of its row
+// (am_other); the lanes of one macro block (b <= 64) combine theirs by shuffles, so every
+// lane of the warp must call it.
+template <class Cfg>
+__device__ __forceinline__ uint32_t mbs_lane_macro_byte(float am, float am_other) {
+  if constexpr (Cfg::kMacroLanes >= 2) am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
+  if constexpr (Cfg::kMacroLanes >= 4) am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 2));
+  if constexpr (Cfg::kBlock == 128) am = fmaxf(am, am_other);
+  return mbs_macro_byte(scale_by_inv_sqrt<Cfg::kBlock>(am));
+}
+
+template <int N>
+__device__ __forceinline__ float abs_max(const float* v) {
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < N; ++i) m = fmaxf(m, fabsf(v[i]));
+  return m;
+}
+
 // Signal and error energy of one group of G rotated sums s, added to fp64 running sums: the
 // same scale byte and quotients as quantize_group (so the same codes), then sum v^2 and
 // sum (v - q)^2 in units of X^2.  A zero NV block scale zeroes every code: the error is then
@@ -261,6 +305,51 @@ __device__ __forceinline__ void group_energy_mma(const float (&s)[G], const floa
   for (int k = 0; k < G / 2; ++k) v[k] = f2_mul(p[k], mm);
   float gs, ge;
   group_energies<G / 2>(v, gs, ge);
+  sig = fma(static_cast<double>(gs), X2, sig);
+  err = fma(static_cast<double>(ge), X2, err);
+}
+
+// One lane's piece of a block: BW codes (BW / 8 code words) from element `off` of block `row`,
+// and their BW / g scale bytes.
+template <class Cfg, int BW>
+__device__ __forceinline__ void store_piece(const MmaArgs& a, int64_t row, int off, const uint32_t (&words)[BW / 8],
+                                            const uint32_t (&sbytes)[BW / Cfg::kGroup]) {
+  constexpr int B = Cfg::kBlock, G = Cfg::kGroup, NG = BW / G;
+  uint8_t* cp = a.codes + row * (B / 2) + off / 2;
+  if constexpr (BW == 16) {
+    stg64(cp, words[0], words[1]);
+  } else {
+#pragma unroll
+    for (int k = 0; k < BW / 32; ++k)
+      stg128(cp + 16 * k, words[4 * k], words[4 * k + 1], words[4 * k + 2], words[4 * k + 3]);
+  }
+  uint8_t* sp = a.scales + row * (B / G) + off / G;
+  if constexpr (NG == 1) {
+    *sp = static_cast<uint8_t>(sbytes[0]);
+  } else if constexpr (NG == 2) {
+    *reinterpret_cast<uint16_t*>(sp) = static_cast<uint16_t>(sbytes[0] | (sbytes[1] << 8));
+  } else {
+    static_assert(NG == 4, "a slice piece holds 1, 2 or 4 groups");
+    *reinterpret_cast<uint32_t*>(sp) = sbytes[0] | (sbytes[1] << 8) | (sbytes[2] << 16) | (sbytes[3] << 24);
+  }
+}
+
+// group_energy_mma for MBS-Static: the quotients and codes of quantize_group_mbs, energies in
+// units of X^2 = 2^(2 (byte - 127)) s_M^2 (sM2).
+template <class Cfg, int G>
+__device__ __forceinline__ void group_energy_mma_mbs(const float (&s)[G], NvDivisor dv, double sM2, double& sig,
+                                                     double& err) {
+  f32x2 p[G / 2];
+#pragma unroll
+  for (int k = 0; k < G / 2; ++k) p[k] = f2_pack(s[2 * k], s[2 * k + 1]);
+  f32x2 yq[G / 2];
+  nv_quotients<Cfg::kBlock, G / 2>(p, dv, yq);
+  const int byte = mx_scale_byte<Cfg::kRule>(pairs_amax<G / 2>(yq));
+  f32x2 v[G / 2];
+  mx_quotients<G / 2>(yq, byte, 1.0f, v);
+  float gs, ge;
+  group_energies<G / 2>(v, gs, ge);
+  const double X2 = mx_scale_sq(byte) * sM2;
   sig = fma(static_cast<double>(gs), X2, sig);
   err = fma(static_cast<double>(ge), X2, err);
 }
@@ -545,6 +634,93 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
       tc_fence_after();
       const int col0 = half * EC;                      // first column of this warp's slice
       const uint32_t tq = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + d * Cfg::kSuperCols + col0;
+      if constexpr (Cfg::kFmt == kMBS) {
+        // MBS-Static.  Pass 1 keeps only the largest magnitude of each piece (and, for b = 128,
+        // of the row's other column half); once the macro byte is known, each group is read
+        // again from tensor memory and quantized (or measured).  Few values are live at a time,
+        // and the accumulator buffer is released after the second pass.
+        constexpr int BWm = B < EC ? B : EC;
+        constexpr int PCm = EC / BWm;
+        // 32 columns (two loads) per wait
+        float am[PCm];
+#pragma unroll
+        for (int pc = 0; pc < PCm; ++pc) {
+          am[pc] = 0.0f;
+#pragma unroll
+          for (int c32 = 0; c32 < BWm / 32; ++c32) {
+            float w0[16], w1[16];
+            tmem_ld16(tq + pc * BWm + 32 * c32, w0);
+            tmem_ld16(tq + pc * BWm + 32 * c32 + 16, w1);
+            tmem_wait_ld();
+            am[pc] = fmaxf(am[pc], fmaxf(abs_max<16>(w0), abs_max<16>(w1)));
+          }
+        }
+        float am_other = 0.0f;
+        if constexpr (B == 128) {
+          const uint32_t tp = tq - col0 + (EC - col0);
+#pragma unroll
+          for (int c32 = 0; c32 < EC / 32; ++c32) {
+            float w0[16], w1[16];
+            tmem_ld16(tp + 32 * c32, w0);
+            tmem_ld16(tp + 32 * c32 + 16, w1);
+            tmem_wait_ld();
+            am_other = fmaxf(am_other, fmaxf(abs_max<16>(w0), abs_max<16>(w1)));
+          }
+        }
+#pragma unroll
+        for (int pc = 0; pc < PCm; ++pc) {
+          const int col = col0 + pc * BWm;
+          const int j = col / B, off = col % B;
+          const int64_t row = t * Cfg::kRowsPerTile + j * 128 + lane_row;
+          const uint32_t m8 = mbs_lane_macro_byte<Cfg>(am[pc], am_other);
+          const float sM = mbs_macro_scale(m8);
+          const NvDivisor mdv = nv_divisor<B>(sM);
+          if constexpr (!Cfg::kQE) {
+            // the macro byte from the macro block's first lane (b = 128: the first half's warp)
+            const bool first = Cfg::kMacroLanes > 1 ? (lane % Cfg::kMacroLanes) == 0 : half == 0;
+            if (first && row < a.n_rows) a.macro[row * B / 128] = static_cast<uint8_t>(m8);
+          }
+#pragma unroll
+          for (int q = 0; q < BWm / G; ++q) {
+            float gv[G];
+            {
+              static_assert(G == 32, "an MBS group is two 16-column loads");
+              float w0[16], w1[16];
+              tmem_ld16(tq + pc * BWm + q * G, w0);
+              tmem_ld16(tq + pc * BWm + q * G + 16, w1);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                gv[e] = w0[e];
+                gv[16 + e] = w1[e];
+              }
+            }
+            if constexpr (Cfg::kQE) {
+              if (row < a.n_rows)
+                group_energy_mma_mbs<Cfg, G>(gv, mdv, static_cast<double>(sM) * static_cast<double>(sM), qe_sig,
+                                             qe_err);
+            } else {
+              // each group's codes and scale go out as soon as they are made
+              uint32_t gw[G / 8];
+              uint32_t sb[1];
+              sb[0] = quantize_group_mbs<Cfg, G>(gv, mdv, gw);
+#pragma unroll
+              for (int e = 0; e < G / 8; ++e) {
+                const int chunk = (off + q * G) / 8 + e;
+                if constexpr (Cfg::kBulk) {
+                  if (chunk & 1) gw[e] ^= flip_basis0;
+                  if (chunk & 2) gw[e] ^= flip_basis1;
+                }
+              }
+              if (row < a.n_rows) store_piece<Cfg, G>(a, row, off + q * G, gw, sb);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty_bar(d));
+        continue;
+      }
       float v[EC];
 #pragma unroll
       for (int c16 = 0; c16 < EC / 16; ++c16) {
@@ -619,26 +795,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
             }
           }
         }
-        if (row < a.n_rows) {
-          uint8_t* cp = a.codes + row * (B / 2) + off / 2;
-          if constexpr (BW == 16) {
-            stg64(cp, words[0], words[1]);
-          } else {
-#pragma unroll
-            for (int k = 0; k < BW / 32; ++k)
-              stg128(cp + 16 * k, words[4 * k], words[4 * k + 1], words[4 * k + 2], words[4 * k + 3]);
-          }
-          uint8_t* sp = a.scales + row * (B / G) + off / G;
-          constexpr int NG = BW / G;
-          if constexpr (NG == 1) {
-            *sp = static_cast<uint8_t>(sbytes[0]);
-          } else if constexpr (NG == 2) {
-            *reinterpret_cast<uint16_t*>(sp) = static_cast<uint16_t>(sbytes[0] | (sbytes[1] << 8));
-          } else {
-            static_assert(NG == 4, "a slice piece holds 1, 2 or 4 groups");
-            *reinterpret_cast<uint32_t*>(sp) = sbytes[0] | (sbytes[1] << 8) | (sbytes[2] << 16) | (sbytes[3] << 24);
-          }
-        }
+        if (row < a.n_rows) store_piece<Cfg, BW>(a, row, off, words, sbytes);
       }
       (void)NGW;
     }

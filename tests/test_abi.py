@@ -98,6 +98,11 @@ def test_mbs_validation_without_gpu(F):
     assert dq(p.handle, A, A, None, 4, 256, 0, A, None) == F.FP4Q_ERR_UNSUPPORTED
     dm = lambda *a: F.raw_call("fp4q_dequantize_mbs", *a)
     assert dm(p.handle, A, A, None, 4, 256, 0, A, None) == F.FP4Q_ERR_ARG
+    # the tensor-core kernel takes MBS plans whose blocks hold whole groups (b >= 32)
+    assert F.raw_call("fp4q_plan_set_kernel", p.handle, F.FP4Q_KERNEL_TENSOR_CORE) == F.FP4Q_OK
+    p16 = F.fp4q_plan_create(F.FP4Q_MXFP4_MBS, 32, 16, F.FP4Q_SCALE_OAS)
+    assert F.raw_call("fp4q_plan_set_kernel", p16.handle, F.FP4Q_KERNEL_TENSOR_CORE) == F.FP4Q_ERR_UNSUPPORTED
+    F.fp4q_plan_destroy(p16)
     mx = F.fp4q_plan_create(F.FP4Q_MXFP4, 32, 32, F.FP4Q_SCALE_OAS)
     assert mq(mx.handle, A, 4, 256, A, A, A, None) == F.FP4Q_ERR_UNSUPPORTED
     assert dm(mx.handle, A, A, A, 4, 256, 0, A, None) == F.FP4Q_ERR_UNSUPPORTED

@@ -36,11 +36,16 @@ def check_macro(res, out, label):
     assert not bad.any(), (label, int(bad.sum()))
 
 
-@pytest.mark.parametrize("b", BLOCKS)
+# (block, kernel): the butterfly for every block, the tensor-core kernel where blocks hold whole groups
+CASES = [(b, 1) for b in BLOCKS] + [(b, 2) for b in BLOCKS if b >= 32]
+
+
+@pytest.mark.parametrize("b,kernel", CASES, ids=[f"b{b}-{'tc' if k == 2 else 'bf'}" for b, k in CASES])
 @pytest.mark.parametrize("rule", RULES, ids=[W.RULE_NAMES[r] for r in RULES])
-def test_mbs_matches_oracle(F, b, rule):
+def test_mbs_matches_oracle(F, b, kernel, rule):
     import gpu_util as gu
     plan = F.fp4q_plan_create(o.MXFP4_MBS, 32, b, rule)
+    F.fp4q_plan_set_kernel(plan, kernel)
     for i, (M, K) in enumerate([(1, 128), (3, 256), (37, 768), (130, 4096), (300, 1536)]):
         x = make_input(M, K, seed=3000 + 10 * b + rule + 100 * i, adversarial=M >= 8)
         res = o.rotate_quantize_mbs(x, 32, b, rule)
@@ -55,13 +60,15 @@ def test_mbs_matches_oracle(F, b, rule):
             assert_parity(res_r, out["codes"][real], out["scales"][real], label + " rows 8+")
 
 
-@pytest.mark.parametrize("b", [1, 32, 128])
-def test_mbs_dequantize_and_error(F, b):
+@pytest.mark.parametrize("b,kernel", [(1, 1), (32, 1), (128, 1), (32, 2), (64, 2), (128, 2)],
+                         ids=["b1-bf", "b32-bf", "b128-bf", "b32-tc", "b64-tc", "b128-tc"])
+def test_mbs_dequantize_and_error(F, b, kernel):
     import gpu_util as gu
     from test_quant_error import assert_energies, run_qe
     M, K = 256, 2048
     x = make_input(M, K, seed=77 + b, adversarial=False)
     plan = F.fp4q_plan_create(o.MXFP4_MBS, 32, b, o.SCALE_OAS)
+    F.fp4q_plan_set_kernel(plan, kernel)
     out = gu.run_rotate_quantize_mbs(F, plan, x)
     flat = gu.run_dequantize_mbs(F, plan, out["codes"], out["scales"], out["macro"], unrotate=False)
     ref = o.dequantize_mbs(out["codes"], out["scales"], out["macro"], 32, b)
@@ -72,11 +79,13 @@ def test_mbs_dequantize_and_error(F, b):
     assert_energies(run_qe(F, plan, x), o.quant_error(x, o.MXFP4_MBS, 32, b, o.SCALE_OAS), f"mbs b{b}")
 
 
-def test_mbs_with_signs(F):
+@pytest.mark.parametrize("b,kernel", [(32, 1), (32, 2), (128, 2)], ids=["b32-bf", "b32-tc", "b128-tc"])
+def test_mbs_with_signs(F, b, kernel):
     import gpu_util as gu
-    M, K, b = 100, 1024, 32
+    M, K = 100, 1024
     x = make_input(M, K, seed=5, adversarial=False)
     plan = F.fp4q_plan_create(o.MXFP4_MBS, 32, b, o.SCALE_FLOOR_OCP)
+    F.fp4q_plan_set_kernel(plan, kernel)
     mask = W.random_sign_mask(K, 31)
     md = torch.from_numpy(mask.view(np.int32)).cuda()
     F.fp4q_plan_set_signs(plan, md, K)

@@ -61,21 +61,27 @@ def test_signed_rotate_quantize_matches_oracle(F, combo, kernel):
             assert abs(float(out["tensor_scale"]) - float(res["tensor_scale"])) <= 2.5e-7 * float(res["tensor_scale"])
 
 
-@pytest.mark.parametrize("b", [1, 16, 128])
-def test_signed_amax_and_quant_error(F, b):
+@pytest.mark.parametrize("b,kernel", [(1, 1), (16, 1), (128, 1), (16, 2), (32, 2), (128, 2)],
+                         ids=["b1-bf", "b16-bf", "b128-bf", "b16-tc", "b32-tc", "b128-tc"])
+def test_signed_amax_and_quant_error(F, b, kernel):
+    """The signed amax (butterfly-only pass) and the signed error pass on either kernel."""
     import gpu_util as gu
     from test_quant_error import assert_energies, run_qe
     M, K = 300, 1024
     x = make_input(M, K, seed=40 + b, adversarial=False)
     plan, s = signed_plan(F, (o.NVFP4, 16, b, o.SCALE_NV_STATIC), K, seed=7)
+    F.fp4q_plan_set_kernel(plan, kernel)
     ours = gu.run_amax(F, plan, x)
     ref = o.nv_tensor_scale(o.rotated_amax(x, b, signs=s))
     assert abs(float(ours) - float(ref)) <= 2.5e-7 * float(ref)
     assert ref != o.nv_tensor_scale(o.rotated_amax(x, b)) or b == 1
     qe_ref = o.quant_error(x, o.NVFP4, 16, b, o.SCALE_NV_STATIC, tensor_scale=ref, signs=s)
     assert_energies(run_qe(F, plan, x, tensor_scale=ref), qe_ref, f"b{b} signed")
-    mplan, ms = signed_plan(F, (o.MXFP4, 32, b, o.SCALE_OAS), K, seed=8)
-    assert_energies(run_qe(F, mplan, x), o.quant_error(x, o.MXFP4, 32, b, o.SCALE_OAS, signs=ms), f"mx b{b} signed")
+    if b >= 32 or kernel == 1:
+        mplan, ms = signed_plan(F, (o.MXFP4, 32, b, o.SCALE_OAS), K, seed=8)
+        F.fp4q_plan_set_kernel(mplan, kernel)
+        assert_energies(run_qe(F, mplan, x), o.quant_error(x, o.MXFP4, 32, b, o.SCALE_OAS, signs=ms),
+                        f"mx b{b} signed")
 
 
 @pytest.mark.parametrize("b", [2, 32, 128])
