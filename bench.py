@@ -306,6 +306,11 @@ def run_gpu(args):
                            "bytes_per_call": nbytes}
         extra["dynamic_mode"]["note"] = "reads X twice (amax pass, then quantize); bytes are the algorithmic ones"
 
+    # context for the roofline at this size: a plain device copy that reads and writes the same
+    # total bytes (half each way), timed the same way over as many rotating buffers
+    if rank == 0:
+        extra["copy_same_bytes"] = time_copy(torch, bytes_call, n_buf, stream, peak)
+
     # the randomised rotation (per-channel random signs) on the same workload, on the kernel the plan picks
     if rank == 0:
         extra["signed_rotation"] = time_signed(torch, F, w, xs, codes, scales, ts if is_nv else None, stream, peak,
@@ -514,6 +519,34 @@ def time_gemm(torch, F, fmt, M, N, K, stream, steps=50):
     return {"M": M, "N": N, "K": K, "us_per_call": round(us, 2), "TFLOPs": round(tflops, 1),
             "frac_of_fp4_peak": round(tflops / peak, 4), "fp4_peak_TFLOPs": round(peak, 1), "peak_source": kind,
             "bound": "tensor"}
+
+
+def time_copy(torch, nbytes, n_buf, stream, peak, steps=2000):
+    """A device-to-device copy of nbytes / 2 bytes (so nbytes move through HBM), over n_buf
+    rotating buffer pairs, replayed from a CUDA graph and timed with CUDA events: what a plain
+    copy achieves at the size of one call.  A reference point, not part of the path."""
+    half = nbytes // 2 // 16 * 16
+    srcs = [torch.empty(half, dtype=torch.uint8, device="cuda").fill_(1) for _ in range(n_buf)]
+    dsts = [torch.empty(half, dtype=torch.uint8, device="cuda") for _ in range(n_buf)]
+
+    def launch(i):
+        dsts[i].copy_(srcs[i], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        g, g_rem, reps = time_graph_steps(torch, launch, n_buf, steps, 3, stream)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        a1.record(stream)
+    torch.cuda.synchronize()
+    us = a0.elapsed_time(a1) * 1e3 / steps
+    gbs = 2 * half / us / 1e3
+    del srcs, dsts
+    return {"bytes_per_call": 2 * half, "us_per_call": round(us, 3), "GBps": round(gbs, 1),
+            "pct_of_hbm_peak": round(100 * gbs / peak, 2), "buffers": n_buf}
 
 
 def time_plan(torch, F, plan, w, xs, codes, scales, ts, stream, steps):
