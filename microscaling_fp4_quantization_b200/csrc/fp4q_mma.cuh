@@ -74,8 +74,8 @@ struct MmaConfig {
   static constexpr int kEpiCols = kSuperCols / kSlices;   // columns per epilogue warp
   static constexpr int kCtasPerSm = (FMT == kNV && B <= 64) ? 1 : 2;
   // plans with per-channel signs: these warps flip the signs of each landed stage's elements
-  // (four where one CTA has the SM, two beside a second CTA)
-  static constexpr int kSignWarps = kCtasPerSm == 1 ? 4 : 2;
+  // (eight where one CTA has the SM, two beside a second CTA)
+  static constexpr int kSignWarps = kCtasPerSm == 1 ? 8 : 2;
   static constexpr int kThreads = 32 * (2 + kEpiWarps + kSignWarps);
   static constexpr int kTmemCols = 2 * kSuperCols;   // two accumulator buffers
   static constexpr float kC = inv_sqrt_block(B);
