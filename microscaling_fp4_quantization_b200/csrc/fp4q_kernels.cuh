@@ -657,42 +657,51 @@ __global__ void __launch_bounds__(Cfg::kThreads) rotate_quantize_kernel(RQArgs a
 // ---------------------------------------------------------------- quantization error
 
 // E2M1 code word (element 0 in the low nibble) -> the eight values, as four fp32 pairs.
-// Nibble c = s|k (k = magnitude code) becomes the fp32 bit pattern s<<31 | k<<22, which is
-// 2^-126 * {0, 0.5, 1, 1.5, 2, 3, 4, 6}[k] (k = 1 a subnormal), then an exact product by
-// 2^126 (subnormals are kept: nothing here is compiled with flush-to-zero).
-__device__ __forceinline__ void e2m1x8_decode(uint32_t w, f32x2 (&d)[4]) {
-  const f32x2 up = f2_pack(0x1p126f, 0x1p126f);
-#pragma unroll
-  for (int t = 0; t < 4; ++t) {
-    const uint32_t n0 = w >> (8 * t), n1 = w >> (8 * t + 4);
-    const uint32_t b0 = ((n0 & 7u) << 22) | ((n0 & 8u) << 28);
-    const uint32_t b1 = ((n1 & 7u) << 22) | ((n1 & 8u) << 28);
-    d[t] = f2_mul(f2_pack(__uint_as_float(b0), __uint_as_float(b1)), up);
-  }
+// The magnitude bits of nibble E of a code word, as the fp32 pattern k << 22 (k = magnitude
+// code 0..7).  That pattern is 2^-126 * {0, 0.5, 1, 1.5, 2, 3, 4, 6}[k] exactly (k = 1 a
+// subnormal; nothing here is compiled with flush-to-zero).
+template <int E>
+__device__ __forceinline__ float e2m1_mag_scaled(uint32_t w) {
+  constexpr int s = 22 - 4 * E;
+  return __uint_as_float((s >= 0 ? (w << s) : (w >> -s)) & 0x01C00000u);
 }
 
 // Error energy of one group of quotients v (= y / X) against their E2M1 codes, and its
-// signal energy, both in units of X^2: sum (v - q)^2 and sum v^2 (fp32, pairwise lanes).
+// signal energy, both in units of X^2: sum (v - q)^2 and sum v^2 (fp32; even and odd elements
+// in separate sums).  E2M1 rounding keeps the sign of v, so v - q = sign(v) (|v| - |q|), and
+// |v| - |q| is one fused multiply-add of the scaled magnitude by -2^126 (the product is exact).
 template <int NP>
 __device__ __forceinline__ void group_energies(const f32x2 (&v)[NP], float& sig, float& err) {
-  f32x2 as = f2_pack(0.0f, 0.0f), ae = f2_pack(0.0f, 0.0f);
+  f32x2 as = f2_pack(0.0f, 0.0f);
+  float e0 = 0.0f, e1 = 0.0f;
 #pragma unroll
   for (int j = 0; j < NP / 4; ++j) {
     f32x2 vv[4];
 #pragma unroll
     for (int t = 0; t < 4; ++t) vv[t] = v[4 * j + t];
-    f32x2 d[4];
-    e2m1x8_decode(e2m1x8_pairs(vv), d);
+    const uint32_t w = e2m1x8_pairs(vv);
+    float lo[4], hi[4], q0[4], q1[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) f2_unpack(vv[t], lo[t], hi[t]);
+    q0[0] = e2m1_mag_scaled<0>(w);
+    q1[0] = e2m1_mag_scaled<1>(w);
+    q0[1] = e2m1_mag_scaled<2>(w);
+    q1[1] = e2m1_mag_scaled<3>(w);
+    q0[2] = e2m1_mag_scaled<4>(w);
+    q1[2] = e2m1_mag_scaled<5>(w);
+    q0[3] = e2m1_mag_scaled<6>(w);
+    q1[3] = e2m1_mag_scaled<7>(w);
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
-      const f32x2 e = f2_sub(vv[t], d[t]);
       as = f2_fma(vv[t], vv[t], as);
-      ae = f2_fma(e, e, ae);
+      const float d0 = fmaf(q0[t], -0x1p126f, fabsf(lo[t]));
+      const float d1 = fmaf(q1[t], -0x1p126f, fabsf(hi[t]));
+      e0 = fmaf(d0, d0, e0);
+      e1 = fmaf(d1, d1, e1);
     }
   }
-  float a0, a1, e0, e1;
+  float a0, a1;
   f2_unpack(as, a0, a1);
-  f2_unpack(ae, e0, e1);
   sig = a0 + a1;
   err = e0 + e1;
 }
