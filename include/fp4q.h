@@ -260,6 +260,13 @@ fp4q_status fp4q_rotate_quantize_nvfp4_dynamic_noalloc(const void* x_bf16, int64
  * wait ran out in a kernel since the last read).  Synchronizes the current device. */
 fp4q_status fp4q_device_status(void);
 
+/* Self-test of the failure path: launches one warp that waits on a shared-memory barrier
+ * nothing arrives on.  The wait is bounded like every wait in the library; after about one
+ * second it records FP4Q_ERR_TIMEOUT in the device status word and the kernel returns, so
+ * the CUDA context stays usable and the next fp4q_device_status returns FP4Q_ERR_TIMEOUT.
+ * No fault, trap or unbounded wait is involved.  stream: as for the other calls. */
+fp4q_status fp4q_selftest_wait_timeout(void* stream);
+
 /* Static string for a status code. */
 const char* fp4q_status_string(fp4q_status status);
 

@@ -665,6 +665,10 @@ fp4q_status fp4q_gemm(int format, const void* a_codes, const void* a_scales, con
   return launch_gemm<kNV>(ac, as, a_tensor_scale, bc, bs, b_tensor_scale, M, N, K, d, s);
 }
 
+fp4q_status fp4q_selftest_wait_timeout(void* stream) {
+  return launch_wait_timeout_selftest(static_cast<cudaStream_t>(stream));
+}
+
 fp4q_status fp4q_device_status(void) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");

@@ -146,6 +146,8 @@ fp4q_status status_mbs(unsigned int* v);
 fp4q_status status_qe(unsigned int* v);
 fp4q_status status_mma(unsigned int* v);
 fp4q_status status_mma_qe(unsigned int* v);
+// One warp whose bounded wait runs out (fp4q_selftest_wait_timeout).
+fp4q_status launch_wait_timeout_selftest(cudaStream_t stream);
 fp4q_status status_dequant(unsigned int* v);
 fp4q_status status_gemm(unsigned int* v);
 

@@ -25,6 +25,13 @@ fp4q_status launch_quant_error_empty(const double* partials, double* out, cudaSt
   return FP4Q_OK;
 }
 
+fp4q_status launch_wait_timeout_selftest(cudaStream_t stream) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return FP4Q_OK;
+}
+
 }  // namespace host
 }  // namespace fp4q
 

@@ -863,6 +863,16 @@ __global__ void __launch_bounds__(Cfg::kThreads) quant_error_kernel(QEArgs a) {
   }
 }
 
+// One warp waits on a barrier that nothing arrives on: the bounded wait gives up after
+// kWaitLimitNs, records kStatusTimeout and the kernel returns (the failure path's self-test).
+static __global__ void wait_timeout_selftest_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = static_cast<uint32_t>(__cvta_generic_to_shared(&bar));
+  if (threadIdx.x == 0) mbar_init(b, 1);
+  __syncwarp();
+  mbar_wait_bounded(b, 0u);   // phase 0 never completes
+}
+
 // The same result for an empty X (no CTA to finish): {0, 0, +inf}.  One warp.
 static __global__ void quant_error_empty_kernel(const double* __restrict__ partials, double* __restrict__ out) {
   pdl_launch_dependents();

@@ -46,6 +46,7 @@ _SIGS = {
     "fp4q_dequantize_mbs": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _int, _vp, _vp]),
     "fp4q_gemm": (_int, [_int, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp]),
     "fp4q_device_status": (_int, []),
+    "fp4q_selftest_wait_timeout": (_int, [_vp]),
     "fp4q_status_string": (ctypes.c_char_p, [_int]),
     "fp4q_last_cuda_error": (ctypes.c_char_p, []),
     "fp4q_version": (_int, []),
@@ -194,6 +195,11 @@ def fp4q_gemm(fmt: int, a_codes, a_scales, a_tensor_scale, b_codes, b_scales, b_
 
 def fp4q_device_status() -> int:
     return _lib.fp4q_device_status()
+
+
+def fp4q_selftest_wait_timeout(stream=None) -> None:
+    """One warp whose bounded wait runs out: the next fp4q_device_status is FP4Q_ERR_TIMEOUT."""
+    _check(_lib.fp4q_selftest_wait_timeout(_stream(stream)), "fp4q_selftest_wait_timeout")
 
 
 def fp4q_status_string(status: int) -> str:
