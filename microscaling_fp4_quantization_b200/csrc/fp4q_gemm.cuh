@@ -15,7 +15,7 @@
 // 48-column scale-factor buffers and the 256-column accumulator (a second accumulator, which
 // would let the epilogue overlap the next tile, does not fit next to them at this width;
 // measured, the narrower tiles that make room cost more in the mainloop than the overlap
-// saves).  Roles (10 warps):
+// saves).  Roles (14 warps):
 //   warp 0      producer: TMA loads of the A (128 rows x 128 B) and B (256 rows x 128 B) code
 //               tiles, 128-byte swizzled, completion on the stage's "full" barrier;
 //   warp 1      TMEM owner and MMA issuer: per stage, tcgen05.cp of the stage's scale factors
@@ -23,9 +23,10 @@
 //               four MMAs, then tcgen05.commit to free the stage; after a tile, commit to the
 //               epilogue (issuing a stage's copies a stage earlier measured no faster: the copies
 //               and the MMAs share the tensor pipe);
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (lane quarter = warp % 4), times alpha,
+//   warps 2..9  epilogue, two per TMEM lane quarter (warp % 4), each taking half of the 256
+//               accumulator columns: tcgen05.ld of the accumulator, times alpha,
 //               to bf16, stored straight to D; then frees the accumulator;
-//   warps 6..9  scale rearrangers, one per ring slot: each reads the row-major scale bytes of
+//   warps 10..13 scale rearrangers, one per ring slot: each reads the row-major scale bytes of
 //               its slot's stages and writes them in the layout tcgen05.cp reads (per MMA and
 //               128 rows: 32 rows of 16 bytes, row l = the 4-byte scale words of rows l, l+32,
 //               l+64, l+96), then "sf full".  A warp loads its next stage's words before it
@@ -77,7 +78,10 @@ struct GemmConfig {
   static_assert(kBN % 16 == 0 && kAccCol0 % 16 == 0, "MMA N and accumulator columns in steps of 16");
   static constexpr int kBRowGroups = kBN / 32;             // 32-row groups of B (2 copy blocks of 4)
   static_assert(kBN % 32 == 0 && kBRowGroups <= 8, "B tile of at most 256 rows in 32-row groups");
-  static constexpr int kEpiWarp0 = 2, kScaleWarp0 = 6;
+  // eight epilogue warps drain the single accumulator twice as fast as four (the MMAs of
+  // the next tile wait for it)
+  static constexpr int kEpiWarps = 8;
+  static constexpr int kEpiWarp0 = 2, kScaleWarp0 = kEpiWarp0 + kEpiWarps;
   static constexpr int kThreads = 32 * (kScaleWarp0 + kStages);
   // instruction descriptor: E2M1 x E2M1 (format 1), K-major A and B, N >> 3, scale format
   // (1 = E8M0, 0 = E4M3), M >> 4; dense, no negation, scale-factor ids 0
@@ -173,7 +177,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
     }
     for (int d = 0; d < 2; ++d) {
       mbar_init(acc_full(d), 1);
-      mbar_init(acc_empty(d), 4);
+      mbar_init(acc_empty(d), Cfg::kEpiWarps);
     }
     fence_mbar_init();
   }
@@ -313,8 +317,10 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
         mbar_wait_bounded(acc_full((tc - 1) % Cfg::kAccBufs), static_cast<uint32_t>(((tc - 1) / Cfg::kAccBufs) & 1));
     }
   } else {
-    // ---------------- epilogue: warps 2..5, TMEM lane quarter warp % 4
+    // ---------------- epilogue: warps 2..9, TMEM lane quarter warp % 4, column half (warp - 2) / 4
     const int q = warp & 3;
+    constexpr int kColChunks = Cfg::kBN / 16 / (Cfg::kEpiWarps / 4);   // 16-column chunks per warp
+    const int c0 = ((warp - Cfg::kEpiWarp0) >> 2) * kColChunks;
     pdl_wait();   // the tensor scales come from earlier kernels, and D may still be read by one
     const float alpha = Cfg::kFmt == kNV ? (*g.a_tensor_scale) * (*g.b_tensor_scale) : 1.0f;
     int tc = 0;
@@ -326,19 +332,24 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
       tc_fence_after();
       const int64_t row = static_cast<int64_t>(tm) * Cfg::kBM + 32 * q + lane;
       const uint32_t acc = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + Cfg::kAccCol0 + d * Cfg::kBN;
+      static_assert(kColChunks % 2 == 0, "chunks are read in pairs");
 #pragma unroll 1
-      for (int c = 0; c < Cfg::kBN / 16; ++c) {
-        float v[16];
-        tmem_ld16(acc + c * 16, v);
+      for (int c = c0; c < c0 + kColChunks; c += 2) {
+        float v[2][16];
+        tmem_ld16(acc + c * 16, v[0]);   // two 16-column chunks per wait
+        tmem_ld16(acc + c * 16 + 16, v[1]);
         tmem_wait_ld();
-        const int64_t col0 = static_cast<int64_t>(tn) * Cfg::kBN + 16 * c;
-        if (row < g.M && col0 < g.N) {
-          uint32_t w[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(v[2 * i] * alpha, v[2 * i + 1] * alpha);
-          uint16_t* dp = g.d + row * g.N + col0;
-          stg128(dp, w[0], w[1], w[2], w[3]);
-          stg128(dp + 8, w[4], w[5], w[6], w[7]);
+        for (int h = 0; h < 2; ++h) {
+          const int64_t col0 = static_cast<int64_t>(tn) * Cfg::kBN + 16 * (c + h);
+          if (row < g.M && col0 < g.N) {
+            uint32_t w[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(v[h][2 * i] * alpha, v[h][2 * i + 1] * alpha);
+            uint16_t* dp = g.d + row * g.N + col0;
+            stg128(dp, w[0], w[1], w[2], w[3]);
+            stg128(dp + 8, w[4], w[5], w[6], w[7]);
+          }
         }
       }
       // the accumulator can be reused once every epilogue warp has read it
