@@ -656,7 +656,6 @@ __global__ void __launch_bounds__(Cfg::kThreads) rotate_quantize_kernel(RQArgs a
 
 // ---------------------------------------------------------------- quantization error
 
-// E2M1 code word (element 0 in the low nibble) -> the eight values, as four fp32 pairs.
 // The magnitude bits of nibble E of a code word, as the fp32 pattern k << 22 (k = magnitude
 // code 0..7).  That pattern is 2^-126 * {0, 0.5, 1, 1.5, 2, 3, 4, 6}[k] exactly (k = 1 a
 // subnormal; nothing here is compiled with flush-to-zero).
