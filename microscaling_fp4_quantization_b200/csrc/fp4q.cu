@@ -32,7 +32,7 @@ fp4q_status cuda_fail(cudaError_t e, const char* what) {
   return FP4Q_ERR_CUDA;
 }
 
-fp4q_status kernel_info_impl(const void* kernel, int smem_bytes, int threads, KernelInfo* out) {
+fp4q_status kernel_info_impl(const void* kernel, int smem_bytes, int threads, KernelInfo* out, int max_smem_bytes) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
@@ -46,7 +46,8 @@ fp4q_status kernel_info_impl(const void* kernel, int smem_bytes, int threads, Ke
   KernelInfo ki;
   e = cudaDeviceGetAttribute(&ki.sm_count, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           max_smem_bytes > smem_bytes ? max_smem_bytes : smem_bytes);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
   // all of the unified L1 / shared storage as shared memory: these kernels stage through it
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);

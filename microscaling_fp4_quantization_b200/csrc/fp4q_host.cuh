@@ -46,11 +46,21 @@ struct KernelInfo {
   int ctas_per_sm = 0;
   int sm_count = 0;
 };
-fp4q_status kernel_info_impl(const void* kernel, int smem_bytes, int threads, KernelInfo* out);
+// Occupancy is computed for smem_bytes; the kernel may be launched with up to max_smem_bytes
+// (when larger) of dynamic shared memory.  The first call for a kernel sets both, so every
+// call for one kernel passes the same sizes.
+fp4q_status kernel_info_impl(const void* kernel, int smem_bytes, int threads, KernelInfo* out, int max_smem_bytes);
 
 template <class K>
-fp4q_status kernel_info(K kernel, int smem_bytes, int threads, KernelInfo* out) {
-  return kernel_info_impl(reinterpret_cast<const void*>(kernel), smem_bytes, threads, out);
+fp4q_status kernel_info(K kernel, int smem_bytes, int threads, KernelInfo* out, int max_smem_bytes = 0) {
+  return kernel_info_impl(reinterpret_cast<const void*>(kernel), smem_bytes, threads, out, max_smem_bytes);
+}
+
+// The butterfly kernels (rotate + quantize, error pass, amax) may stage a sign mask of up to
+// kSignSmemMaxWords words behind their stages.
+template <class Cfg, class K>
+fp4q_status butterfly_kernel_info(K kernel, KernelInfo* out) {
+  return kernel_info(kernel, Cfg::kSmemBytes, Cfg::kThreads, out, Cfg::kSmemBytes + 4 * kSignSmemMaxWords);
 }
 
 // Launch with programmatic stream serialization, so the kernel's start overlaps the tail of
@@ -93,7 +103,9 @@ template <class Cfg>
 ChannelSigns channel_signs(const uint32_t* mask, int64_t K) {
   if (!mask) return ChannelSigns{nullptr, 1, 0};
   const int upr = static_cast<int>(K / Cfg::kE);
-  return ChannelSigns{mask, upr, static_cast<int>(Cfg::kUnitsPerStage % upr)};
+  const int64_t words = (K + 31) / 32;   // the caller's mask, ceil(K / 32) words
+  return ChannelSigns{mask, upr, static_cast<int>(Cfg::kUnitsPerStage % upr),
+                      words <= kSignSmemMaxWords ? static_cast<int>(words) : 0};
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,

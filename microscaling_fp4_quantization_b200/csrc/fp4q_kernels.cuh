@@ -139,7 +139,23 @@ struct ChannelSigns {
   const uint32_t* mask;
   int upr;
   int stage_step;
+  int smem_words = 0;   // butterfly kernels: words of the mask to stage in shared memory (0: read it in place)
 };
+
+// Most mask words a butterfly CTA stages in shared memory (16 KB: K <= 131072).
+constexpr int kSignSmemMaxWords = 4096;
+
+// Butterfly kernels with channel signs: the CTA copies the mask's words behind its stages
+// (dynamic shared memory from byte `offset`) and reads them from there; called by every thread
+// of the CTA, after the grid dependency (the mask may come from an earlier kernel).
+__device__ __forceinline__ ChannelSigns stage_signs_in_smem(ChannelSigns sg, uint8_t* smem, int offset) {
+  if (sg.mask == nullptr || sg.smem_words == 0) return sg;
+  uint32_t* ms = reinterpret_cast<uint32_t*>(smem + offset);
+  for (int w = threadIdx.x; w < sg.smem_words; w += blockDim.x) ms[w] = __ldg(sg.mask + w);
+  __syncthreads();
+  sg.mask = ms;
+  return sg;
+}
 
 struct RQArgs {
   const uint16_t* x;       // bf16 [n_units * E]
@@ -195,9 +211,9 @@ __device__ __forceinline__ UnitSigns<E> unit_signs(const uint32_t* mask, int cu)
   const int c0 = cu * E;
   if constexpr (E >= 32) {
 #pragma unroll
-    for (int i = 0; i < E / 32; ++i) m.w[i] = __ldg(mask + (c0 >> 5) + i);
+    for (int i = 0; i < E / 32; ++i) m.w[i] = mask[(c0 >> 5) + i];   // shared or global memory
   } else {
-    m.w[0] = (__ldg(mask + (c0 >> 5)) >> (c0 & 31)) & 0xFFFFu;
+    m.w[0] = (mask[c0 >> 5] >> (c0 & 31)) & 0xFFFFu;
   }
   return m;
 }
@@ -648,9 +664,11 @@ __global__ void __launch_bounds__(Cfg::kThreads) rotate_quantize_kernel(RQArgs a
   auto body = [&](const f32x2 (&p)[Cfg::kPairs], int64_t unit) {
     quantize_store_unit<Cfg>(p, unit, lx, s_g, nv_den, nv_rden, a);
   };
-  if (a.signs.mask)
-    stream_units<Cfg, true>(a.x, a.n_units, smem + warp * Cfg::kWarpSmem, lx.tau, body, a.signs);
-  else
+  if (a.signs.mask) {
+    pdl_wait();
+    const ChannelSigns sg = stage_signs_in_smem(a.signs, smem, Cfg::kSmemBytes);
+    stream_units<Cfg, true>(a.x, a.n_units, smem + warp * Cfg::kWarpSmem, lx.tau, body, sg);
+  } else
     stream_units<Cfg>(a.x, a.n_units, smem + warp * Cfg::kWarpSmem, lx.tau, body);
 }
 
@@ -828,9 +846,11 @@ __global__ void __launch_bounds__(Cfg::kThreads) quant_error_kernel(QEArgs a) {
   const float nv_rden = __frcp_rn(nv_den);
   double sig = 0.0, err = 0.0;
   auto body = [&](const f32x2 (&p)[Cfg::kPairs], int64_t) { unit_energies<Cfg>(p, s_g, nv_den, nv_rden, sig, err); };
-  if (a.signs.mask)
-    stream_units<Cfg, true>(a.x, a.n_units, smem + warp * Cfg::kWarpSmem, lx.tau, body, a.signs);
-  else
+  if (a.signs.mask) {
+    pdl_wait();
+    const ChannelSigns sg = stage_signs_in_smem(a.signs, smem, Cfg::kSmemBytes);
+    stream_units<Cfg, true>(a.x, a.n_units, smem + warp * Cfg::kWarpSmem, lx.tau, body, sg);
+  } else
     stream_units<Cfg>(a.x, a.n_units, smem + warp * Cfg::kWarpSmem, lx.tau, body);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -890,9 +910,11 @@ __global__ void __launch_bounds__(Cfg::kThreads) rotated_amax_kernel(const uint1
   const LaneXor lx = lane_xor<Cfg>(threadIdx.x & 31);
   float m = 0.0f;
   auto body = [&](const f32x2 (&p)[Cfg::kPairs], int64_t) { m = fmaxf(m, pairs_amax<Cfg::kPairs>(p)); };
-  if (signs.mask)
-    stream_units<Cfg, true>(x, n_units, smem + warp * Cfg::kWarpSmem, lx.tau, body, signs);
-  else
+  if (signs.mask) {
+    pdl_wait();
+    const ChannelSigns sg = stage_signs_in_smem(signs, smem, Cfg::kSmemBytes);
+    stream_units<Cfg, true>(x, n_units, smem + warp * Cfg::kWarpSmem, lx.tau, body, sg);
+  } else
     stream_units<Cfg>(x, n_units, smem + warp * Cfg::kWarpSmem, lx.tau, body);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));

@@ -16,13 +16,14 @@ fp4q_status launch_rq(RQArgs a, int64_t n_elems, cudaStream_t stream, int64_t K)
   a.signs = channel_signs<Cfg>(a.signs.mask, K);
   auto kernel = rotate_quantize_kernel<Cfg>;
   KernelInfo ki;
-  fp4q_status st = kernel_info(kernel, Cfg::kSmemBytes, Cfg::kThreads, &ki);
+  fp4q_status st = butterfly_kernel_info<Cfg>(kernel, &ki);
   if (st != FP4Q_OK) return st;
   const int64_t warps_needed = (a.n_units + Cfg::kUnitsPerStage - 1) / Cfg::kUnitsPerStage;
   int64_t ctas = (warps_needed + Cfg::kWarps - 1) / Cfg::kWarps;
   const int64_t max_ctas = static_cast<int64_t>(ki.sm_count) * ki.ctas_per_sm;
   if (ctas > max_ctas) ctas = max_ctas;
-  cudaError_t e = launch_pdl(kernel, dim3(static_cast<unsigned>(ctas)), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, a);
+  cudaError_t e = launch_pdl(kernel, dim3(static_cast<unsigned>(ctas)), dim3(Cfg::kThreads),
+                             Cfg::kSmemBytes + 4 * a.signs.smem_words, stream, a);
   if (e != cudaSuccess) return cuda_fail(e, "rotate_quantize launch");
   return FP4Q_OK;
 }
@@ -107,7 +108,7 @@ fp4q_status launch_mma_qe(const QEArgs& qa, int64_t n_elems, cudaStream_t stream
 template <class Cfg>
 fp4q_status qe_wave(int* n) {
   KernelInfo ki;
-  fp4q_status r = kernel_info(quant_error_kernel<Cfg>, Cfg::kSmemBytes, Cfg::kThreads, &ki);
+  fp4q_status r = butterfly_kernel_info<Cfg>(quant_error_kernel<Cfg>, &ki);
   *n = ki.sm_count * ki.ctas_per_sm;
   return r;
 }
@@ -118,7 +119,7 @@ fp4q_status launch_qe(fp4q_plan p, QEArgs a, int64_t n_elems, double* out, cudaS
   a.signs = channel_signs<Cfg>(p->signs, p->signs_K);
   auto kernel = quant_error_kernel<Cfg>;
   KernelInfo ki;
-  fp4q_status st = kernel_info(kernel, Cfg::kSmemBytes, Cfg::kThreads, &ki);
+  fp4q_status st = butterfly_kernel_info<Cfg>(kernel, &ki);
   if (st != FP4Q_OK) return st;
   const int64_t warps_needed = (a.n_units + Cfg::kUnitsPerStage - 1) / Cfg::kUnitsPerStage;
   int64_t ctas = (warps_needed + Cfg::kWarps - 1) / Cfg::kWarps;
@@ -126,7 +127,8 @@ fp4q_status launch_qe(fp4q_plan p, QEArgs a, int64_t n_elems, double* out, cudaS
   if (ctas > max_ctas) ctas = max_ctas;
   if (ctas > p->n_err_partials) ctas = p->n_err_partials;
   a.out = out;
-  cudaError_t e = launch_pdl(kernel, dim3(static_cast<unsigned>(ctas)), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, a);
+  cudaError_t e = launch_pdl(kernel, dim3(static_cast<unsigned>(ctas)), dim3(Cfg::kThreads),
+                             Cfg::kSmemBytes + 4 * a.signs.smem_words, stream, a);
   if (e != cudaSuccess) return cuda_fail(e, "quant_error launch");
   return FP4Q_OK;
 }
@@ -134,7 +136,7 @@ fp4q_status launch_qe(fp4q_plan p, QEArgs a, int64_t n_elems, double* out, cudaS
 template <class Cfg>
 fp4q_status amax_wave(int* n) {
   KernelInfo ki;
-  fp4q_status r = kernel_info(rotated_amax_kernel<Cfg>, Cfg::kSmemBytes, Cfg::kThreads, &ki);
+  fp4q_status r = butterfly_kernel_info<Cfg>(rotated_amax_kernel<Cfg>, &ki);
   *n = ki.sm_count * ki.ctas_per_sm;
   return r;
 }
@@ -143,11 +145,12 @@ template <class Cfg>
 fp4q_status launch_amax_cfg(const uint16_t* x, int64_t n_elems, float* partials, int n_partials, ChannelSigns sg,
                             cudaStream_t stream, bool pdl) {
   cudaError_t e;
+  const size_t smem = Cfg::kSmemBytes + 4 * static_cast<size_t>(sg.smem_words);
   if (pdl) {
-    e = launch_pdl(rotated_amax_kernel<Cfg>, dim3(n_partials), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, x,
+    e = launch_pdl(rotated_amax_kernel<Cfg>, dim3(n_partials), dim3(Cfg::kThreads), smem, stream, x,
                    n_elems / Cfg::kE, partials, sg);
   } else {
-    rotated_amax_kernel<Cfg><<<n_partials, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(x, n_elems / Cfg::kE, partials, sg);
+    rotated_amax_kernel<Cfg><<<n_partials, Cfg::kThreads, smem, stream>>>(x, n_elems / Cfg::kE, partials, sg);
     e = cudaGetLastError();
   }
   if (e != cudaSuccess) return cuda_fail(e, "amax launch");
