@@ -128,3 +128,22 @@ def test_weight_path_gemm_identity(F):
     for A, q in ((X, xq), (Wt, wq)):
         res = o.rotate_quantize(A, o.MXFP4, 32, b, o.SCALE_OAS, signs=s)
         assert_parity(res, q["codes"], q["scales"], "weight path")
+
+
+@pytest.mark.parametrize("combo,kernel", [((o.MXFP4, 32, 32, o.SCALE_OAS), 1), ((o.MXFP4, 32, 32, o.SCALE_OAS), 2),
+                                          ((o.NVFP4, 16, 16, o.SCALE_NV_STATIC), 1),
+                                          ((o.NVFP4, 16, 128, o.SCALE_NV_STATIC), 2)],
+                         ids=["mx-b32-bf", "mx-b32-tc", "nv-b16-bf", "nv-b128-tc"])
+def test_signed_rows_longer_than_the_staged_mask(F, combo, kernel):
+    """K = 135168: the mask (4224 words, 16.5 KB) is larger than either kernel stages in shared
+    memory, so both read it where the caller keeps it."""
+    import gpu_util as gu
+    fmt, g, b, rule = combo
+    M, K = 3, 135168
+    plan, s = signed_plan(F, combo, K, seed=77)
+    F.fp4q_plan_set_kernel(plan, kernel)
+    x = make_input(M, K, seed=4242 + b, adversarial=False)
+    s_g = o.nv_tensor_scale(o.rotated_amax(x, b, signs=s)) if rule == o.SCALE_NV_STATIC else None
+    res = o.rotate_quantize(x, fmt, g, b, rule, tensor_scale=s_g, signs=s)
+    out = gu.run_rotate_quantize(F, plan, x, tensor_scale=s_g)
+    assert_parity(res, out["codes"], out["scales"], f"{combo_id(combo)} K={K} signed")
