@@ -454,23 +454,35 @@ def dequantize(codes: np.ndarray, scales: np.ndarray, fmt: int, group: int, bloc
 E2M1_MIDPOINTS = (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0)
 
 
-def _near_scaled_power(A: np.ndarray, base: float, tol: float) -> np.ndarray:
-    """|A - base*2^k| <= tol * base*2^k for the nearest k (A > 0)."""
+def _dist_scaled_power(A: np.ndarray, base: float) -> np.ndarray:
+    """Relative distance |A - base*2^k| / (base*2^k) to the nearest point base*2^k (A > 0);
+    +inf where A = 0 (no boundary near zero)."""
     A = np.asarray(A, np.float64)
-    out = np.zeros(A.shape, bool)
+    out = np.full(A.shape, np.inf)
     pos = A > 0
     k = np.round(np.log2(A[pos] / base))
     ref = base * np.exp2(k)
-    out[pos] = np.abs(A[pos] - ref) <= tol * ref
+    out[pos] = np.abs(A[pos] - ref) / ref
     return out
 
 
-def flags(res: dict, tol: float = 1e-5):
-    """Elements and groups whose exact value lies within ``tol`` (relative) of a place
-    where the code changes: an E2M1 midpoint for elements; the scale rule's boundary
-    (2^k floor, 1.5*2^k ceil, 1.75*2^k OAS, an E4M3 midpoint for NV) for groups.
+def boundary_distance(res: dict):
+    """How far each decision of the oracle's result lies from a place where it flips.
 
-    Returns (element_flags (M, K) bool, group_flags (M, K/group) bool)."""
+    Element: the relative distance of the exact |y| / S to the nearest E2M1 rounding midpoint
+    (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5: the codes change only there; above 6 everything
+    saturates to 6, so 6 is no boundary).  Group: the relative distance of its exact amax to
+    the nearest boundary of the scale rule, where the scale byte steps:
+      floor (OCP)  2^k            (floor(log2 A) steps)
+      ceil         1.5 * 2^k      (ceil(log2(A / 6)) steps at 6 * 2^j = 1.5 * 2^(j+2))
+      OAS          1.5 * 2^k and 1.75 * 2^k (the ceil rule's boundary, and the top of the
+                   [3, 3.5] window it pushes down)
+      NV           the nearest midpoint between two E4M3 values of s_b = A / (6 s_g)
+    and, for MBS, also the distance of the macro block's exact 256 f to an integer (where
+    the ceil of m8 steps), divided by 256, for every group of the block.  The group rule of
+    MBS sees A / s_M.  Distances are +inf where there is no boundary (a zero amax).
+
+    Returns (element distances (M, K), group distances (M, K/group)), float64."""
     y64 = res["y64"]
     M, K = y64.shape
     g = res["group"]
@@ -479,35 +491,53 @@ def flags(res: dict, tol: float = 1e-5):
     S = res["S64"]
     with np.errstate(divide="ignore", invalid="ignore"):
         a = np.where(S[..., None] > 0, yg / np.where(S > 0, S, 1.0)[..., None], 0.0)
-    el = np.zeros(a.shape, bool)
+    el = np.full(a.shape, np.inf)
     for mp in E2M1_MIDPOINTS:
-        el |= np.abs(a - mp) <= tol * mp
+        el = np.minimum(el, np.abs(a - mp) / mp)
+    # a zero scale (all-zero group, or a zero NV block scale) makes every code 0: no element
+    # boundary there
+    el = np.where((S > 0)[..., None], el, np.inf)
     rule = res["rule"]
     if res["fmt"] in (MXFP4, MXFP4_MBS):
         if res["fmt"] == MXFP4_MBS:
-            # the group rule sees A / s_M; a macro block whose exact 256 f lies within tol of an
-            # integer (where the ceil can step) flags all of its groups
             sM = np.repeat(mbs_macro_scale(res["macro"]).astype(np.float64), MBS_MACRO // g, axis=1)
             A64 = A64 / sM
-            ym = np.abs(y64.reshape(M, K // MBS_MACRO, MBS_MACRO))
-            r = ym.max(axis=2) / 6.0 if K else np.zeros((M, 0))
-            mm, _ = np.frexp(r)
-            t = np.where(r > 0, (2.0 * mm - 1.0) * 256.0, 0.0)
-            near_m = (np.abs(t - np.round(t)) <= tol * 256.0) & (r > 0)
+            dm = mbs_macro_distance(res)
         base = {SCALE_FLOOR_OCP: 1.0, SCALE_CEIL_NOCLIP: 1.5, SCALE_OAS: 1.75}[rule]
-        gr = _near_scaled_power(A64, base, tol)
+        gr = _dist_scaled_power(A64, base)
         if rule == SCALE_OAS:
-            gr |= _near_scaled_power(A64, 1.5, tol)
+            gr = np.minimum(gr, _dist_scaled_power(A64, 1.5))
         if res["fmt"] == MXFP4_MBS:
-            gr |= np.repeat(near_m, MBS_MACRO // g, axis=1)
+            gr = np.minimum(gr, np.repeat(dm, MBS_MACRO // g, axis=1))
     else:
         s_b = A64 / (6.0 * np.float64(res["tensor_scale"]))
         T = e4m3_table()
         mids = (T[1:] + T[:-1]) / 2.0
         idx = np.clip(np.searchsorted(mids, s_b), 1, len(mids) - 1)
-        near = np.minimum(np.abs(s_b - mids[idx - 1]) / mids[idx - 1], np.abs(s_b - mids[idx]) / mids[idx])
-        gr = near <= tol
+        gr = np.minimum(np.abs(s_b - mids[idx - 1]) / mids[idx - 1], np.abs(s_b - mids[idx]) / mids[idx])
     return el.reshape(M, K), gr
+
+
+def mbs_macro_distance(res: dict) -> np.ndarray:
+    """MBS: for every macro block, the distance of its exact 256 f (A_M / 6 = 2^E (1 + f)) to
+    the nearest integer, divided by 256 — where m8 = ceil(256 f) steps.  +inf for a zero
+    block.  Shape (M, K/128)."""
+    y64 = res["y64"]
+    M, K = y64.shape
+    ym = np.abs(y64.reshape(M, K // MBS_MACRO, MBS_MACRO))
+    r = ym.max(axis=2) / 6.0 if K else np.zeros((M, 0))
+    mm, _ = np.frexp(r)
+    t = np.where(r > 0, (2.0 * mm - 1.0) * 256.0, 0.0)
+    return np.where(r > 0, np.abs(t - np.round(t)) / 256.0, np.inf)
+
+
+def flags(res: dict, tol: float = 1e-5):
+    """The flagged set F of the parity rule: elements and groups whose exact value lies
+    within ``tol`` (relative) of a place where the code changes (``boundary_distance``).
+
+    Returns (element_flags (M, K) bool, group_flags (M, K/group) bool)."""
+    el, gr = boundary_distance(res)
+    return el <= tol, gr <= tol
 
 
 # ----------------------------------------------------------------------------------

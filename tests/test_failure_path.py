@@ -6,7 +6,7 @@ import numpy as np
 import pytest
 
 import oracle as o
-from parity import assert_parity
+from oracle.parity import assert_parity
 from test_parity_small import make_input
 
 pytestmark = pytest.mark.gpu

@@ -13,7 +13,7 @@ import torch
 
 import oracle as o
 from microscaling_fp4_quantization_b200 import workloads as W
-from parity import assert_parity
+from oracle.parity import assert_parity
 from test_parity_small import make_input
 
 pytestmark = pytest.mark.gpu
@@ -29,9 +29,9 @@ def F(cuda_device):
 
 
 def check_macro(res, out, label):
-    _, gr = o.flags(res)
-    M = res["macro"].shape[0]
-    flagged_macro = gr.reshape(M, -1, 4).all(axis=2)
+    """Macro bytes match except on macro blocks whose exact 256 f is within 1e-5 (times 256)
+    of an integer (compare() also judges them, given the bytes; this names them alone)."""
+    flagged_macro = o.mbs_macro_distance(res) <= 1e-5
     bad = (res["macro"] != out["macro"]) & ~flagged_macro
     assert not bad.any(), (label, int(bad.sum()))
 
@@ -51,13 +51,14 @@ def test_mbs_matches_oracle(F, b, kernel, rule):
         res = o.rotate_quantize_mbs(x, 32, b, rule)
         out = gu.run_rotate_quantize_mbs(F, plan, x)
         label = f"mbs b{b} {W.RULE_NAMES[rule]} {M}x{K}"
-        assert_parity(res, out["codes"], out["scales"], label, count_bound=M < 8)
+        assert_parity(res, out["codes"], out["scales"], label, count_bound=M < 8, macro_gpu=out["macro"])
         check_macro(res, out, label)
         if M >= 8:
             real = slice(8, M)
             res_r = {k: (v[real] if isinstance(v, np.ndarray) and v.ndim == 2 and v.shape[0] == M else v)
                      for k, v in res.items()}
-            assert_parity(res_r, out["codes"][real], out["scales"][real], label + " rows 8+")
+            assert_parity(res_r, out["codes"][real], out["scales"][real], label + " rows 8+",
+                          macro_gpu=out["macro"][real])
 
 
 @pytest.mark.parametrize("b,kernel", [(1, 1), (32, 1), (128, 1), (32, 2), (64, 2), (128, 2)],
@@ -91,7 +92,7 @@ def test_mbs_with_signs(F, b, kernel):
     F.fp4q_plan_set_signs(plan, md, K)
     out = gu.run_rotate_quantize_mbs(F, plan, x)
     res = o.rotate_quantize_mbs(x, 32, b, o.SCALE_FLOOR_OCP, signs=o.sign_vector(mask, K))
-    assert_parity(res, out["codes"], out["scales"], "mbs signed")
+    assert_parity(res, out["codes"], out["scales"], "mbs signed", macro_gpu=out["macro"])
     check_macro(res, out, "mbs signed")
 
 

@@ -16,7 +16,7 @@ import test_oracle_pins as pins
 
 def patch(monkeypatch, name, fn):
     monkeypatch.setattr(core, name, fn)
-    monkeypatch.setattr(o, name, fn)
+    monkeypatch.setattr(o, name, fn, raising=False)
 
 
 def fails(fn, *args):
@@ -330,3 +330,116 @@ def test_gemm_pins_catch_planted_mistake(monkeypatch, fn, catchers):
     patch(monkeypatch, "gemm_fp4", fn)
     for catcher in catchers:
         assert fails(catcher), f"pin missed {fn.__name__}"
+
+
+# ---- the flagged set F of the parity rule (pins in test_oracle_flags.py)
+
+import test_oracle_flags as fpins  # noqa: E402
+
+_orig_bd = core.boundary_distance
+_orig_dsp = core._dist_scaled_power
+_orig_mmd = core.mbs_macro_distance
+
+
+def bd_widened(res):
+    """A window three times too wide (3e-5 instead of 1e-5)."""
+    el, gr = _orig_bd(res)
+    return el / 3.0, gr / 3.0
+
+
+def dsp_shifted(A, base):
+    """Group boundaries shifted by 1e-5 relative (the window centred off the boundary)."""
+    return _orig_dsp(np.asarray(A, np.float64) / (1.0 + 1e-5), base)
+
+
+def dsp_base_ignored(A, base):
+    """Every rule measured against powers of two (the floor rule's boundary)."""
+    return _orig_dsp(A, 1.0)
+
+
+def bd_nv_values_not_midpoints(res):
+    """NV: distance to the E4M3 values instead of the midpoints between them."""
+    el, gr = _orig_bd(res)
+    if res["fmt"] != o.NVFP4:
+        return el, gr
+    y64 = res["y64"]
+    M, K = y64.shape
+    A = np.abs(y64.reshape(M, K // 16, 16)).max(axis=2)
+    s_b = A / (6.0 * np.float64(res["tensor_scale"]))
+    T = core.e4m3_table()[1:]
+    d = np.min(np.abs(s_b[..., None] - T) / T, axis=-1)
+    return el, d
+
+
+def bd_nv_tensor_scale_ignored(res):
+    if res["fmt"] != o.NVFP4:
+        return _orig_bd(res)
+    return _orig_bd(dict(res, tensor_scale=np.float32(1.0)))
+
+
+def bd_elements_not_divided(res):
+    """Element distances of y itself, not of y / S."""
+    return _orig_bd(dict(res, S64=np.ones_like(res["S64"])))[0], _orig_bd(res)[1]
+
+
+def mmd_unscaled(res):
+    """The macro distance in units of 256 f (the window 256 times too wide)."""
+    return _orig_mmd(res) * 256.0 / 65536.0
+
+
+FLAG_MUTATIONS = [
+    ("boundary_distance", bd_widened,
+     [(fpins.test_element_flags_at_every_midpoint, 1.0), (fpins.test_group_flags_floor, 0)]),
+    ("_dist_scaled_power", dsp_shifted,
+     [(fpins.test_group_flags_floor, 3), (fpins.test_group_flags_ceil, -1), (fpins.test_group_flags_oas, 0)]),
+    ("_dist_scaled_power", dsp_base_ignored,
+     [(fpins.test_group_flags_ceil, 0), (fpins.test_group_flags_oas, 3)]),
+    ("boundary_distance", bd_nv_values_not_midpoints,
+     [(fpins.test_nv_group_flags_at_e4m3_midpoints, 1.0)]),
+    ("boundary_distance", bd_nv_tensor_scale_ignored,
+     [(fpins.test_nv_group_flags_at_e4m3_midpoints, 0.5), (fpins.test_nv_group_flags_use_the_tensor_scale,)]),
+    ("boundary_distance", bd_elements_not_divided,
+     [(fpins.test_element_flags_at_every_midpoint, 0.125), (fpins.test_element_flags_use_the_group_divisor,)]),
+    ("mbs_macro_distance", mmd_unscaled,
+     [(fpins.test_mbs_macro_flags,)]),
+]
+
+
+@pytest.mark.parametrize("name,fn,catchers", FLAG_MUTATIONS, ids=[m[1].__name__ for m in FLAG_MUTATIONS])
+def test_flag_pins_catch_planted_mistake(monkeypatch, name, fn, catchers):
+    patch(monkeypatch, name, fn)
+    for catcher in catchers:
+        assert fails(catcher[0], *catcher[1:]), f"{catcher[0].__name__} missed {fn.__name__}"
+
+
+@pytest.mark.parametrize("shift", ["dropped", "shifted"])
+def test_flag_pins_catch_wrong_midpoints(monkeypatch, shift):
+    """A midpoint left out (5.0), or every element window centred 1e-5 off its midpoint."""
+    mids = (0.25, 0.75, 1.25, 1.75, 2.5, 3.5) if shift == "dropped" else \
+        tuple(m * (1 + 1e-5) for m in core.E2M1_MIDPOINTS)
+    monkeypatch.setattr(core, "E2M1_MIDPOINTS", mids)
+    assert fails(fpins.test_element_flags_at_every_midpoint, 1.0)
+
+
+def test_flag_pins_catch_a_zero_sign_forgiven_everywhere(monkeypatch):
+    """The sign of a zero code forgiven whatever the exact rotated value is."""
+    from oracle import parity
+    monkeypatch.setattr(parity, "small_zero", lambda res, tol=1e-5: np.ones(res["y64"].shape, bool))
+    assert fails(fpins.test_compare_forgives_a_zero_sign_only_near_zero)
+
+
+def test_flag_pins_catch_group_flags_forgiving_agreeing_groups(monkeypatch):
+    """An element mismatch forgiven by its group's flag although both sides chose the same scale."""
+    from oracle import parity
+    orig = parity.compare
+
+    def lax(res, codes_gpu, scales_gpu, tol=1e-5, label="", macro_gpu=None):
+        r = orig(res, codes_gpu, scales_gpu, tol, label, macro_gpu)
+        _, gr = core.flags(res, tol)
+        qo, qg = core.unpack_nibbles(res["codes"]), core.unpack_nibbles(np.asarray(codes_gpu, np.uint8))
+        in_flagged = ((qo != qg) & np.repeat(gr, res["group"], axis=1)).sum()
+        r.unflagged_code_mismatch = max(0, r.unflagged_code_mismatch - int(in_flagged))
+        return r
+
+    monkeypatch.setattr(parity, "compare", lax)
+    assert fails(fpins.test_compare_judges_codes_in_an_agreeing_group_on_their_own)

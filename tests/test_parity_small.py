@@ -7,7 +7,7 @@ import pytest
 
 import oracle as o
 from microscaling_fp4_quantization_b200 import workloads as W
-from parity import assert_parity, rotated_value_error
+from oracle.parity import assert_parity, rotated_value_error
 
 pytestmark = pytest.mark.gpu
 
@@ -136,6 +136,37 @@ def test_amax_entry_point(F, b):
         ref = o.nv_tensor_scale(o.rotated_amax(x, b))
         assert abs(float(ours) - float(ref)) <= 2.5e-7 * float(ref), (M, K, ours, ref)
     assert gu.run_amax(F, plan, np.zeros((4, 128), np.uint16)) == np.float32(1.0)
+
+
+def exact_sum_input(M, K, seed):
+    """Rows of small integers times a power of two per row: every block sum of up to 128 of
+    them is an integer below 2^14 times that power of two, exact in fp32, so the kernel's
+    butterfly sums equal the exact sums and its rotated values RN(s / sqrt(b)) equal the
+    oracle's fp64 product rounded once."""
+    rng = np.random.default_rng(seed)
+    x = rng.integers(-64, 65, (M, K)).astype(np.float32)
+    x *= np.ldexp(1.0, rng.integers(-30, 30, (M, 1))).astype(np.float32)
+    return W.f32_to_bf16_bits(x)
+
+
+@pytest.mark.parametrize("b", BLOCKS)
+def test_amax_equals_the_definition_on_exact_sums(F, b):
+    """s_g = fp32(A_t / 2688) with A_t the largest fp32 rotated value: bit for bit, for every
+    block size (1 / sqrt(b) irrational for b = 2, 8, 32, 128), through fp4q_amax and through a
+    DYNAMIC plan's own amax pass, on both kernels."""
+    import gpu_util as gu
+    plan = F.fp4q_plan_create(o.NVFP4, 16, b, o.SCALE_NV_STATIC)
+    for i, (M, K) in enumerate([(1, 128), (300, 1024), (2048, 4096)]):
+        x = exact_sum_input(M, K, seed=31 * b + i)
+        ref = o.nv_tensor_scale(o.rotated_amax(x, b))
+        assert gu.run_amax(F, plan, x) == ref, (b, M, K)
+        res = o.rotate_quantize(x, o.NVFP4, 16, b, o.SCALE_NV_DYNAMIC)
+        for kernel in (1, 2) if b >= 16 else (1,):
+            dyn = F.fp4q_plan_create(o.NVFP4, 16, b, o.SCALE_NV_DYNAMIC)
+            F.fp4q_plan_set_kernel(dyn, kernel)
+            out = gu.run_rotate_quantize(F, dyn, x)
+            assert out["tensor_scale"] == ref, (b, M, K, kernel)
+            assert_parity(res, out["codes"], out["scales"], f"nv-b{b} exact sums {M}x{K} dynamic kernel {kernel}")
 
 
 def test_empty_input_is_a_no_op(F):

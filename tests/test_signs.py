@@ -13,7 +13,7 @@ import torch
 
 import oracle as o
 from microscaling_fp4_quantization_b200 import workloads as W
-from parity import assert_parity, rotated_value_error
+from oracle.parity import assert_parity, rotated_value_error
 from test_parity_small import COMBOS, combo_id, make_input
 
 pytestmark = pytest.mark.gpu
@@ -147,3 +147,34 @@ def test_signed_rows_longer_than_the_staged_mask(F, combo, kernel):
     res = o.rotate_quantize(x, fmt, g, b, rule, tensor_scale=s_g, signs=s)
     out = gu.run_rotate_quantize(F, plan, x, tensor_scale=s_g)
     assert_parity(res, out["codes"], out["scales"], f"{combo_id(combo)} K={K} signed")
+
+
+@pytest.mark.parametrize("b,kernel", [(16, 1), (128, 1), (16, 2), (128, 2)],
+                         ids=["b16-bf", "b128-bf", "b16-tc", "b128-tc"])
+def test_unstaged_mask_on_every_signed_path(F, b, kernel):
+    """K = 135168 (a 16.5 KB mask, read in place by every kernel): the NV amax pass (fp4q_amax
+    and a DYNAMIC plan), the error pass and dequantize with rotate-back all switch between a
+    staged and an in-place mask by the same rule as rotate + quantize."""
+    import gpu_util as gu
+    from test_quant_error import assert_energies, run_qe
+    M, K = 3, 135168
+    x = make_input(M, K, seed=4343 + b, adversarial=False)
+    plan, s = signed_plan(F, (o.NVFP4, 16, b, o.SCALE_NV_DYNAMIC), K, seed=78)
+    F.fp4q_plan_set_kernel(plan, kernel)
+    ref_sg = o.nv_tensor_scale(o.rotated_amax(x, b, signs=s))
+    res = o.rotate_quantize(x, o.NVFP4, 16, b, o.SCALE_NV_DYNAMIC, signs=s)
+    out = gu.run_rotate_quantize(F, plan, x)
+    assert abs(float(out["tensor_scale"]) - float(ref_sg)) <= 2.5e-7 * float(ref_sg)
+    assert_parity(res, out["codes"], out["scales"], f"nv-b{b} K={K} signed dynamic kernel {kernel}")
+    assert abs(float(gu.run_amax(F, plan, x)) - float(ref_sg)) <= 2.5e-7 * float(ref_sg)
+    assert_energies(run_qe(F, plan, x), o.quant_error(x, o.NVFP4, 16, b, o.SCALE_NV_DYNAMIC, signs=s),
+                    f"nv-b{b} K={K} signed error pass")
+    back = gu.run_dequantize(F, plan, out["codes"], out["scales"], out["tensor_scale"], unrotate=True)
+    ref_back = o.dequantize(out["codes"], out["scales"], o.NVFP4, 16, b, tensor_scale=out["tensor_scale"],
+                            unrotate_back=True, signs=s)
+    assert np.max(np.abs(back - ref_back)) <= 1e-6 * np.abs(ref_back).max()
+    mx, smx = signed_plan(F, (o.MXFP4, 32, b, o.SCALE_OAS), K, seed=79)
+    if b >= 32 or kernel == 1:
+        F.fp4q_plan_set_kernel(mx, kernel)
+        assert_energies(run_qe(F, mx, x), o.quant_error(x, o.MXFP4, 32, b, o.SCALE_OAS, signs=smx),
+                        f"mx-b{b} K={K} signed error pass")
