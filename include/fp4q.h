@@ -105,8 +105,17 @@ typedef struct fp4q_plan_s* fp4q_plan;
 
 /* Create a plan.  format: fp4q_format; group: 32 (MXFP4) or 16 (NVFP4); hadamard_block:
  * 1, 2, 4, ..., 128 (1 = no rotation); scale_rule: an fp4q_scale_rule valid for the
- * format.  Writes the plan to *out.  FP4Q_SCALE_NV_DYNAMIC plans allocate their partial-
- * maximum array on the current CUDA device, which every later call must also use. */
+ * format.  Writes the plan to *out.
+ *
+ * Device binding.  A plan made while a CUDA device is current belongs to the CUDA context
+ * current at creation (the device's primary context, unless the caller made another one
+ * current through the driver API): its scratch arrays (see Ownership) are allocated there.
+ * fp4q_rotate_quantize(_dump, _mbs), fp4q_amax, fp4q_quant_error and fp4q_dequantize(_mbs)
+ * must then be called with that context current; with another device or another context
+ * current they return FP4Q_ERR_ARG before launching anything (and before their shape and
+ * pointer checks), and fp4q_last_cuda_error() says so.  After cudaDeviceReset a plan made before it
+ * is unusable: destroy it and make a new one.  A plan made on a machine without a CUDA
+ * device owns no device memory and is bound to none. */
 fp4q_status fp4q_plan_create(fp4q_plan* out, int format, int group, int hadamard_block,
                              int scale_rule);
 
@@ -248,9 +257,11 @@ fp4q_status fp4q_gemm(int format, const void* a_codes, const void* a_scales, con
  * nothing carries over from earlier calls; calls that overlap on the GPU (other streams, other
  * host threads) share the array and race.
  *
- * Allocation: none — no cudaMalloc, cudaFree or allocating library routine.  The first call
- * on each device does a one-time set-up there (it looks up the array's device address and
- * configures the kernels); make that first call outside any stream capture. */
+ * Allocation: none — no cudaMalloc, cudaFree or allocating library routine.  Every call looks
+ * up the array's device address in the context current at the time (a host-side lookup), so
+ * it stays right after cudaDeviceReset or under a context the caller made current.  The first
+ * call in each context also configures the kernels there (shared-memory attributes); make
+ * that first call outside any stream capture. */
 fp4q_status fp4q_rotate_quantize_nvfp4_dynamic_noalloc(const void* x_bf16, int64_t M, int64_t K,
                                                        int hadamard_block, void* codes_out,
                                                        void* scales_out, float* tensor_scale_out,

@@ -18,8 +18,26 @@ namespace host {
 
 namespace {
 thread_local char g_last_cuda_error[kLastErrorBytes] = "";
+std::mutex g_ctx_mu;
+// kernel, context, the dynamic shared memory occupancy is computed for, threads per CTA
+struct InfoKey {
+  const void* kernel;
+  uint64_t ctx;
+  int smem, threads;
+  bool operator==(const InfoKey& o) const {
+    return kernel == o.kernel && ctx == o.ctx && smem == o.smem && threads == o.threads;
+  }
+};
+struct InfoKeyHash {
+  size_t operator()(const InfoKey& k) const {
+    uint64_t h = reinterpret_cast<uint64_t>(k.kernel) * 0x9E3779B97F4A7C15ull;
+    h ^= k.ctx + 0x632BE59BD9B4E019ull + (h << 6) + (h >> 2);
+    h ^= (static_cast<uint64_t>(static_cast<uint32_t>(k.smem)) << 20) ^ static_cast<uint64_t>(k.threads);
+    return static_cast<size_t>(h);
+  }
+};
 std::mutex g_info_mu;
-std::unordered_map<uint64_t, KernelInfo> g_info;
+std::unordered_map<InfoKey, KernelInfo, InfoKeyHash> g_info;
 std::mutex g_encode_mu;
 EncodeTiledFn g_encode = nullptr;
 }  // namespace
@@ -32,11 +50,59 @@ fp4q_status cuda_fail(cudaError_t e, const char* what) {
   return FP4Q_ERR_CUDA;
 }
 
+// Identity of the CUDA context current on this thread (0 when none is current yet).  Kernel
+// attributes and occupancy belong to a context: after cudaDeviceReset, or under a context the
+// caller made current through the driver API, the module is loaded afresh, so the cache below
+// is keyed on this identity rather than on the device index.
+fp4q_status current_context_id(uint64_t* out) {
+  typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+  typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_ctx_mu);
+    if (!get_current || !get_id) {
+      void* f1 = nullptr;
+      void* f2 = nullptr;
+      cudaDriverEntryPointQueryResult q1, q2;
+      cudaError_t e = cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1);
+      if (e == cudaSuccess) e = cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetDriverEntryPoint(cuCtxGetCurrent / cuCtxGetId)");
+      if (q1 != cudaDriverEntryPointSuccess || q2 != cudaDriverEntryPointSuccess || !f1 || !f2)
+        return cuda_fail(cudaErrorNotSupported, "cuCtxGetCurrent / cuCtxGetId");
+      get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+      get_id = reinterpret_cast<CtxGetIdFn>(f2);
+    }
+  }
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return cuda_fail(cudaErrorDeviceUninitialized, "cuCtxGetCurrent");
+  unsigned long long id = 0;
+  if (ctx && get_id(ctx, &id) != CUDA_SUCCESS) return cuda_fail(cudaErrorDeviceUninitialized, "cuCtxGetId");
+  *out = ctx ? static_cast<uint64_t>(id) + 1 : 0;
+  return FP4Q_OK;
+}
+
+fp4q_status bound_context_id(uint64_t* out) {
+  fp4q_status st = current_context_id(out);
+  if (st != FP4Q_OK || *out != 0) return st;
+  // nothing is current on this thread yet: bind the current device's primary context, as the
+  // runtime's first call on this thread that needs a context would (it displaces nothing)
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaSetDevice(dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+  return current_context_id(out);
+}
+
 fp4q_status kernel_info_impl(const void* kernel, int smem_bytes, int threads, KernelInfo* out, int max_smem_bytes) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  const uint64_t key = (reinterpret_cast<uint64_t>(kernel) << 8) ^ static_cast<uint64_t>(dev);
+  const int attr_smem = max_smem_bytes > smem_bytes ? max_smem_bytes : smem_bytes;
+  uint64_t ctx = 0;
+  fp4q_status st = bound_context_id(&ctx);
+  if (st != FP4Q_OK) return st;
+  const InfoKey key{kernel, ctx, smem_bytes, threads};
   std::lock_guard<std::mutex> lk(g_info_mu);
   auto it = g_info.find(key);
   if (it != g_info.end()) {
@@ -46,8 +112,7 @@ fp4q_status kernel_info_impl(const void* kernel, int smem_bytes, int threads, Ke
   KernelInfo ki;
   e = cudaDeviceGetAttribute(&ki.sm_count, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           max_smem_bytes > smem_bytes ? max_smem_bytes : smem_bytes);
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, attr_smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
   // all of the unified L1 / shared storage as shared memory: these kernels stage through it
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
@@ -84,6 +149,27 @@ constexpr uint32_t kPlanMagic = 0xF4F4A11Cu;
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 bool valid_plan(fp4q_plan p) { return p != nullptr && p->magic == kPlanMagic; }
+
+// A plan's device memory (the partial maxima, the error pass's scratch) was allocated in the
+// CUDA context current when the plan was made (the device's primary context, unless the
+// caller made another one current), so every call that launches must be made with that
+// context current: another device, or another context on the same device, cannot reach it.
+// Checked before anything is launched.
+fp4q_status check_device(fp4q_plan p, const char* who) {
+  if (p->device < 0) return FP4Q_OK;   // made without a device: it owns no device memory
+  uint64_t ctx = 0;
+  fp4q_status st = bound_context_id(&ctx);
+  if (st != FP4Q_OK) return st;
+  if (ctx != p->context) {
+    int dev = -1;
+    (void)cudaGetDevice(&dev);
+    std::snprintf(last_error_buffer(), kLastErrorBytes,
+                  "%s: the plan belongs to a CUDA context on device %d, but another context (device %d) is current",
+                  who, p->device, dev);
+    return FP4Q_ERR_ARG;
+  }
+  return FP4Q_OK;
+}
 
 // Whether the tensor-core kernel serves this plan.  AUTO takes it for tensors of at least
 // kMmaMinElems elements: below that its fixed start-up (TMEM allocation, H_b, filling a
@@ -133,7 +219,9 @@ fp4q_status rotate_quantize_impl(fp4q_plan p, const void* x, int64_t M, int64_t 
   if (!valid_plan(p)) return FP4Q_ERR_ARG;
   // an MBS plan also stores macro-scale bytes: only fp4q_rotate_quantize_mbs (macro != null) serves it
   if ((p->format == FP4Q_MXFP4_MBS) != (macro != nullptr)) return FP4Q_ERR_UNSUPPORTED;
-  fp4q_status st = check_shape(p, M, K);
+  fp4q_status st = check_device(p, "fp4q_rotate_quantize");
+  if (st != FP4Q_OK) return st;
+  st = check_shape(p, M, K);
   if (st != FP4Q_OK) return st;
   if (M * K == 0) return FP4Q_OK;
   if (!x || !codes || !scales || (dump && !y_out)) return FP4Q_ERR_ARG;
@@ -293,24 +381,14 @@ fp4q_status qe_grid(int format, int block, int rule, int* n) {
 
 // ---- no-allocation NVFP4 dynamic path: partial maxima in a fixed device array
 
-constexpr int kNoAllocMaxDevices = 64;
-std::mutex g_noalloc_mu;
-float* g_noalloc_ptr[kNoAllocMaxDevices] = {};
-
-// Device address of the no-allocation scratch on the current device, looked up once per device.
+// Device address of the no-allocation scratch in the context current now.  Looked up on every
+// call (a host-side lookup): an address kept from an earlier call would be stale after
+// cudaDeviceReset, or under another context the caller made current.
 fp4q_status noalloc_scratch(float** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= kNoAllocMaxDevices) return FP4Q_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    float* ptr = nullptr;
-    fp4q_status st = noalloc_partials_symbol(&ptr);
-    if (st != FP4Q_OK) return st;
-    g_noalloc_ptr[dev] = ptr;
-  }
-  *out = g_noalloc_ptr[dev];
+  float* ptr = nullptr;
+  fp4q_status st = noalloc_partials_symbol(&ptr);
+  if (st != FP4Q_OK) return st;
+  *out = ptr;
   return FP4Q_OK;
 }
 
@@ -395,6 +473,7 @@ fp4q_status fp4q_plan_create(fp4q_plan* out, int format, int group, int hadamard
   p->unit = group > hadamard_block ? group : hadamard_block;
   if (format == FP4Q_MXFP4_MBS) p->unit = 128;   // one macro block per unit (b <= 128)
   p->device = -1;
+  p->context = 0;
   p->partials = nullptr;
   p->n_partials = 0;
   p->kernel = FP4Q_KERNEL_AUTO;
@@ -429,8 +508,10 @@ fp4q_status fp4q_plan_create(fp4q_plan* out, int format, int group, int hadamard
     if (e == cudaSuccess) e = cudaMemset(p->err_partials, 0, bytes);
     if (e != cudaSuccess) st = cuda_fail(e, "cudaMalloc error partials");
   }
+  if (st == FP4Q_OK) st = bound_context_id(&p->context);   // the context the allocations were made in
   if (st != FP4Q_OK) {
     if (p->partials) cudaFree(p->partials);
+    if (p->err_partials) cudaFree(p->err_partials);
     p->magic = 0;
     delete p;
     return st;
@@ -501,7 +582,9 @@ fp4q_status fp4q_amax(fp4q_plan plan, const void* x_bf16, int64_t M, int64_t K, 
                       void* stream) {
   if (!valid_plan(plan)) return FP4Q_ERR_ARG;
   if (plan->format != FP4Q_NVFP4) return FP4Q_ERR_UNSUPPORTED;
-  fp4q_status st = check_shape(plan, M, K);
+  fp4q_status st = check_device(plan, "fp4q_amax");
+  if (st != FP4Q_OK) return st;
+  st = check_shape(plan, M, K);
   if (st != FP4Q_OK) return st;
   if (!tensor_scale_out) return FP4Q_ERR_ARG;
   if (M * K > 0 && !x_bf16) return FP4Q_ERR_ARG;
@@ -515,7 +598,9 @@ fp4q_status fp4q_amax(fp4q_plan plan, const void* x_bf16, int64_t M, int64_t K, 
 fp4q_status fp4q_quant_error(fp4q_plan plan, const void* x_bf16, int64_t M, int64_t K, float* tensor_scale,
                              double* out, void* stream) {
   if (!valid_plan(plan)) return FP4Q_ERR_ARG;
-  fp4q_status st = check_shape(plan, M, K);
+  fp4q_status st = check_device(plan, "fp4q_quant_error");
+  if (st != FP4Q_OK) return st;
+  st = check_shape(plan, M, K);
   if (st != FP4Q_OK) return st;
   if (!out) return FP4Q_ERR_ARG;
   if (plan->format == FP4Q_NVFP4 && !tensor_scale) return FP4Q_ERR_ARG;
@@ -594,7 +679,9 @@ namespace {
 fp4q_status dequantize_impl(fp4q_plan plan, const void* codes, const void* scales, const void* macro,
                             const float* tensor_scale, int64_t M, int64_t K, int unrotate, float* out_f32,
                             void* stream) {
-  fp4q_status st = check_shape(plan, M, K);
+  fp4q_status st = check_device(plan, "fp4q_dequantize");
+  if (st != FP4Q_OK) return st;
+  st = check_shape(plan, M, K);
   if (st != FP4Q_OK) return st;
   if (M * K == 0) return FP4Q_OK;
   if (!codes || !scales || !out_f32 || (plan->format == FP4Q_NVFP4 && !tensor_scale)) return FP4Q_ERR_ARG;

@@ -21,6 +21,7 @@ struct fp4q_plan_s {
   int format, group, block, rule;
   int unit;        // elements per butterfly unit: max(block, group), 128 for MBS
   int device;
+  uint64_t context; // identity of the CUDA context its device arrays were allocated in (0: none)
   float* partials; // NV plans: per-CTA rotated amaxima (device)
   int n_partials;
   int kernel;      // fp4q_kernel
@@ -34,21 +35,25 @@ struct fp4q_plan_s {
 namespace fp4q {
 namespace host {
 
+// Identity of the CUDA context current on the calling thread (cuCtxGetId), binding the
+// current device's primary context first when none is current.
+fp4q_status bound_context_id(uint64_t* out);
+
 // Records the CUDA error message (fp4q_last_cuda_error) and returns FP4Q_ERR_CUDA.
 fp4q_status cuda_fail(cudaError_t e, const char* what);
 // The thread's message buffer behind fp4q_last_cuda_error.
 char* last_error_buffer();
 constexpr int kLastErrorBytes = 512;
 
-// Per (kernel, device) one-time set-up: opt in to the dynamic shared memory the kernel
-// needs and record how many CTAs fit on one SM.
+// Per (kernel, CUDA context, launch size) one-time set-up: opt in to the dynamic shared memory
+// the kernel needs and record how many CTAs of that size fit on one SM.
 struct KernelInfo {
   int ctas_per_sm = 0;
   int sm_count = 0;
 };
-// Occupancy is computed for smem_bytes; the kernel may be launched with up to max_smem_bytes
-// (when larger) of dynamic shared memory.  The first call for a kernel sets both, so every
-// call for one kernel passes the same sizes.
+// Occupancy is computed for smem_bytes, the dynamic shared memory of the launch; the kernel
+// may be launched with up to max_smem_bytes (when larger), which every call for one kernel
+// passes alike.  Results are cached per (kernel, context, smem_bytes, threads).
 fp4q_status kernel_info_impl(const void* kernel, int smem_bytes, int threads, KernelInfo* out, int max_smem_bytes);
 
 template <class K>
@@ -57,10 +62,12 @@ fp4q_status kernel_info(K kernel, int smem_bytes, int threads, KernelInfo* out, 
 }
 
 // The butterfly kernels (rotate + quantize, error pass, amax) may stage a sign mask of up to
-// kSignSmemMaxWords words behind their stages.
+// kSignSmemMaxWords words behind their stages; occupancy is that of a launch staging
+// smem_words of them (0: an unsigned launch, or a mask read in place).
 template <class Cfg, class K>
-fp4q_status butterfly_kernel_info(K kernel, KernelInfo* out) {
-  return kernel_info(kernel, Cfg::kSmemBytes, Cfg::kThreads, out, Cfg::kSmemBytes + 4 * kSignSmemMaxWords);
+fp4q_status butterfly_kernel_info(K kernel, KernelInfo* out, int smem_words = 0) {
+  return kernel_info(kernel, Cfg::kSmemBytes + 4 * smem_words, Cfg::kThreads, out,
+                     Cfg::kSmemBytes + 4 * kSignSmemMaxWords);
 }
 
 // Launch with programmatic stream serialization, so the kernel's start overlaps the tail of

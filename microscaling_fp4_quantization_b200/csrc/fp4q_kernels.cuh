@@ -899,7 +899,8 @@ static __global__ void quant_error_empty_kernel(const double* __restrict__ parti
   qe_final_sum(partials, 0, out);
 }
 
-// Rotated amax: every CTA writes max |fl(y)| over its warps' ranges to partials[blockIdx.x].
+// Rotated amax: every CTA writes max |fl(y)| over its warps' ranges to partials[blockIdx.x], with
+// fl(y) = RN(s / sqrt(b)) of the raw butterfly sum s, the value the quantizer takes its decisions on.
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::kThreads) rotated_amax_kernel(const uint16_t* __restrict__ x, int64_t n_units,
                                                                      float* __restrict__ partials, ChannelSigns signs) {
@@ -924,7 +925,9 @@ __global__ void __launch_bounds__(Cfg::kThreads) rotated_amax_kernel(const uint1
     float r = 0.0f;
 #pragma unroll
     for (int i = 0; i < Cfg::kWarps; ++i) r = fmaxf(r, s_max[i]);
-    partials[blockIdx.x] = r * Cfg::kC;
+    // RN(r / sqrt(b)): the correctly rounded scaling is monotone, so this is the maximum of the
+    // elements' own fp32 values RN(sum / sqrt(b)), as the quantizer's group maxima are
+    partials[blockIdx.x] = scale_by_inv_sqrt<Cfg::kBlock>(r);
   }
 }
 

@@ -16,7 +16,7 @@ fp4q_status launch_rq(RQArgs a, int64_t n_elems, cudaStream_t stream, int64_t K)
   a.signs = channel_signs<Cfg>(a.signs.mask, K);
   auto kernel = rotate_quantize_kernel<Cfg>;
   KernelInfo ki;
-  fp4q_status st = butterfly_kernel_info<Cfg>(kernel, &ki);
+  fp4q_status st = butterfly_kernel_info<Cfg>(kernel, &ki, a.signs.smem_words);
   if (st != FP4Q_OK) return st;
   const int64_t warps_needed = (a.n_units + Cfg::kUnitsPerStage - 1) / Cfg::kUnitsPerStage;
   int64_t ctas = (warps_needed + Cfg::kWarps - 1) / Cfg::kWarps;
@@ -119,7 +119,7 @@ fp4q_status launch_qe(fp4q_plan p, QEArgs a, int64_t n_elems, double* out, cudaS
   a.signs = channel_signs<Cfg>(p->signs, p->signs_K);
   auto kernel = quant_error_kernel<Cfg>;
   KernelInfo ki;
-  fp4q_status st = butterfly_kernel_info<Cfg>(kernel, &ki);
+  fp4q_status st = butterfly_kernel_info<Cfg>(kernel, &ki, a.signs.smem_words);
   if (st != FP4Q_OK) return st;
   const int64_t warps_needed = (a.n_units + Cfg::kUnitsPerStage - 1) / Cfg::kUnitsPerStage;
   int64_t ctas = (warps_needed + Cfg::kWarps - 1) / Cfg::kWarps;
@@ -144,6 +144,11 @@ fp4q_status amax_wave(int* n) {
 template <class Cfg>
 fp4q_status launch_amax_cfg(const uint16_t* x, int64_t n_elems, float* partials, int n_partials, ChannelSigns sg,
                             cudaStream_t stream, bool pdl) {
+  // the attribute for the largest (signed) launch on the current context, as the other
+  // butterfly launchers set it
+  KernelInfo ki;
+  fp4q_status st = butterfly_kernel_info<Cfg>(rotated_amax_kernel<Cfg>, &ki, sg.smem_words);
+  if (st != FP4Q_OK) return st;
   cudaError_t e;
   const size_t smem = Cfg::kSmemBytes + 4 * static_cast<size_t>(sg.smem_words);
   if (pdl) {
