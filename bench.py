@@ -203,6 +203,24 @@ def time_graph_steps(torch, launch, n_buf: int, steps: int, warmup: int, stream)
     return g, g_rem, reps
 
 
+def time_replays(torch, g, g_rem, reps, stream) -> float:
+    """Device milliseconds of `reps` replays of graph g (then g_rem once), between two CUDA
+    events on `stream`.  One untimed replay of g is queued first: the host then submits the
+    timed replays while the device is still busy, so the region starts with work queued
+    behind the first event and no host submission gap lands inside it."""
+    with torch.cuda.stream(stream):
+        g.replay()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        a1.record(stream)
+    torch.cuda.synchronize()
+    return a0.elapsed_time(a1)
+
+
 def run_gpu(args):
     import torch
     from microscaling_fp4_quantization_b200 import fp4q as F
@@ -258,21 +276,12 @@ def run_gpu(args):
         import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(reps):
-            g.replay()
-        if g_rem is not None:
-            g_rem.replay()
-        e1.record(stream)
-    torch.cuda.synchronize()
+    ms_local = time_replays(torch, g, g_rem, reps, stream)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
     sampler.stop()
-    ms = max_over_ranks(torch, e0.elapsed_time(e1), world, dev)
+    ms = max_over_ranks(torch, ms_local, world, dev)
     ms_step = ms / args.steps
     value = whole_job_gbs(world, bytes_call, args.steps, ms)
     kernel_us = ms_step * 1e3
@@ -293,15 +302,9 @@ def run_gpu(args):
             steps2 = max(50, min(args.steps, 400))
             with torch.cuda.stream(stream):
                 g2, g2r, reps2 = time_graph_steps(torch, fn, n_buf, steps2, 3, stream)
-                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a0.record(stream)
-                for _ in range(reps2):
-                    g2.replay()
-                if g2r is not None:
-                    g2r.replay()
-                a1.record(stream)
+                ms_ = time_replays(torch, g2, g2r, reps2, stream)
             torch.cuda.synchronize()
-            us = a0.elapsed_time(a1) * 1e3 / steps2
+            us = ms_ * 1e3 / steps2
             extra[name] = {"us_per_call": round(us, 3), "GBps_algorithmic": round(nbytes / us / 1e3, 1),
                            "bytes_per_call": nbytes}
         extra["dynamic_mode"]["note"] = "reads X twice (amax pass, then quantize); bytes are the algorithmic ones"
@@ -309,7 +312,7 @@ def run_gpu(args):
     # context for the roofline at this size: a plain device copy that reads and writes the same
     # total bytes (half each way), timed the same way over as many rotating buffers
     if rank == 0:
-        extra["copy_same_bytes"] = time_copy(torch, bytes_call, n_buf, stream, peak)
+        extra["copy_same_bytes"] = time_copy(torch, bytes_call, n_buf, stream, peak, steps=args.steps)
 
     # the randomised rotation (per-channel random signs) on the same workload, on the kernel the plan picks
     if rank == 0:
@@ -373,6 +376,17 @@ def run_gpu(args):
                "h2d_bytes_per_step": int(x_host.numel() * 2),
                "d2h_bytes_per_step": int(codes_h[0].numel() + scales_h[0].numel()), "steps": n_e2e,
                "pipelined": f"{nb} buffer sets, copy-in / quantize / copy-out on three streams"}
+
+    # the other target workloads, each timed like the headline (same step count, a lead-in
+    # replay, clocks sampled through its region), on the kernel AUTO picks (rank 0)
+    targets = {}
+    if rank == 0 and not args.headline_only:
+        cache = {}
+        for tw in TARGET_WORKLOADS:
+            if tw.name != w.name:
+                targets[tw.name] = time_target(torch, F, tw, dev, stream, peak, args.steps, cache)
+        del cache
+        torch.cuda.empty_cache()
 
     # the other workloads' throughput, each timed the same way (rank 0, when asked)
     others = {}
@@ -442,6 +456,8 @@ def run_gpu(args):
             "cpu_baseline": cpu,
             "extra": extra,
         }
+        if targets:
+            line["targets"] = targets
         if others:
             line["workloads"] = others
         print(json.dumps(line), flush=True)
@@ -537,16 +553,10 @@ def time_gemm(torch, F, fmt, M, N, K, stream, steps=200):
             gph.replay()
             stream.synchronize()
         sampler.start()
-        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
-        for _ in range(reps):
-            gph.replay()
-        if g_rem is not None:
-            g_rem.replay()
-        a1.record(stream)
+        ms_ = time_replays(torch, gph, g_rem, reps, stream)
     torch.cuda.synchronize()
     sampler.stop()
-    us = a0.elapsed_time(a1) * 1e3 / steps
+    us = ms_ * 1e3 / steps
     tflops = 2.0 * M * N * K / (us * 1e-6) / 1e12
     peak, kind = tensor_peak_fp4()
     peak_s, _ = tensor_peak_fp4(sustained=True)
@@ -571,15 +581,9 @@ def time_copy(torch, nbytes, n_buf, stream, peak, steps=2000):
 
     with torch.cuda.stream(stream):
         g, g_rem, reps = time_graph_steps(torch, launch, n_buf, steps, 3, stream)
-        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
-        for _ in range(reps):
-            g.replay()
-        if g_rem is not None:
-            g_rem.replay()
-        a1.record(stream)
+        ms_ = time_replays(torch, g, g_rem, reps, stream)
     torch.cuda.synchronize()
-    us = a0.elapsed_time(a1) * 1e3 / steps
+    us = ms_ * 1e3 / steps
     gbs = 2 * half / us / 1e3
     del srcs, dsts
     return {"bytes_per_call": 2 * half, "us_per_call": round(us, 3), "GBps": round(gbs, 1),
@@ -596,15 +600,9 @@ def time_plan(torch, F, plan, w, xs, codes, scales, ts, stream, steps):
 
     with torch.cuda.stream(stream):
         g, g_rem, reps = time_graph_steps(torch, launch, len(xs), steps, 3, stream)
-        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
-        for _ in range(reps):
-            g.replay()
-        if g_rem is not None:
-            g_rem.replay()
-        a1.record(stream)
+        ms_ = time_replays(torch, g, g_rem, reps, stream)
     torch.cuda.synchronize()
-    return a0.elapsed_time(a1) * 1e3 / steps
+    return ms_ * 1e3 / steps
 
 
 def time_signed(torch, F, w, xs, codes, scales, ts, stream, peak, steps, kernel="auto"):
@@ -662,15 +660,9 @@ def time_quant_error(torch, F, w, plan, xs, ts, stream, peak, steps):
 
     with torch.cuda.stream(stream):
         g, g_rem, reps = time_graph_steps(torch, launch, len(xs), steps, 3, stream)
-        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
-        for _ in range(reps):
-            g.replay()
-        if g_rem is not None:
-            g_rem.replay()
-        a1.record(stream)
+        ms_ = time_replays(torch, g, g_rem, reps, stream)
     torch.cuda.synchronize()
-    us = a0.elapsed_time(a1) * 1e3 / steps
+    us = ms_ * 1e3 / steps
     launch(0)
     torch.cuda.synchronize()
     sig, err, q = out.tolist()
@@ -704,15 +696,9 @@ def time_mbs(torch, F, w, dev, stream, peak, kernel="auto"):
     steps = 200 if nbytes > 1e8 else 2000
     with torch.cuda.stream(stream):
         g, g_rem, reps = time_graph_steps(torch, launch, n_buf, steps, 5, stream)
-        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
-        for _ in range(reps):
-            g.replay()
-        if g_rem is not None:
-            g_rem.replay()
-        a1.record(stream)
+        ms_ = time_replays(torch, g, g_rem, reps, stream)
     torch.cuda.synchronize()
-    us = a0.elapsed_time(a1) * 1e3 / steps
+    us = ms_ * 1e3 / steps
     gbs = nbytes / us / 1e3
     qe_mbs = time_quant_error(torch, F, w, plan, xs, None, stream, peak, 20)
     plain = F.fp4q_plan_create(w.fmt, w.group, w.block, w.rule)
@@ -726,6 +712,60 @@ def time_mbs(torch, F, w, dev, stream, peak, kernel="auto"):
     del xs, codes, scales, macro
     torch.cuda.empty_cache()
     return out
+
+
+# The workloads the fused kernel is graded on besides the headline (8192 x 8192 MXFP4 b128 under
+# both rules, and the 32768 x 14336 prefill under NVFP4 and MXFP4 b128), then the small one and
+# the decode rows (latency: microseconds per call).
+TARGET_WORKLOADS = (W.MX_8K_FLOOR, W.MX_8K_CEIL, W.PREFILL_NV, W.PREFILL_MX, W.SMALL_MX) + W.DECODE
+
+
+def time_target(torch, F, w, dev, stream, peak, steps, cache):
+    """One target workload on the kernel AUTO picks: `steps` calls over rotating buffers (more
+    than L2 in total, or one buffer larger than L2), replayed from a CUDA graph after a short
+    untimed soak, timed with CUDA events, SM clocks sampled through the timed region.  Inputs
+    with the same seed and shape are generated once (`cache`)."""
+    M, K = w.M, w.K
+    key = (w.seed, M, K)
+    if key not in cache:
+        cache.clear()
+        cache[key] = torch.from_numpy(w.generate().view(np.int16)).view(torch.bfloat16)
+    xh = cache[key]
+    plan = F.fp4q_plan_create(w.fmt, w.group, w.block, w.rule)
+    bytes_call = w.bytes_per_call()
+    n_buf = max(1, math.ceil(3 * L2_BYTES / bytes_call)) if bytes_call < 2 * L2_BYTES else 1
+    n_buf = min(n_buf, 64)
+    xs = [xh.to(dev) for _ in range(n_buf)]
+    codes = [torch.empty((M, K // 2), dtype=torch.uint8, device=dev) for _ in range(n_buf)]
+    scales = [torch.empty((M, K // w.group), dtype=torch.uint8, device=dev) for _ in range(n_buf)]
+    ts = torch.ones(1, dtype=torch.float32, device=dev)
+    nv = w.fmt == W.NVFP4
+    if nv:
+        F.fp4q_amax(plan, xs[0], M, K, ts, stream=torch.cuda.current_stream())
+
+    def launch(i):
+        F.fp4q_rotate_quantize(plan, xs[i], M, K, codes[i], scales[i], ts if nv else None,
+                               stream=torch.cuda.current_stream())
+
+    sampler = ClockSampler(dev.index)
+    with torch.cuda.stream(stream):
+        g, g_rem, reps = time_graph_steps(torch, launch, n_buf, steps, 3, stream)
+        # the samples cover the soak (the same replays) and the timed region
+        sampler.start()
+        t_end = time.time() + 0.2
+        while time.time() < t_end:
+            g.replay()
+            stream.synchronize()
+    ms = time_replays(torch, g, g_rem, reps, stream)
+    sampler.stop()
+    assert F.fp4q_device_status() == F.FP4Q_OK
+    us = ms * 1e3 / steps
+    gbs = bytes_call / us / 1e3
+    del xs, codes, scales, g, g_rem
+    return {"GBps": round(gbs, 1), "pct_of_hbm_peak": round(100 * gbs / peak, 2), "us_per_call": round(us, 3),
+            "elements_per_s": round(M * K / (us * 1e-6), 1), "bytes_per_call": bytes_call, "steps": steps,
+            "buffers": n_buf, "kernel": kernel_name(w, "auto"), "format": "NVFP4" if nv else "MXFP4",
+            "hadamard_block": w.block, "scale_rule": W.RULE_NAMES[w.rule], "clocks": sampler.summary()}
 
 
 def time_other(torch, F, w, dev, stream, peak, kernel="auto"):
@@ -752,15 +792,9 @@ def time_other(torch, F, w, dev, stream, peak, kernel="auto"):
     steps = 200 if bytes_call > 1e8 else 2000
     with torch.cuda.stream(stream):
         g, g_rem, reps = time_graph_steps(torch, launch, n_buf, steps, 5, stream)
-        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
-        for _ in range(reps):
-            g.replay()
-        if g_rem is not None:
-            g_rem.replay()
-        a1.record(stream)
+        ms_ = time_replays(torch, g, g_rem, reps, stream)
     torch.cuda.synchronize()
-    us = a0.elapsed_time(a1) * 1e3 / steps
+    us = ms_ * 1e3 / steps
     gbs = bytes_call / us / 1e3
     out = {"GBps": round(gbs, 1), "pct_of_hbm_peak": round(100 * gbs / peak, 2), "us_per_call": round(us, 3),
            "bytes_per_call": bytes_call, "buffers": n_buf, "kernel": kernel_name(w, kernel)}
@@ -774,20 +808,68 @@ def time_other(torch, F, w, dev, stream, peak, kernel="auto"):
     return out
 
 
-def cpu_baseline(w, args, seconds: float = 10.0):
-    """The oracle, as it stands, on a bounded sample of the workload's rows, on one host
-    thread; GB/s on the sample's algorithmic bytes."""
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine()
+
+
+def _oracle_batch(job):
+    """One batch of the oracle in a pool process (rows of X through rotate_quantize)."""
+    import oracle
+    x, fmt, group, block, rule, ts = job
+    oracle.rotate_quantize(x, fmt, group, block, rule, tensor_scale=ts)
+    return x.shape[0]
+
+
+def oracle_pool(n: int):
+    """A pool of n host processes for the oracle, one BLAS thread each, started with `spawn`
+    (the parent has initialised CUDA; a process forked after that can hang)."""
+    import multiprocessing as mp
+    saved = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+    for k in saved:
+        os.environ[k] = "1"
+    try:
+        return mp.get_context("spawn").Pool(n)
+    finally:
+        for k, v in saved.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+
+
+def oracle_sample(w, rows: int):
+    """The first `rows` rows of the workload and, for NVFP4, the oracle's tensor scale of them."""
+    import oracle
+    x = next(iter(w.row_chunks(chunk_rows=rows)))
+    ts = oracle.nv_tensor_scale(oracle.rotated_amax(x, w.block)) if w.fmt == W.NVFP4 else None
+    return x, ts
+
+
+def cpu_baseline(w, args, seconds: float = 8.0):
+    """The oracle, as it stands, on bounded samples of the workload's rows: once on one host
+    thread, then on every host core (one process per core, each running the oracle on its own
+    batches of rows; rows are independent).  GB/s on the samples' algorithmic bytes.  The
+    line's value is the all-cores figure, with the single-thread one beside it."""
     import oracle
     from threadpoolctl import threadpool_limits
 
     rows_per_batch = max(1, (1 << 20) // w.K)
-    x = None
-    for ch in w.row_chunks(chunk_rows=rows_per_batch):
-        x = ch
-        break
-    ts = None
-    if w.fmt == W.NVFP4:
-        ts = oracle.nv_tensor_scale(oracle.rotated_amax(x, w.block))
+    x, ts = oracle_sample(w, rows_per_batch)
     done_rows = 0
     t0 = time.perf_counter()
     with threadpool_limits(limits=1):
@@ -796,41 +878,61 @@ def cpu_baseline(w, args, seconds: float = 10.0):
             done_rows += x.shape[0]
             if time.perf_counter() - t0 >= seconds:
                 break
-    dt = time.perf_counter() - t0
-    sample_bytes = w.with_rows(done_rows).bytes_per_call()
-    return {"value": round(sample_bytes / dt / 1e9, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{done_rows} rows x {w.K} ({x.shape[0]}-row batches of the same workload), "
-                      f"{dt:.1f} s wall on 1 host thread"}
+    dt1 = time.perf_counter() - t0
+    single = {"value": round(w.with_rows(done_rows).bytes_per_call() / dt1 / 1e9, 5), "unit": "GB/s", "cores": 1,
+              "sample": f"{done_rows} rows x {w.K} ({x.shape[0]}-row batches), {dt1:.1f} s wall on 1 host thread"}
+
+    n = min(host_cores(), 128)
+    job = (x, w.fmt, w.group, w.block, w.rule, ts)
+    with oracle_pool(n) as pool:
+        pool.map(_oracle_batch, [job] * n, chunksize=1)          # start-up and imports, untimed
+        done_rows = 0
+        pending = []
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < seconds:
+            while len(pending) < 2 * n:
+                pending.append(pool.apply_async(_oracle_batch, (job,)))
+            done_rows += pending.pop(0).get()
+        for p in pending:
+            done_rows += p.get()
+        dtn = time.perf_counter() - t0
+    value = w.with_rows(done_rows).bytes_per_call() / dtn / 1e9
+    return {"value": round(value, 5), "unit": "GB/s", "cores": n, "kind": "oracle",
+            "sample": f"{done_rows} rows x {w.K} ({x.shape[0]}-row batches of the same workload, one process per "
+                      f"core, one BLAS thread each), {dtn:.1f} s wall on {n} host cores",
+            "cpu_model": cpu_model(), "host_cores": host_cores(), "single_thread": single}
 
 
 def run_reference(args):
+    """The reference arm: the oracle, as it stands, on every host core.  One step is one
+    bounded sample of the workload: one batch of rows per core, run in parallel."""
     world, rank, _ = dist_setup()
     if rank != 0:
         return
-    import oracle
-    from threadpoolctl import threadpool_limits
     w = W.BY_NAME[args.workload]
-    rows = max(1, (1 << 18) // w.K)          # a bounded sample per step
-    x = next(iter(w.row_chunks(chunk_rows=rows)))
-    ts = oracle.nv_tensor_scale(oracle.rotated_amax(x, w.block)) if w.fmt == W.NVFP4 else None
-    cores = 1
-    with threadpool_limits(limits=cores):
+    rows = max(1, (1 << 18) // w.K)
+    x, ts = oracle_sample(w, rows)
+    n = min(host_cores(), 128)
+    job = (x, w.fmt, w.group, w.block, w.rule, ts)
+    with oracle_pool(n) as pool:
+        pool.map(_oracle_batch, [job] * n, chunksize=1)
         for _ in range(args.warmup):
-            oracle.rotate_quantize(x, w.fmt, w.group, w.block, w.rule, tensor_scale=ts)
+            pool.map(_oracle_batch, [job] * n, chunksize=1)
         t0 = time.perf_counter()
         for _ in range(args.steps):
-            oracle.rotate_quantize(x, w.fmt, w.group, w.block, w.rule, tensor_scale=ts)
+            pool.map(_oracle_batch, [job] * n, chunksize=1)
         dt = time.perf_counter() - t0
-    sb = w.with_rows(x.shape[0]).bytes_per_call()
+    sb = w.with_rows(x.shape[0] * n).bytes_per_call()
     value = sb * args.steps / dt / 1e9
     line = {
         "impl": "reference",
         "metric": METRIC, "value": round(value, 5), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
-        "config": {"workload": w.name, "M": w.M, "K": w.K, "sample_rows_per_step": x.shape[0]},
-        "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{x.shape[0]} rows x {w.K} per step"},
+        "config": {"workload": w.name, "M": w.M, "K": w.K, "sample_rows_per_step": x.shape[0] * n},
+        "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": n, "kind": "oracle",
+                         "sample": f"{x.shape[0]} rows x {w.K} per core per step, {n} host cores",
+                         "cpu_model": cpu_model()},
         "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -843,7 +945,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=W.NV_4K.name, choices=sorted(W.BY_NAME))
     ap.add_argument("--impl", default="fp4q", choices=["fp4q", "reference"])
-    ap.add_argument("--all-workloads", action="store_true", help="also time the other workloads")
+    ap.add_argument("--all-workloads", action="store_true",
+                    help="also time every workload's variants (other kernel, signs, error pass, MBS) and the FP4 GEMM")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the other target workloads (the 'targets' entry of the line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rows", type=int, default=0, help="override the workload's row count M")
     ap.add_argument("--kernel", default="auto", choices=["auto", "butterfly", "tensor_core"],
