@@ -43,11 +43,13 @@ METRIC = "fused rotate+FP4-quantize GB/s (bf16 in + packed out), % of B200 HBM p
 KERNELS = {"auto": 0, "butterfly": 1, "tensor_core": 2}
 
 
-def kernel_name(w, requested: str) -> str:
+def kernel_name(w, requested: str, signed: bool = False) -> str:
     """The kernel a plan with this request runs (auto: tensor core when b >= 16, b >= g and
-    M*K >= 2^22)."""
+    M*K >= 2^22, except MXFP4 with channel signs at b = 128)."""
     if requested != "auto":
         return requested
+    if signed and w.fmt == W.MXFP4 and w.block == 128:
+        return "butterfly"
     return "tensor_core" if (w.block >= 16 and w.block >= w.group and w.numel >= (1 << 22)) else "butterfly"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
@@ -197,8 +199,11 @@ def time_graph_steps(torch, launch, n_buf: int, steps: int, warmup: int, stream)
             for i in range(rem):
                 launch(i % n_buf)
     reps = steps // G
-    # a short untimed soak so that the clocks settle under this load
+    # a short untimed soak so that the clocks settle under this load; every graph is launched
+    # once here, so that no first launch (which uploads the graph) falls in a timed region
     g.replay()
+    if g_rem is not None:
+        g_rem.replay()
     torch.cuda.synchronize()
     return g, g_rem, reps
 
@@ -617,7 +622,7 @@ def time_signed(torch, F, w, xs, codes, scales, ts, stream, peak, steps, kernel=
     nbytes = w.bytes_per_call()
     gbs = nbytes / us / 1e3
     return {"us_per_call": round(us, 3), "GBps": round(gbs, 1), "pct_of_hbm_peak": round(100 * gbs / peak, 2),
-            "bytes_per_call": nbytes, "kernel": kernel_name(w, kernel)}
+            "bytes_per_call": nbytes, "kernel": kernel_name(w, kernel, signed=True)}
 
 
 def run_gemm_only(args):
@@ -761,11 +766,45 @@ def time_target(torch, F, w, dev, stream, peak, steps, cache):
     assert F.fp4q_device_status() == F.FP4Q_OK
     us = ms * 1e3 / steps
     gbs = bytes_call / us / 1e3
-    del xs, codes, scales, g, g_rem
-    return {"GBps": round(gbs, 1), "pct_of_hbm_peak": round(100 * gbs / peak, 2), "us_per_call": round(us, 3),
-            "elements_per_s": round(M * K / (us * 1e-6), 1), "bytes_per_call": bytes_call, "steps": steps,
-            "buffers": n_buf, "kernel": kernel_name(w, "auto"), "format": "NVFP4" if nv else "MXFP4",
-            "hadamard_block": w.block, "scale_rule": W.RULE_NAMES[w.rule], "clocks": sampler.summary()}
+    del g, g_rem
+    out = {"GBps": round(gbs, 1), "pct_of_hbm_peak": round(100 * gbs / peak, 2), "us_per_call": round(us, 3),
+           "elements_per_s": round(M * K / (us * 1e-6), 1), "bytes_per_call": bytes_call, "steps": steps,
+           "buffers": n_buf, "kernel": kernel_name(w, "auto"), "format": "NVFP4" if nv else "MXFP4",
+           "hadamard_block": w.block, "scale_rule": W.RULE_NAMES[w.rule], "clocks": sampler.summary()}
+    if kernel_name(w, "auto") == "tensor_core":
+        # the randomised rotation (per-channel random signs) on the same buffers and kernel
+        out["signed"] = time_signed(torch, F, w, xs, codes, scales, ts if nv else None, stream, peak, steps)
+    if w.block == 128:
+        # the error pass, and (MXFP4) MBS-Static, on the same inputs
+        out["quant_error"] = time_quant_error(torch, F, w, plan, xs, ts if nv else None, stream, peak, steps)
+        if not nv:
+            out["mbs_static"] = time_mbs_on(torch, F, w, xs, stream, peak, steps)
+    del xs, codes, scales
+    return out
+
+
+def time_mbs_on(torch, F, w, xs, stream, peak, steps):
+    """MBS-Static (MXFP4 with 128-element macro scales, the workload's block and rule) on the
+    given input buffers: device time per call, GB/s on its algorithmic bytes (bf16 in; codes,
+    E8M0 group scales and macro bytes out)."""
+    M, K = w.M, w.K
+    plan = F.fp4q_plan_create(F.FP4Q_MXFP4_MBS, 32, w.block, w.rule)
+    dev = xs[0].device
+    codes = [torch.empty((M, K // 2), dtype=torch.uint8, device=dev) for _ in xs]
+    scales = [torch.empty((M, K // 32), dtype=torch.uint8, device=dev) for _ in xs]
+    macro = [torch.empty((M, K // 128), dtype=torch.uint8, device=dev) for _ in xs]
+
+    def launch(i):
+        F.fp4q_rotate_quantize_mbs(plan, xs[i], M, K, codes[i], scales[i], macro[i], stream=torch.cuda.current_stream())
+
+    with torch.cuda.stream(stream):
+        g, g_rem, reps = time_graph_steps(torch, launch, len(xs), steps, 3, stream)
+    us = time_replays(torch, g, g_rem, reps, stream) * 1e3 / steps
+    nbytes = M * K * 2 + M * K // 2 + M * K // 32 + M * K // 128
+    gbs = nbytes / us / 1e3
+    del g, g_rem, codes, scales, macro
+    return {"us_per_call": round(us, 3), "GBps": round(gbs, 1), "pct_of_hbm_peak": round(100 * gbs / peak, 2),
+            "bytes_per_call": nbytes, "kernel": kernel_name(w, "auto")}
 
 
 def time_other(torch, F, w, dev, stream, peak, kernel="auto"):

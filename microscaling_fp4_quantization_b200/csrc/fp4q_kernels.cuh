@@ -674,53 +674,43 @@ __global__ void __launch_bounds__(Cfg::kThreads) rotate_quantize_kernel(RQArgs a
 
 // ---------------------------------------------------------------- quantization error
 
-// The magnitude bits of nibble E of a code word, as the fp32 pattern k << 22 (k = magnitude
-// code 0..7).  That pattern is 2^-126 * {0, 0.5, 1, 1.5, 2, 3, 4, 6}[k] exactly (k = 1 a
-// subnormal; nothing here is compiled with flush-to-zero).
-template <int E>
-__device__ __forceinline__ float e2m1_mag_scaled(uint32_t w) {
-  constexpr int s = 22 - 4 * E;
-  return __uint_as_float((s >= 0 ? (w << s) : (w >> -s)) & 0x01C00000u);
+// The errors q - v of one pair of quotients v against their E2M1 codes q (round to nearest
+// even, saturating at 6): the pair goes to E2M1 and straight back to f16x2 (exact: every E2M1
+// value is an f16 value), then each q - v is one mixed-precision subtraction, rounded once to
+// fp32.  |q - v| is also |(|v| - |q|)| (E2M1 rounding keeps the sign of v), so the squares are
+// the error energies whatever the sign convention.
+__device__ __forceinline__ void e2m1_pair_errors(f32x2 v, float& d0, float& d1) {
+  float v0, v1;
+  f2_unpack(v, v0, v1);
+  asm("{\n .reg .b8 q;\n .reg .b32 h;\n .reg .b16 lo, hi;\n"
+      " cvt.rn.satfinite.e2m1x2.f32 q, %3, %2;\n"
+      " cvt.rn.f16x2.e2m1x2 h, q;\n"
+      " mov.b32 {lo, hi}, h;\n"
+      " sub.rn.f32.f16 %0, lo, %2;\n"
+      " sub.rn.f32.f16 %1, hi, %3;\n}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(v0), "f"(v1));
 }
 
 // Error energy of one group of quotients v (= y / X) against their E2M1 codes, and its
-// signal energy, both in units of X^2: sum (v - q)^2 and sum v^2 (fp32; even and odd elements
-// in separate sums).  E2M1 rounding keeps the sign of v, so v - q = sign(v) (|v| - |q|), and
-// |v| - |q| is one fused multiply-add of the scaled magnitude by -2^126 (the product is exact).
+// signal energy, both in units of X^2: sum (v - q)^2 and sum v^2 (fp32, in pairs of lanes
+// of packed sums).
 template <int NP>
 __device__ __forceinline__ void group_energies(const f32x2 (&v)[NP], float& sig, float& err) {
-  f32x2 as = f2_pack(0.0f, 0.0f);
-  float e0 = 0.0f, e1 = 0.0f;
+  f32x2 as = f2_pack(0.0f, 0.0f), ae = f2_pack(0.0f, 0.0f);
 #pragma unroll
-  for (int j = 0; j < NP / 4; ++j) {
-    f32x2 vv[4];
-#pragma unroll
-    for (int t = 0; t < 4; ++t) vv[t] = v[4 * j + t];
-    const uint32_t w = e2m1x8_pairs(vv);
-    float lo[4], hi[4], q0[4], q1[4];
-#pragma unroll
-    for (int t = 0; t < 4; ++t) f2_unpack(vv[t], lo[t], hi[t]);
-    q0[0] = e2m1_mag_scaled<0>(w);
-    q1[0] = e2m1_mag_scaled<1>(w);
-    q0[1] = e2m1_mag_scaled<2>(w);
-    q1[1] = e2m1_mag_scaled<3>(w);
-    q0[2] = e2m1_mag_scaled<4>(w);
-    q1[2] = e2m1_mag_scaled<5>(w);
-    q0[3] = e2m1_mag_scaled<6>(w);
-    q1[3] = e2m1_mag_scaled<7>(w);
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      as = f2_fma(vv[t], vv[t], as);
-      const float d0 = fmaf(q0[t], -0x1p126f, fabsf(lo[t]));
-      const float d1 = fmaf(q1[t], -0x1p126f, fabsf(hi[t]));
-      e0 = fmaf(d0, d0, e0);
-      e1 = fmaf(d1, d1, e1);
-    }
+  for (int t = 0; t < NP; ++t) {
+    as = f2_fma(v[t], v[t], as);
+    float d0, d1;
+    e2m1_pair_errors(v[t], d0, d1);
+    const f32x2 d = f2_pack(d0, d1);
+    ae = f2_fma(d, d, ae);
   }
-  float a0, a1;
+  float a0, a1, b0, b1;
   f2_unpack(as, a0, a1);
+  f2_unpack(ae, b0, b1);
   sig = a0 + a1;
-  err = e0 + e1;
+  err = b0 + b1;
 }
 
 // 2^(2(byte - 127)) as fp64: X^2 for an MX scale byte.

@@ -223,24 +223,34 @@ __device__ __forceinline__ uint32_t quantize_group(const float (&s)[G], uint32_t
   return byte;
 }
 
-// MBS-Static on G rotated sums s of one group: y' = RN(y / s_M) (dv: the divisor for s_M),
-// then the MXFP4 scale byte of y' under the plan's rule and the E2M1 code words of
-// y' / 2^(byte - 127), as the butterfly kernel's quantizer takes them.
+// MBS-Static on G rotated sums s of one group, with r = RN(1 / (s_M sqrt(b))): y' = RN(s r),
+// within about one ulp of the correctly rounded RN(y / s_M) that the butterfly kernel takes, so a
+// decision can move only where its exact value lies within a few 2^-24 (relative) of a rounding
+// or scale boundary, inside the flagged set (as for the NVFP4 element quotients).  Then the
+// MXFP4 scale byte of y' under the plan's rule (its amax is RN(max |s| r): RN is monotone) and
+// the codes of y' / 2^(byte - 127) = RN(s r 2^(127 - byte)) (the power of two is exact).
 template <class Cfg, int G>
-__device__ __forceinline__ uint32_t quantize_group_mbs(const float (&s)[G], NvDivisor dv, uint32_t (&words)[G / 8]) {
+__device__ __forceinline__ uint32_t quantize_group_mbs(const float (&s)[G], float r, uint32_t (&words)[G / 8]) {
   f32x2 p[G / 2];
 #pragma unroll
   for (int k = 0; k < G / 2; ++k) p[k] = f2_pack(s[2 * k], s[2 * k + 1]);
-  f32x2 yq[G / 2];
-  nv_quotients<Cfg::kBlock, G / 2>(p, dv, yq);
-  const int byte = mx_scale_byte<Cfg::kRule>(pairs_amax<G / 2>(yq));
+  const int byte = mx_scale_byte<Cfg::kRule>(pairs_amax<G / 2>(p) * r);
+  const float m = r * mx_inv_scale(byte);
+  const f32x2 mm = f2_pack(m, m);
 #pragma unroll
   for (int j = 0; j < G / 8; ++j) {
     f32x2 v[4];
-    mx_quotients<4>(&yq[4 * j], byte, 1.0f, v);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) v[t] = f2_mul(p[4 * j + t], mm);
     words[j] = e2m1x8_pairs(v);
   }
   return static_cast<uint32_t>(byte);
+}
+
+// r = RN(1 / (s_M sqrt(b))) for quantize_group_mbs: one fp64 division, rounded to fp32.
+template <int B>
+__device__ __forceinline__ float mbs_multiplier(float sM) {
+  return static_cast<float>(inv_sqrt_block_f64(B) / static_cast<double>(sM));
 }
 
 // The macro-scale byte of MBS-Static for this lane's macro block, from the largest raw sum
@@ -337,16 +347,17 @@ __device__ __forceinline__ void store_piece(const MmaArgs& a, int64_t row, int o
 // group_energy_mma for MBS-Static: the quotients and codes of quantize_group_mbs, energies in
 // units of X^2 = 2^(2 (byte - 127)) s_M^2 (sM2).
 template <class Cfg, int G>
-__device__ __forceinline__ void group_energy_mma_mbs(const float (&s)[G], NvDivisor dv, double sM2, double& sig,
+__device__ __forceinline__ void group_energy_mma_mbs(const float (&s)[G], float r, double sM2, double& sig,
                                                      double& err) {
   f32x2 p[G / 2];
 #pragma unroll
   for (int k = 0; k < G / 2; ++k) p[k] = f2_pack(s[2 * k], s[2 * k + 1]);
-  f32x2 yq[G / 2];
-  nv_quotients<Cfg::kBlock, G / 2>(p, dv, yq);
-  const int byte = mx_scale_byte<Cfg::kRule>(pairs_amax<G / 2>(yq));
+  const int byte = mx_scale_byte<Cfg::kRule>(pairs_amax<G / 2>(p) * r);
+  const float m = r * mx_inv_scale(byte);
+  const f32x2 mm = f2_pack(m, m);
   f32x2 v[G / 2];
-  mx_quotients<G / 2>(yq, byte, 1.0f, v);
+#pragma unroll
+  for (int k = 0; k < G / 2; ++k) v[k] = f2_mul(p[k], mm);
   float gs, ge;
   group_energies<G / 2>(v, gs, ge);
   const double X2 = mx_scale_sq(byte) * sM2;
@@ -674,7 +685,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
           const int64_t row = t * Cfg::kRowsPerTile + j * 128 + lane_row;
           const uint32_t m8 = mbs_lane_macro_byte<Cfg>(am[pc], am_other);
           const float sM = mbs_macro_scale(m8);
-          const NvDivisor mdv = nv_divisor<B>(sM);
+          const float mr = mbs_multiplier<B>(sM);
           if constexpr (!Cfg::kQE) {
             // the macro byte from the macro block's first lane (b = 128: the first half's warp)
             const bool first = Cfg::kMacroLanes > 1 ? (lane % Cfg::kMacroLanes) == 0 : half == 0;
@@ -697,13 +708,13 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
             }
             if constexpr (Cfg::kQE) {
               if (row < a.n_rows)
-                group_energy_mma_mbs<Cfg, G>(gv, mdv, static_cast<double>(sM) * static_cast<double>(sM), qe_sig,
+                group_energy_mma_mbs<Cfg, G>(gv, mr, static_cast<double>(sM) * static_cast<double>(sM), qe_sig,
                                              qe_err);
             } else {
               // each group's codes and scale go out as soon as they are made
               uint32_t gw[G / 8];
               uint32_t sb[1];
-              sb[0] = quantize_group_mbs<Cfg, G>(gv, mdv, gw);
+              sb[0] = quantize_group_mbs<Cfg, G>(gv, mr, gw);
 #pragma unroll
               for (int e = 0; e < G / 8; ++e) {
                 const int chunk = (off + q * G) / 8 + e;
@@ -778,6 +789,9 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
             if constexpr (Cfg::kBulk) {
               if (chunk & 1) w ^= flip_basis0;
               if (chunk & 2) w ^= flip_basis1;
+              // a zero NV block scale gives code 0x0 for every element: the flip above must not
+              // turn them into 0x8
+              if constexpr (Cfg::kFmt == kNV) w = sbytes[q] == 0u ? 0u : w;
             }
             words[q * (G / 8) + e] = w;
           }
