@@ -693,24 +693,25 @@ __device__ __forceinline__ void e2m1_pair_errors(f32x2 v, float& d0, float& d1) 
 }
 
 // Error energy of one group of quotients v (= y / X) against their E2M1 codes, and its
-// signal energy, both in units of X^2: sum (v - q)^2 and sum v^2 (fp32, in pairs of lanes
-// of packed sums).
+// signal energy, both in units of X^2: sum (v - q)^2 and sum v^2 (fp32; even and odd elements
+// in separate sums, the signal as packed pairs, the errors as two scalar sums, which leaves
+// the two differences where the subtractions put them).
 template <int NP>
 __device__ __forceinline__ void group_energies(const f32x2 (&v)[NP], float& sig, float& err) {
-  f32x2 as = f2_pack(0.0f, 0.0f), ae = f2_pack(0.0f, 0.0f);
+  f32x2 as = f2_pack(0.0f, 0.0f);
+  float e0 = 0.0f, e1 = 0.0f;
 #pragma unroll
   for (int t = 0; t < NP; ++t) {
     as = f2_fma(v[t], v[t], as);
     float d0, d1;
     e2m1_pair_errors(v[t], d0, d1);
-    const f32x2 d = f2_pack(d0, d1);
-    ae = f2_fma(d, d, ae);
+    e0 = fmaf(d0, d0, e0);
+    e1 = fmaf(d1, d1, e1);
   }
-  float a0, a1, b0, b1;
+  float a0, a1;
   f2_unpack(as, a0, a1);
-  f2_unpack(ae, b0, b1);
   sig = a0 + a1;
-  err = b0 + b1;
+  err = e0 + e1;
 }
 
 // 2^(2(byte - 127)) as fp64: X^2 for an MX scale byte.
