@@ -456,6 +456,15 @@ def run_gpu(args):
                            else "rotate_quantize_kernel"), "us_per_launch": round(kernel_us, 3),
             },
             "gpu_launches": args.steps,
+            # the pages' own figures, for context only: end-to-end and layer-wise speedups of the
+            # whole MR-GPTQ FP4 stack (quantized GEMMs in vLLM) over FP16, on other workloads
+            "context": {
+                "source": "Bridging the Gap Between Promise and Performance for Microscaling FP4 "
+                          "Quantization: abstract; Technische Zusammenfassung, 3. Wichtige Ergebnisse",
+                "speedup_vs_fp16_B200": {"layer_wise": "up to 3.6x", "end_to_end": "up to 2.2x"},
+                "speedup_vs_fp16_RTX5090": {"layer_wise": "up to 6x", "end_to_end": "up to 4x"},
+                "note": "not a measurement of this path, and not its target",
+            },
             "clocks": sampler.summary(),
             "e2e": e2e,
             "cpu_baseline": cpu,
