@@ -44,11 +44,15 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 
+// One try: the thread may be suspended in hardware until the phase completes, for at most
+// the hint (20 us) before it returns false.  A suspended warp issues nothing, so waiting
+// roles (producer, MMA issuer, sign warps, idle epilogue warps) leave the issue slots to the
+// warps with work (measured: the headline kernel 8.57 -> 8.41 us per call).
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n .reg .pred p;\n"
-      " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 20000;\n"
       " selp.u32 %0, 1, 0, p;\n}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
