@@ -127,7 +127,9 @@ typedef enum {
                                   plans with channel signs and b = 128 stay on the butterfly
                                   kernel (faster there, by measurement)                        */
   FP4Q_KERNEL_BUTTERFLY = 1,   /* in-register fast Walsh-Hadamard butterfly on CUDA cores    */
-  FP4Q_KERNEL_TENSOR_CORE = 2  /* tcgen05 MMA against H_b with TMEM accumulators            */
+  FP4Q_KERNEL_TENSOR_CORE = 2  /* tcgen05 MMA against H_b with TMEM accumulators; tensors of
+                                  2^31 - 1024 or more Hadamard blocks (the limit of its 32-bit
+                                  TMA row coordinates) still run on the butterfly kernel      */
 } fp4q_kernel;
 
 /* Choose the kernel for later rotate + quantize calls of this plan (not thread-safe against
