@@ -42,9 +42,14 @@ fp4q_status launch_mma_common(MmaArgs a, const uint16_t* x, int64_t n_elems, con
   a.n_super = (a.n_rows + Cfg::kRowsPerTile - 1) / Cfg::kRowsPerTile;
   a.sign_bytes = reinterpret_cast<const uint8_t*>(signs.mask);
   a.sign_upr = signs.mask ? K / Cfg::kBlock : 1;
-  // the mask's words (ceil(K / 32) of them), staged in shared memory when they fit
+  // the expanded sign table (4 K bytes) where the configuration has one and it fits, else the
+  // mask's words (ceil(K / 32) of them), staged in shared memory when they fit
   const int64_t mask_bytes = signs.mask ? (K + 127) / 128 * 16 : 0;
-  a.sign_smem = mask_bytes <= Cfg::kMaskSmemMax ? static_cast<int>(mask_bytes) : 0;
+  const int64_t table_bytes = signs.mask ? 4 * K : 0;
+  a.sign_table = signs.mask && Cfg::kSignTable && table_bytes <= Cfg::kSignTableMax ? 1 : 0;
+  a.sign_smem = a.sign_table                      ? static_cast<int>(table_bytes)
+                : mask_bytes <= Cfg::kMaskSmemMax ? static_cast<int>(mask_bytes)
+                                                  : 0;
   CUtensorMap map;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(Cfg::kBlock), static_cast<cuuint64_t>(a.n_rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(Cfg::kBlock) * 2};
@@ -62,7 +67,7 @@ fp4q_status launch_mma_common(MmaArgs a, const uint16_t* x, int64_t n_elems, con
   }
   auto kernel = rotate_quantize_mma_kernel<Cfg>;
   KernelInfo ki;
-  st = kernel_info(kernel, Cfg::kSmemBytes + Cfg::kMaskSmemMax, Cfg::kThreads, &ki);
+  st = kernel_info(kernel, Cfg::kSmemBytes + Cfg::kSignSmemMax, Cfg::kThreads, &ki);
   if (st != FP4Q_OK) return st;
   // CTAs per SM from measurement (the kernel's CTAs are independent, so a CTA that does not
   // fit next to the others simply starts later); tensor memory holds 512 columns per SM

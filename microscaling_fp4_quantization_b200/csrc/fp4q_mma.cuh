@@ -93,10 +93,19 @@ struct MmaConfig {
   static constexpr int kMaskOffset = (kBarOffset + 8 * (3 * kStages + 4) + 15) / 16 * 16;
   static constexpr int kSmemBytes = 1024 + kMaskOffset;   // without the staged sign mask
   // Plans with channel signs stage the mask (K / 8 bytes) after the barriers when it fits
-  // beside kCtasPerSm CTAs (228 KB of shared memory per SM, 1 KB of it reserved per CTA).
-  static constexpr int kMaskRoom = (233472 / kCtasPerSm - 1024 - kSmemBytes) / 16 * 16;
+  // beside kCtasPerSm CTAs: 228 KB of shared memory per SM, of which each CTA also holds 1 KB
+  // reserved by the system and 1 KB of static variables (the kernel's __shared__ scalars,
+  // padded to the 1024-byte alignment of the dynamic array that follows them).
+  static constexpr int kMaskRoom = (233472 / kCtasPerSm - 2048 - kSmemBytes) / 16 * 16;
   static constexpr int kMaskSmemMax = kMaskRoom < 16384 ? kMaskRoom : 16384;
   static_assert(kMaskSmemMax >= 1024, "room for the sign mask of K <= 8192");
+  // Where one CTA has the SM, the sign warps read an expanded table instead of the mask's
+  // bits: the four XOR words of every 8-channel chunk of a row (16 bytes each), stored twice
+  // over so that a block index below 2 K/b needs no wrap; 4 K bytes, staged when they fit
+  // (K <= 16384).
+  static constexpr bool kSignTable = kCtasPerSm == 1;
+  static constexpr int kSignTableMax = kSignTable ? cmin(kMaskRoom, 65536) : 0;
+  static constexpr int kSignSmemMax = cmax(kMaskSmemMax, kSignTableMax);
   static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(B >> 3) << 17) |
                                      (static_cast<uint32_t>(128 >> 4) << 24);
 };
@@ -113,7 +122,8 @@ struct MmaArgs {
   float* y_dump;
   const uint8_t* sign_bytes;   // per-channel signs (bit k of byte k / 8 negates channel k), or null
   int64_t sign_upr;            // Hadamard blocks per matrix row, K / b
-  int sign_smem;               // bytes of the mask staged in shared memory (0: read from global)
+  int sign_smem;               // bytes staged in shared memory (0: the mask is read from global)
+  int sign_table;              // 1: those bytes are the expanded sign table, 0: the mask's words
   uint8_t* macro;              // MBS-Static: the macro-scale bytes [R * b / 128]
   // error pass only: [gridDim.x][2] per-CTA signal, error energies; the ticket counter (0
   // between calls, reset by the last CTA); out [3] = signal, error, QSNR dB
@@ -540,31 +550,86 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
       const uint32_t upr = static_cast<uint32_t>(a.sign_upr);
       const uint32_t row_step = static_cast<uint32_t>(kRowStep) % upr;
       pdl_wait();   // the mask belongs to the caller and may come from an earlier kernel
-      const uint8_t* mask = a.sign_bytes;
-      if (a.sign_smem > 0) {
+      // Hadamard block (within its matrix row) of the lane's first row, kept incrementally:
+      // super-tile t starts at block (t * kRowsPerTile) mod upr, and t advances by gridDim.x
+      const uint32_t tile_step = static_cast<uint32_t>((static_cast<uint64_t>(gridDim.x) * Cfg::kRowsPerTile) % upr);
+      const uint32_t row0_kb = row0 % upr;
+      uint32_t tile_kb = static_cast<uint32_t>((static_cast<uint64_t>(blockIdx.x) * Cfg::kRowsPerTile) % upr);
+      const uint32_t tab_s = stage0 + Cfg::kMaskOffset;
+      if constexpr (Cfg::kSignTable) {
+        if (a.sign_table) {
+          // the expanded table: entry e (and e + K/8) = the XOR words of mask byte e
+          const uint32_t chunks = upr * (B / 8);
+          for (uint32_t e = 32 * sw + lane; e < 2 * chunks; e += 32 * Cfg::kSignWarps)
+            sts128_u4(tab_s + 16u * e, chunk_sign_xor(__ldg(a.sign_bytes + (e < chunks ? e : e - chunks))));
+          asm volatile("bar.sync 2, %0;" ::"r"(32 * Cfg::kSignWarps) : "memory");
+          static_assert(kRegions == 1 && kPerLane % kBatch == 0, "one region, whole batches");
+          // byte offsets, in the table, of the lane's chunks relative to its first: chunk u sits
+          // (u * kRowStep) mod upr blocks further on (the same for every lane and stage)
+          uint32_t dk[kPerLane];
+#pragma unroll
+          for (int u = 0; u < kPerLane; ++u)
+            dk[u] = static_cast<uint32_t>((static_cast<uint64_t>(u) * row_step) % upr) * (2u * B);
+          int64_t i = 0;
+          for (int64_t t = blockIdx.x; t < n_super; t += gridDim.x, ++i) {
+            const int s = static_cast<int>(i % S);
+            const uint32_t ph = static_cast<uint32_t>((i / S) & 1);
+            uint32_t kb_first = tile_kb + row0_kb;
+            if (kb_first >= upr) kb_first -= upr;
+            tile_kb += tile_step;
+            if (tile_kb >= upr) tile_kb -= upr;
+            // logical chunk of the lane's rows: the bulk layout is unswizzled; a swizzled row's
+            // physical chunk is its logical one XOR (row & 7)
+            const uint32_t q = Cfg::kBulk ? pq : (pq ^ (row0 & 7u));
+            const uint32_t tb = tab_s + kb_first * (2u * B) + 16u * q;
+            const uint32_t addr = stage0 + s * Cfg::kStageBytes + 16u * c0;
+            const bool mine = mbar_wait_bounded(full_bar(s), ph);
+            if (!__all_sync(0xFFFFFFFFu, mine)) break;
+#pragma unroll
+            for (int j = 0; j < kPerLane; j += kBatch) {
+              uint4 w[kBatch], f[kBatch];
+#pragma unroll
+              for (int u = 0; u < kBatch; ++u) {
+                f[u] = lds128(tb + dk[j + u]);
+                w[u] = lds128(addr + 16u * kLaneStride * (j + u));
+              }
+#pragma unroll
+              for (int u = 0; u < kBatch; ++u)
+                sts128_u4(addr + 16u * kLaneStride * (j + u),
+                          make_uint4(w[u].x ^ f[u].x, w[u].y ^ f[u].y, w[u].z ^ f[u].z, w[u].w ^ f[u].w));
+            }
+            fence_proxy_async_smem();   // the tensor core reads the stage through the async proxy
+            __syncwarp();
+            if (lane == 0) mbar_arrive(signed_bar(s));
+          }
+        }
+      }
+      const uint8_t* mask_g = a.sign_bytes;
+      const bool staged = a.sign_smem > 0;
+      const uint32_t mask_s = tab_s;
+      if (staged && !a.sign_table) {
         // the mask's words, once per CTA, into shared memory (a few hundred bytes to 16 KB)
         uint32_t* ms = reinterpret_cast<uint32_t*>(smem + Cfg::kMaskOffset);
         const uint32_t* mg = reinterpret_cast<const uint32_t*>(a.sign_bytes);
         const int words = static_cast<int>((static_cast<int64_t>(upr) * B + 31) / 32);   // the caller's ceil(K / 32)
         for (int w = 32 * sw + lane; w < words; w += 32 * Cfg::kSignWarps) ms[w] = __ldg(mg + w);
         asm volatile("bar.sync 2, %0;" ::"r"(32 * Cfg::kSignWarps) : "memory");
-        mask = smem + Cfg::kMaskOffset;
       }
       int64_t i = 0;
-      for (int64_t t = blockIdx.x; t < n_super; t += gridDim.x, ++i) {
+      for (int64_t t = blockIdx.x; !a.sign_table && t < n_super; t += gridDim.x, ++i) {
         const int s = static_cast<int>(i % S);
         const uint32_t ph = static_cast<uint32_t>((i / S) & 1);
+        uint32_t kb_first = tile_kb + row0_kb;
+        if (kb_first >= upr) kb_first -= upr;
+        tile_kb += tile_step;
+        if (tile_kb >= upr) tile_kb -= upr;
         const bool mine = mbar_wait_bounded(full_bar(s), ph);
         if (!__all_sync(0xFFFFFFFFu, mine)) break;
-        // Hadamard block (within its matrix row) of the lane's first row
-        const uint32_t kb_first = static_cast<uint32_t>(
-            (static_cast<uint64_t>((t * Cfg::kRowsPerTile) % upr) + row0) % upr);
 #pragma unroll 1
         for (int h = 0; h < kRegions; ++h) {
           // logical chunk of the lane's rows: the bulk layout is unswizzled; a swizzled row's
           // physical chunk is its logical one XOR (row & 7)
           const uint32_t q = Cfg::kBulk ? pq : 8u * h + (pq ^ (row0 & 7u));
-          const uint8_t* mq = mask + q;
           uint32_t kb = kb_first;
           uint32_t addr = stage0 + s * Cfg::kStageBytes + h * kRegionBytes + 16u * c0;
 #pragma unroll 1
@@ -573,7 +638,8 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
             uint32_t m[kBatch];
 #pragma unroll
             for (int u = 0; u < kBatch; ++u) {
-              m[u] = mq[kb * (B / 8)];
+              const uint32_t mi = kb * (B / 8) + q;   // the chunk's mask byte
+              m[u] = staged ? lds_u8(mask_s + mi) : static_cast<uint32_t>(__ldg(mask_g + mi));
               kb += row_step;
               if (kb >= upr) kb -= upr;
               w[u] = lds128(addr + 16u * kLaneStride * u);
