@@ -45,12 +45,14 @@ KERNELS = {"auto": 0, "butterfly": 1, "tensor_core": 2}
 
 def kernel_name(w, requested: str, signed: bool = False) -> str:
     """The kernel a plan with this request runs (auto: tensor core when b >= 16, b >= g and
-    M*K >= 2^22, except MXFP4 with channel signs at b = 128)."""
+    M*K >= 2^22, except MXFP4 with channel signs at b = 128 and M*K >= 3 * 2^26)."""
     if requested != "auto":
         return requested
-    if signed and w.fmt == W.MXFP4 and w.block == 128:
+    if signed and w.fmt == W.MXFP4 and w.block == 128 and w.numel >= (3 << 26):
         return "butterfly"
     return "tensor_core" if (w.block >= 16 and w.block >= w.group and w.numel >= (1 << 22)) else "butterfly"
+
+
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 SPEC_HBM_GBS = 8000.0

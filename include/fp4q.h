@@ -124,8 +124,9 @@ typedef enum {
   FP4Q_KERNEL_AUTO = 0,        /* the tensor-core kernel when every Hadamard block holds whole
                                   scale groups (b >= 16 and b >= g) and M*K >= 2^22, else the
                                   butterfly kernel (which starts faster on small tensors); MXFP4
-                                  plans with channel signs and b = 128 stay on the butterfly
-                                  kernel (faster there, by measurement)                        */
+                                  plans with channel signs and b = 128 take the butterfly
+                                  kernel from M*K >= 3 * 2^26 on (faster there, by
+                                  measurement)                                                 */
   FP4Q_KERNEL_BUTTERFLY = 1,   /* in-register fast Walsh-Hadamard butterfly on CUDA cores    */
   FP4Q_KERNEL_TENSOR_CORE = 2  /* tcgen05 MMA against H_b with TMEM accumulators; tensors of
                                   2^31 - 1024 or more Hadamard blocks (the limit of its 32-bit

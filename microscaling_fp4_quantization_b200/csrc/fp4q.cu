@@ -173,11 +173,14 @@ fp4q_status check_device(fp4q_plan p, const char* who) {
 
 // Whether the tensor-core kernel serves this plan.  AUTO takes it for tensors of at least
 // kMmaMinElems elements: below that its fixed start-up (TMEM allocation, H_b, filling a
-// three-stage pipeline) costs more than the butterfly kernel's extra instructions.  AUTO keeps
-// MXFP4 plans with channel signs and b = 128 on the butterfly kernel: there the tensor-core
-// kernel's pass that flips the signs in each landed stage holds it near 70 % of HBM bandwidth,
-// where the butterfly, which flips them as it loads, runs at 72-81 % (measured).
+// three-stage pipeline) costs more than the butterfly kernel's extra instructions.  MXFP4
+// plans with channel signs and b = 128 go to the butterfly kernel from kSignedMxMmaMaxElems
+// elements on: there the tensor-core kernel's pass that flips the signs in each landed stage
+// holds it near 80 % of HBM bandwidth, where the butterfly, which flips them as it loads, runs
+// at 84-87 %; below, the tensor core is the faster of the two (73-84 % against 65-80 %,
+// measured from 4096 x 8192 to 32768 x 14336).
 constexpr int64_t kMmaMinElems = int64_t(1) << 22;
+constexpr int64_t kSignedMxMmaMaxElems = int64_t(3) << 26;
 bool mma_capable(fp4q_plan p) { return p->block >= 16 && p->block >= p->group; }
 // The tensor-core kernel addresses its tiles with 32-bit TMA coordinates (rows of one Hadamard
 // block each); larger tensors go to the butterfly kernel.
@@ -185,7 +188,7 @@ constexpr int64_t kMmaMaxRows = (int64_t(1) << 31) - 1024;
 bool use_mma(fp4q_plan p, int64_t n_elems) {
   if (!mma_capable(p) || n_elems / p->block >= kMmaMaxRows) return false;
   if (p->kernel == FP4Q_KERNEL_TENSOR_CORE) return true;
-  if (p->signs && p->format == FP4Q_MXFP4 && p->block == 128) return false;
+  if (p->signs && p->format == FP4Q_MXFP4 && p->block == 128 && n_elems >= kSignedMxMmaMaxElems) return false;
   return p->kernel == FP4Q_KERNEL_AUTO && n_elems >= kMmaMinElems;
 }
 

@@ -233,6 +233,17 @@ __device__ __forceinline__ uint4 chunk_sign_xor(uint32_t mb) {
   return r;
 }
 
+// The same four XOR words folded into one: bit 15 - i holds the sign of element 2i and bit
+// 31 - i that of element 2i + 1, so word i of the chunk's XOR is (w << i) & 0x80008000.
+__device__ __forceinline__ uint32_t chunk_sign_word(uint32_t mb) {
+  const uint4 f = chunk_sign_xor(mb);
+  return f.x | (f.y >> 1) | (f.z >> 2) | (f.w >> 3);
+}
+
+__device__ __forceinline__ uint4 chunk_sign_xor_word(uint32_t w) {
+  return make_uint4(w & 0x80008000u, (w << 1) & 0x80008000u, (w << 2) & 0x80008000u, (w << 3) & 0x80008000u);
+}
+
 // Sign byte of original chunk q = j ^ tau of a unit (tau only touches the low three bits,
 // so the word is one of two known at compile time).
 template <int E>
@@ -744,44 +755,44 @@ __device__ __forceinline__ void unit_energies(const f32x2 (&p)[Cfg::kPairs], flo
       sig = fma(static_cast<double>(gs), X2, sig);
       err = fma(static_cast<double>(ge), X2, err);
     }
-    return;
-  }
+  } else {
 #pragma unroll
-  for (int q = 0; q < NG; ++q) {
-    const f32x2* pg = &p[q * G / 2];
-    const float A = scale_by_inv_sqrt<Cfg::kBlock>(pairs_amax<G / 2>(pg));
-    f32x2 v[G / 2];
-    double X2;
-    if constexpr (Cfg::kFmt == kMX) {
-      const int byte = mx_scale_byte<Cfg::kRule>(A);
-      mx_quotients<G / 2>(pg, byte, c, v);
-      X2 = mx_scale_sq(byte);
-    } else {
-      const float s_b = div_rn_markstein(A, nv_den, nv_rden);
-      const uint32_t byte = e4m3_encode(s_b);
-      const float S = e4m3_decode(byte) * s_g;
-      if (S == 0.0f) {
-        // a zero block scale: every code is 0, the error is the whole signal
-        constexpr double c64 = inv_sqrt_block_f64(Cfg::kBlock);
-        double e2 = 0.0;
+    for (int q = 0; q < NG; ++q) {
+      const f32x2* pg = &p[q * G / 2];
+      const float A = scale_by_inv_sqrt<Cfg::kBlock>(pairs_amax<G / 2>(pg));
+      f32x2 v[G / 2];
+      double X2;
+      if constexpr (Cfg::kFmt == kMX) {
+        const int byte = mx_scale_byte<Cfg::kRule>(A);
+        mx_quotients<G / 2>(pg, byte, c, v);
+        X2 = mx_scale_sq(byte);
+      } else {
+        const float s_b = div_rn_markstein(A, nv_den, nv_rden);
+        const uint32_t byte = e4m3_encode(s_b);
+        const float S = e4m3_decode(byte) * s_g;
+        if (S == 0.0f) {
+          // a zero block scale: every code is 0, the error is the whole signal
+          constexpr double c64 = inv_sqrt_block_f64(Cfg::kBlock);
+          double e2 = 0.0;
 #pragma unroll
-        for (int t = 0; t < G / 2; ++t) {
-          float lo, hi;
-          f2_unpack(pg[t], lo, hi);
-          const double a = lo * c64, b = hi * c64;
-          e2 = fma(a, a, fma(b, b, e2));
+          for (int t = 0; t < G / 2; ++t) {
+            float lo, hi;
+            f2_unpack(pg[t], lo, hi);
+            const double a = lo * c64, b = hi * c64;
+            e2 = fma(a, a, fma(b, b, e2));
+          }
+          sig += e2;
+          err += e2;
+          continue;
         }
-        sig += e2;
-        err += e2;
-        continue;
+        nv_quotients<Cfg::kBlock, G / 2>(pg, nv_divisor<Cfg::kBlock>(S), v);
+        X2 = static_cast<double>(S) * static_cast<double>(S);
       }
-      nv_quotients<Cfg::kBlock, G / 2>(pg, nv_divisor<Cfg::kBlock>(S), v);
-      X2 = static_cast<double>(S) * static_cast<double>(S);
+      float gs, ge;
+      group_energies<G / 2>(v, gs, ge);
+      sig = fma(static_cast<double>(gs), X2, sig);
+      err = fma(static_cast<double>(ge), X2, err);
     }
-    float gs, ge;
-    group_energies<G / 2>(v, gs, ge);
-    sig = fma(static_cast<double>(gs), X2, sig);
-    err = fma(static_cast<double>(ge), X2, err);
   }
 }
 

@@ -46,8 +46,13 @@ fp4q_status launch_mma_common(MmaArgs a, const uint16_t* x, int64_t n_elems, con
   // mask's words (ceil(K / 32) of them), staged in shared memory when they fit
   const int64_t mask_bytes = signs.mask ? (K + 127) / 128 * 16 : 0;
   const int64_t table_bytes = signs.mask ? 4 * K : 0;
-  a.sign_table = signs.mask && Cfg::kSignTable && table_bytes <= Cfg::kSignTableMax ? 1 : 0;
-  a.sign_smem = a.sign_table                      ? static_cast<int>(table_bytes)
+  const int64_t word_bytes = signs.mask ? 4 * (K / Cfg::kBlock + Cfg::kSignExt) * (Cfg::kBlock / 8) : 0;
+  a.sign_table = !signs.mask                                                 ? 0
+                 : Cfg::kSignTable && table_bytes <= Cfg::kSignTableMax      ? 1
+                 : !Cfg::kSignTable && word_bytes <= Cfg::kMaskSmemMax       ? 2
+                                                                             : 0;
+  a.sign_smem = a.sign_table == 1                 ? static_cast<int>(table_bytes)
+                : a.sign_table == 2               ? static_cast<int>(word_bytes)
                 : mask_bytes <= Cfg::kMaskSmemMax ? static_cast<int>(mask_bytes)
                                                   : 0;
   CUtensorMap map;

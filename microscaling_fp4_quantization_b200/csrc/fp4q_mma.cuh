@@ -106,6 +106,19 @@ struct MmaConfig {
   static constexpr bool kSignTable = kCtasPerSm == 1;
   static constexpr int kSignTableMax = kSignTable ? cmin(kMaskRoom, 65536) : 0;
   static constexpr int kSignSmemMax = cmax(kMaskSmemMax, kSignTableMax);
+  // The sign warps' walk over a stage: a region (the whole stage in the bulk layout, one K-half
+  // of swizzled 128-byte rows otherwise) holds kSignCpr 16-byte chunks per row; a lane's chunks
+  // sit kSignRowStep rows apart, kSignPerLane of them per region.
+  static constexpr int kSignCpr = kBulk ? B / 8 : 8;
+  static constexpr int kSignRegions = kBulk ? 1 : kHalves;
+  static constexpr int kSignLaneStride = 32 * kSignWarps;
+  static constexpr int kSignRowStep = kSignLaneStride / kSignCpr;
+  static constexpr int kSignPerLane = kStageBytes / kSignRegions / 16 / kSignLaneStride;
+  // Where two CTAs share the SM, the sign warps read a word table when it fits: one 32-bit
+  // word per 8-channel chunk (bit 15 - i holds the sign of element 2i, bit 31 - i that of
+  // element 2i + 1), for blocks 0 .. K/b - 1 + kSignExt, block k >= K/b repeating block
+  // k - K/b, so that a lane's chunks of a stage sit at fixed offsets from its first.
+  static constexpr int kSignExt = (kSignPerLane - 1) * kSignRowStep;
   static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(B >> 3) << 17) |
                                      (static_cast<uint32_t>(128 >> 4) << 24);
 };
@@ -123,7 +136,7 @@ struct MmaArgs {
   const uint8_t* sign_bytes;   // per-channel signs (bit k of byte k / 8 negates channel k), or null
   int64_t sign_upr;            // Hadamard blocks per matrix row, K / b
   int sign_smem;               // bytes staged in shared memory (0: the mask is read from global)
-  int sign_table;              // 1: those bytes are the expanded sign table, 0: the mask's words
+  int sign_table;              // those bytes are: 1 the expanded sign table, 2 the word table, 0 the mask's words
   uint8_t* macro;              // MBS-Static: the macro-scale bytes [R * b / 128]
   // error pass only: [gridDim.x][2] per-CTA signal, error energies; the ticket counter (0
   // between calls, reset by the last CTA); out [3] = signal, error, QSNR dB
@@ -534,12 +547,12 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
     // row; a lane's chunks sit kRowStep rows apart and, as kRowStep is a multiple of the
     // 8-row swizzle period, all carry the same logical chunk q of their rows.
     if (a.sign_bytes != nullptr) {
-      constexpr int kCpr = Cfg::kBulk ? B / 8 : 8;                 // chunks per row of a region
-      constexpr int kRegions = Cfg::kBulk ? 1 : Cfg::kHalves;
+      constexpr int kCpr = Cfg::kSignCpr;                          // chunks per row of a region
+      constexpr int kRegions = Cfg::kSignRegions;
       constexpr int kRegionBytes = Cfg::kStageBytes / kRegions;
-      constexpr int kLaneStride = 32 * Cfg::kSignWarps;            // chunks between a lane's chunks
-      constexpr int kRowStep = kLaneStride / kCpr;
-      constexpr int kPerLane = kRegionBytes / 16 / kLaneStride;    // chunks per lane per region
+      constexpr int kLaneStride = Cfg::kSignLaneStride;            // chunks between a lane's chunks
+      constexpr int kRowStep = Cfg::kSignRowStep;
+      constexpr int kPerLane = Cfg::kSignPerLane;                  // chunks per lane per region
       constexpr int kBatch = Cfg::kCtasPerSm == 1 ? 4 : 8;
       static_assert(kLaneStride % kCpr == 0 && (Cfg::kBulk || kRowStep % 8 == 0), "lane chunk walk");
       static_assert(kPerLane % kBatch == 0, "whole batches per region");
@@ -556,12 +569,40 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
       const uint32_t row0_kb = row0 % upr;
       uint32_t tile_kb = static_cast<uint32_t>((static_cast<uint64_t>(blockIdx.x) * Cfg::kRowsPerTile) % upr);
       const uint32_t tab_s = stage0 + Cfg::kMaskOffset;
+      // the mask words behind this lane's table entries: word 32 sw + lane + k * kLaneStride
+      // (ceil(chunks / 4) words in all), loaded together
+      auto load_mask_words = [&](auto& mw, uint32_t chunks) {
+        const uint32_t* mg = reinterpret_cast<const uint32_t*>(a.sign_bytes);
+        const uint32_t nw = (chunks + 3) / 4;
+        constexpr int N = sizeof(mw) / sizeof(mw[0]);
+#pragma unroll
+        for (int k = 0; k < N; ++k) {
+          const uint32_t w = 32u * sw + lane + static_cast<uint32_t>(k * kLaneStride);
+          mw[k] = w < nw ? __ldg(mg + w) : 0u;
+        }
+      };
       if constexpr (Cfg::kSignTable) {
-        if (a.sign_table) {
-          // the expanded table: entry e (and e + K/8) = the XOR words of mask byte e
+        if (a.sign_table == 1) {
+          // the expanded table: entry e (and e + K/8) = the XOR words of mask byte e; every
+          // mask word a lane needs is loaded before any is used (one memory latency, not one
+          // per word)
           const uint32_t chunks = upr * (B / 8);
-          for (uint32_t e = 32 * sw + lane; e < 2 * chunks; e += 32 * Cfg::kSignWarps)
-            sts128_u4(tab_s + 16u * e, chunk_sign_xor(__ldg(a.sign_bytes + (e < chunks ? e : e - chunks))));
+          constexpr int kWordsPerLane = (Cfg::kSignTableMax / 32 / 4 + kLaneStride - 1) / kLaneStride;
+          uint32_t mw[kWordsPerLane];
+          load_mask_words(mw, chunks);
+#pragma unroll
+          for (int k = 0; k < kWordsPerLane; ++k) {
+            const uint32_t e0 = 4u * (32u * sw + lane + static_cast<uint32_t>(k * kLaneStride));
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t e = e0 + j;
+              if (e < chunks) {
+                const uint4 f = chunk_sign_xor((mw[k] >> (8 * j)) & 0xFFu);
+                sts128_u4(tab_s + 16u * e, f);
+                sts128_u4(tab_s + 16u * (e + chunks), f);
+              }
+            }
+          }
           asm volatile("bar.sync 2, %0;" ::"r"(32 * Cfg::kSignWarps) : "memory");
           static_assert(kRegions == 1 && kPerLane % kBatch == 0, "one region, whole batches");
           // byte offsets, in the table, of the lane's chunks relative to its first: chunk u sits
@@ -604,6 +645,69 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
           }
         }
       }
+      if constexpr (!Cfg::kSignTable) {
+        if (a.sign_table == 2) {
+          // the word table: word e = the sign word of mask byte e mod (K/8); the mask words
+          // are all loaded first, as for the expanded table
+          const uint32_t chunks = upr * (B / 8);
+          const uint32_t words = (upr + static_cast<uint32_t>(Cfg::kSignExt)) * (B / 8);
+          constexpr int kWordsPerLane = (Cfg::kMaskSmemMax / 4 / 4 + kLaneStride - 1) / kLaneStride;
+          uint32_t mw[kWordsPerLane];
+          load_mask_words(mw, chunks);
+#pragma unroll
+          for (int k = 0; k < kWordsPerLane; ++k) {
+            const uint32_t e0 = 4u * (32u * sw + lane + static_cast<uint32_t>(k * kLaneStride));
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t w = chunk_sign_word((mw[k] >> (8 * j)) & 0xFFu);
+              if (e0 + j < chunks)
+                for (uint32_t e = e0 + j; e < words; e += chunks) sts32(tab_s + 4u * e, w);
+            }
+          }
+          asm volatile("bar.sync 2, %0;" ::"r"(32 * Cfg::kSignWarps) : "memory");
+          constexpr uint32_t kWordStep = 4u * kRowStep * (B / 8);    // table bytes between a lane's chunks
+          int64_t i = 0;
+          for (int64_t t = blockIdx.x; t < n_super; t += gridDim.x, ++i) {
+            const int s = static_cast<int>(i % S);
+            const uint32_t ph = static_cast<uint32_t>((i / S) & 1);
+            uint32_t kb_first = tile_kb + row0_kb;
+            if (kb_first >= upr) kb_first -= upr;
+            tile_kb += tile_step;
+            if (tile_kb >= upr) tile_kb -= upr;
+            const bool mine = mbar_wait_bounded(full_bar(s), ph);
+            if (!__all_sync(0xFFFFFFFFu, mine)) break;
+#pragma unroll 1
+            for (int h = 0; h < kRegions; ++h) {
+              // logical chunk of the lane's rows: the bulk layout is unswizzled; a swizzled row's
+              // physical chunk is its logical one XOR (row & 7)
+              const uint32_t q = Cfg::kBulk ? pq : 8u * h + (pq ^ (row0 & 7u));
+              uint32_t tb = tab_s + 4u * (kb_first * (B / 8) + q);
+              uint32_t addr = stage0 + s * Cfg::kStageBytes + h * kRegionBytes + 16u * c0;
+#pragma unroll 1
+              for (int j = 0; j < kPerLane; j += kBatch) {
+                uint4 w[kBatch];
+                uint32_t m[kBatch];
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u) {
+                  m[u] = lds32(tb + kWordStep * u);
+                  w[u] = lds128(addr + 16u * kLaneStride * u);
+                }
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u) {
+                  const uint4 f = chunk_sign_xor_word(m[u]);
+                  sts128_u4(addr + 16u * kLaneStride * u,
+                            make_uint4(w[u].x ^ f.x, w[u].y ^ f.y, w[u].z ^ f.z, w[u].w ^ f.w));
+                }
+                tb += kWordStep * kBatch;
+                addr += 16u * kLaneStride * kBatch;
+              }
+            }
+            fence_proxy_async_smem();   // the tensor core reads the stage through the async proxy
+            __syncwarp();
+            if (lane == 0) mbar_arrive(signed_bar(s));
+          }
+        }
+      }
       const uint8_t* mask_g = a.sign_bytes;
       const bool staged = a.sign_smem > 0;
       const uint32_t mask_s = tab_s;
@@ -616,7 +720,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
         asm volatile("bar.sync 2, %0;" ::"r"(32 * Cfg::kSignWarps) : "memory");
       }
       int64_t i = 0;
-      for (int64_t t = blockIdx.x; !a.sign_table && t < n_super; t += gridDim.x, ++i) {
+      for (int64_t t = blockIdx.x; a.sign_table == 0 && t < n_super; t += gridDim.x, ++i) {
         const int s = static_cast<int>(i % S);
         const uint32_t ph = static_cast<uint32_t>((i / S) & 1);
         uint32_t kb_first = tile_kb + row0_kb;
