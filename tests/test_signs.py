@@ -149,6 +149,35 @@ def test_signed_rows_longer_than_the_staged_mask(F, combo, kernel):
     assert_parity(res, out["codes"], out["scales"], f"{combo_id(combo)} K={K} signed")
 
 
+SIGN_SOURCE_CASES = [((o.NVFP4, 16, 16, o.SCALE_NV_STATIC), 4096), ((o.NVFP4, 16, 16, o.SCALE_NV_STATIC), 32768),
+                     ((o.NVFP4, 16, 64, o.SCALE_NV_DYNAMIC), 32768), ((o.MXFP4, 32, 32, o.SCALE_CEIL_NOCLIP), 4096),
+                     ((o.MXFP4, 32, 32, o.SCALE_CEIL_NOCLIP), 32768), ((o.MXFP4, 32, 128, o.SCALE_FLOOR_OCP), 8192),
+                     ((o.MXFP4, 32, 128, o.SCALE_FLOOR_OCP), 32768), ((o.NVFP4, 16, 128, o.SCALE_NV_STATIC), 14336),
+                     ((o.NVFP4, 16, 128, o.SCALE_NV_STATIC), 32768)]
+
+
+@pytest.mark.parametrize("combo,K", SIGN_SOURCE_CASES,
+                         ids=[f"{combo_id(c)}-K{K}" for c, K in SIGN_SOURCE_CASES])
+def test_tensor_core_sign_sources(F, combo, K):
+    """The tensor-core kernel reads the signs from one of three shared-memory sources, chosen
+    by K: the expanded table (one CTA per SM, 4 K bytes up to 64 KB: NVFP4 b <= 64, K <= 16384),
+    the word table (two CTAs per SM, while it fits beside them: K = 4096 at b = 32, K = 8192 and
+    14336 at b = 128) and the mask's bytes (K = 32768 in every configuration).  Each against the
+    oracle, on every row kind."""
+    import gpu_util as gu
+    fmt, g, b, rule = combo
+    M = 40
+    plan, s = signed_plan(F, combo, K, seed=90 + b)
+    F.fp4q_plan_set_kernel(plan, F.FP4Q_KERNEL_TENSOR_CORE)
+    x = make_input(M, K, seed=4545 + b + K, adversarial=True)
+    s_g = o.nv_tensor_scale(o.rotated_amax(x, b, signs=s)) if rule == o.SCALE_NV_STATIC else None
+    res = o.rotate_quantize(x, fmt, g, b, rule, tensor_scale=s_g, signs=s)
+    out = gu.run_rotate_quantize(F, plan, x, tensor_scale=s_g, dump=True)
+    assert_parity(res, out["codes"], out["scales"], f"{combo_id(combo)} {M}x{K} signed, tensor core",
+                  count_bound=False)
+    assert rotated_value_error(out["y"], res) <= 1e-5, (M, K)
+
+
 @pytest.mark.parametrize("b,kernel", [(16, 1), (128, 1), (16, 2), (128, 2)],
                          ids=["b16-bf", "b128-bf", "b16-tc", "b128-tc"])
 def test_unstaged_mask_on_every_signed_path(F, b, kernel):
