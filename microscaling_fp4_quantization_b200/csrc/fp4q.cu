@@ -206,7 +206,21 @@ fp4q_status amax_grid(int b, int* n) {
   });
 }
 
-fp4q_status launch_amax(fp4q_plan p, const uint16_t* x, int64_t n_elems, cudaStream_t stream) {
+// The amax pass runs on the tensor-core kernel where the plan's rotate + quantize calls would
+// (b >= 16; AUTO from kMmaMinElems elements on): its 32 KB stages keep HBM busier than the
+// butterfly kernel's 2 KB copies.  A plan held to the butterfly kernel keeps its amax pass
+// there too, so that its maxima come from the same fp32 sums.
+fp4q_status launch_amax(fp4q_plan p, const uint16_t* x, int64_t n_elems, int64_t K, cudaStream_t stream) {
+  const bool tc = p->block >= 16 && n_elems / p->block < kMmaMaxRows && p->kernel != FP4Q_KERNEL_BUTTERFLY &&
+                  (p->kernel == FP4Q_KERNEL_TENSOR_CORE || n_elems >= kMmaMinElems);
+  if (tc) {
+    return with_block(p->block, [&]<int B>() -> fp4q_status {
+      if constexpr (B >= 16)
+        return launch_mma_amax<MmaConfig<kNV, B, kRuleNvStatic, false, false, true>>(
+            x, n_elems, p->partials, p->n_partials, ChannelSigns{p->signs, 1, 0}, stream, K);
+      return FP4Q_ERR_UNSUPPORTED;
+    });
+  }
   return with_block(p->block, [&]<int B>() -> fp4q_status {
     if (n_elems % AmaxCfg<B, 32>::kE == 0)
       return launch_amax_cfg<AmaxCfg<B, 32>>(x, n_elems, p->partials, p->n_partials,
@@ -253,7 +267,7 @@ fp4q_status rotate_quantize_impl(fp4q_plan p, const void* x, int64_t M, int64_t 
   a.signs = ChannelSigns{p->signs, 1, 0};
   a.macro = static_cast<uint8_t*>(macro);
   if (p->format == FP4Q_NVFP4 && p->rule == FP4Q_SCALE_NV_DYNAMIC) {
-    st = launch_amax(p, a.x, n, s);
+    st = launch_amax(p, a.x, n, K, s);
     if (st != FP4Q_OK) return st;
   }
   if (use_mma(p, n)) {
@@ -600,7 +614,7 @@ fp4q_status fp4q_amax(fp4q_plan plan, const void* x_bf16, int64_t M, int64_t K, 
   if (M * K > 0 && !x_bf16) return FP4Q_ERR_ARG;
   if ((x_bf16 && !aligned(x_bf16, 16)) || !aligned(tensor_scale_out, 4)) return FP4Q_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = launch_amax(plan, static_cast<const uint16_t*>(x_bf16), M * K, s);
+  st = launch_amax(plan, static_cast<const uint16_t*>(x_bf16), M * K, K, s);
   if (st != FP4Q_OK) return st;
   return launch_tensor_scale_finalize(plan->partials, plan->n_partials, tensor_scale_out, s);
 }
@@ -637,7 +651,7 @@ fp4q_status fp4q_quant_error(fp4q_plan plan, const void* x_bf16, int64_t M, int6
   a.ticket = reinterpret_cast<unsigned int*>(plan->err_partials + 2 * static_cast<int64_t>(plan->n_err_partials));
   a.out = out;
   if (plan->format == FP4Q_NVFP4 && plan->rule == FP4Q_SCALE_NV_DYNAMIC) {
-    st = launch_amax(plan, a.x, n, s);
+    st = launch_amax(plan, a.x, n, K, s);
     if (st != FP4Q_OK) return st;
   }
   if (use_mma(plan, n)) {

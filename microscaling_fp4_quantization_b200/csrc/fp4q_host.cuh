@@ -132,6 +132,11 @@ template <class Cfg>
 fp4q_status launch_mma(const uint16_t* x, int64_t n_elems, const RQArgs& ra, cudaStream_t stream, int64_t K);
 template <class Cfg>
 fp4q_status launch_mma_qe(const QEArgs& qa, int64_t n_elems, cudaStream_t stream, int64_t K, int max_ctas);
+// The amax pass on the tensor-core kernel: slots entries of partials, one per CTA of a grid of
+// at most that many (the rest zero).
+template <class Cfg>
+fp4q_status launch_mma_amax(const uint16_t* x, int64_t n_elems, float* partials, int slots, const ChannelSigns& signs,
+                            cudaStream_t stream, int64_t K);
 template <class Cfg>
 fp4q_status launch_qe(fp4q_plan p, QEArgs a, int64_t n_elems, double* out, cudaStream_t stream);
 // CTAs of one full wave of a configuration's error kernel / amax kernel.

@@ -1,5 +1,5 @@
-// Explicit instantiations of the tensor-core (tcgen05) error pass: the rotate + quantize kernel
-// with the epilogue that accumulates energies.  One kernel family per translation unit, so
+// Explicit instantiations of the tensor-core (tcgen05) error pass and amax pass: the rotate +
+// quantize kernel with the epilogue that accumulates energies, or keeps the largest magnitude.  One kernel family per translation unit, so
 // that the library's kernels compile in parallel (see fp4q_host.cuh).
 #include "fp4q_launch.cuh"
 
@@ -15,6 +15,12 @@ namespace host {
 FP4Q_MMA_QE_MX(32) FP4Q_MMA_QE_MX(64) FP4Q_MMA_QE_MX(128)
 FP4Q_MMA_QE_MBS(32) FP4Q_MMA_QE_MBS(64) FP4Q_MMA_QE_MBS(128)
 FP4Q_MMA_QE_NV(16) FP4Q_MMA_QE_NV(32) FP4Q_MMA_QE_NV(64) FP4Q_MMA_QE_NV(128)
+
+// the amax pass (the NVFP4 configuration, epilogue keeping the largest magnitude)
+#define FP4Q_MMA_AMAX(B)                                                                                 \
+  template fp4q_status launch_mma_amax<MmaConfig<kNV, B, kRuleNvStatic, false, false, true>>(            \
+      const uint16_t*, int64_t, float*, int, const ChannelSigns&, cudaStream_t, int64_t);
+FP4Q_MMA_AMAX(16) FP4Q_MMA_AMAX(32) FP4Q_MMA_AMAX(64) FP4Q_MMA_AMAX(128)
 
 }  // namespace host
 }  // namespace fp4q

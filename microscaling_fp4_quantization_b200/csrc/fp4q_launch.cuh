@@ -116,6 +116,15 @@ fp4q_status launch_mma_qe(const QEArgs& qa, int64_t n_elems, cudaStream_t stream
 }
 
 template <class Cfg>
+fp4q_status launch_mma_amax(const uint16_t* x, int64_t n_elems, float* partials, int slots, const ChannelSigns& signs,
+                            cudaStream_t stream, int64_t K) {
+  MmaArgs a = {};
+  a.amax_out = partials;
+  a.amax_slots = slots;
+  return launch_mma_common<Cfg>(a, x, n_elems, signs, stream, K, slots);
+}
+
+template <class Cfg>
 fp4q_status qe_wave(int* n) {
   KernelInfo ki;
   fp4q_status r = butterfly_kernel_info<Cfg>(quant_error_kernel<Cfg>, &ki);

@@ -37,14 +37,18 @@ namespace fp4q {
 
 // QE: the error pass.  The epilogue makes the same scale decisions and codes as the quantizer
 // and accumulates the signal and error energies instead of storing anything.
-template <int FMT, int B, int RULE, bool DUMP, bool QE = false>
+// AMAX: the amax pass of the NVFP4 per-tensor scale.  The epilogue keeps only the largest
+// magnitude of the rotated sums and each CTA writes its maximum, scaled by 1/sqrt(b).
+template <int FMT, int B, int RULE, bool DUMP, bool QE = false, bool AMAX = false>
 struct MmaConfig {
   static constexpr int kFmt = FMT;
   static constexpr int kBlock = B;
   static constexpr int kRule = RULE;
   static constexpr bool kDump = DUMP;
   static constexpr bool kQE = QE;
+  static constexpr bool kAmax = AMAX;
   static_assert(!(QE && DUMP), "the error pass stores nothing");
+  static_assert(!(AMAX && (QE || DUMP || FMT != kNV)), "the amax pass runs in the NVFP4 configuration alone");
   static constexpr int kGroup = FMT == kNV ? 16 : 32;   // MXFP4 and MBS-Static: 32
   static_assert(B >= 16 && B >= kGroup && B <= 128, "one block holds whole groups");
   // MBS-Static: a 128-element macro block is 128 / b consecutive rows (TMEM lanes of one warp)
@@ -143,6 +147,11 @@ struct MmaArgs {
   double* qe_partials;
   unsigned int* qe_ticket;
   double* qe_out;
+  // amax pass only: amax_out[CTA] = RN(max |rotated sum| / sqrt(b)) of the CTA's rows; CTA 0
+  // also zeroes amax_out[gridDim.x .. amax_slots), so that a reduction over all the slots
+  // sees only this call's maxima
+  float* amax_out;
+  int amax_slots;
 };
 
 // Offset of byte `off` inside a swizzled K-major tile (rows of 32 / 64 / 128 bytes): the
@@ -397,6 +406,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
   __shared__ float s_tensor_scale;
   __shared__ double s_qe[Cfg::kQE ? Cfg::kEpiWarps : 1][2];   // error pass: energies per epilogue warp
   __shared__ bool s_qe_last;
+  __shared__ float s_amax[Cfg::kAmax ? Cfg::kEpiWarps : 1];   // amax pass: maximum per epilogue warp
   pdl_launch_dependents();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
@@ -769,7 +779,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
     const int lane_row = 32 * quarter + lane;
     pdl_wait();   // the tensor scale (or the partial maxima) and the outputs belong to earlier kernels
     float s_g = 1.0f;
-    if constexpr (Cfg::kFmt == kNV) {
+    if constexpr (Cfg::kFmt == kNV && !Cfg::kAmax) {
       constexpr int kEpiThreads = 32 * Cfg::kEpiWarps;
       if (warp == 2) {
         if constexpr (Cfg::kRule == kRuleNvDynamic) {
@@ -806,6 +816,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
     constexpr int EC = Cfg::kEpiCols;                 // 16, 32 or 64 columns
     constexpr int NGW = EC / G;                        // groups per warp slice
     double qe_sig = 0.0, qe_err = 0.0;                 // error pass: this lane's running energies
+    float amax_m = 0.0f;                               // amax pass: this lane's largest |sum|
     int64_t i = 0;
     for (int64_t t = blockIdx.x; t < n_super; t += gridDim.x, ++i) {
       const int d = static_cast<int>(i & 1);
@@ -918,6 +929,19 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
       // The slice holds whole blocks (b < EC), exactly one block (b == EC) or half of one.
       constexpr int BW = B < EC ? B : EC;              // block elements in one slice piece
       constexpr int PIECES = EC / BW;                  // block pieces in the slice
+      if constexpr (Cfg::kAmax) {
+        // magnitudes only: a column's sign flip from the bulk layout does not change them
+#pragma unroll
+        for (int pc = 0; pc < PIECES; ++pc) {
+          const int j = (col0 + pc * BW) / B;
+          const int64_t row = t * Cfg::kRowsPerTile + j * 128 + lane_row;
+          if (row < a.n_rows) {
+#pragma unroll
+            for (int e = 0; e < BW; ++e) amax_m = fmaxf(amax_m, fabsf(v[pc * BW + e]));
+          }
+        }
+        continue;
+      }
       if constexpr (Cfg::kQE) {
         // energies only; a column's sign flip from the bulk layout changes neither v^2 nor
         // (v - q)^2 (E2M1 rounds the magnitude)
@@ -982,6 +1006,22 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
         if (row < a.n_rows) store_piece<Cfg, BW>(a, row, off, words, sbytes);
       }
       (void)NGW;
+    }
+    if constexpr (Cfg::kAmax) {
+      constexpr int kEpiThreads = 32 * Cfg::kEpiWarps;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax_m = fmaxf(amax_m, __shfl_xor_sync(0xFFFFFFFFu, amax_m, o));
+      if (lane == 0) s_amax[warp - 2] = amax_m;
+      asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
+      if (warp == 2 && lane == 0) {
+        float r = 0.0f;
+#pragma unroll
+        for (int w = 0; w < Cfg::kEpiWarps; ++w) r = fmaxf(r, s_amax[w]);
+        // RN(r / sqrt(b)), monotone: the largest of the elements' own RN(sum / sqrt(b))
+        a.amax_out[blockIdx.x] = scale_by_inv_sqrt<B>(r);
+      }
+      if (blockIdx.x == 0)
+        for (int i = static_cast<int>(gridDim.x) + (tid - 64); i < a.amax_slots; i += kEpiThreads) a.amax_out[i] = 0.0f;
     }
     if constexpr (Cfg::kQE) {
       // the CTA's energies (epilogue warps in order), then the last CTA to finish sums the

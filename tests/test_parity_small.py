@@ -153,13 +153,17 @@ def exact_sum_input(M, K, seed):
 def test_amax_equals_the_definition_on_exact_sums(F, b):
     """s_g = fp32(A_t / 2688) with A_t the largest fp32 rotated value: bit for bit, for every
     block size (1 / sqrt(b) irrational for b = 2, 8, 32, 128), through fp4q_amax and through a
-    DYNAMIC plan's own amax pass, on both kernels."""
+    DYNAMIC plan's own amax pass, on both kernels (each runs the amax pass on the kernel its
+    plan names; AUTO on the tensor core from 2^22 elements on, b >= 16)."""
     import gpu_util as gu
-    plan = F.fp4q_plan_create(o.NVFP4, 16, b, o.SCALE_NV_STATIC)
+    kernels = (0, 1, 2) if b >= 16 else (0, 1)
     for i, (M, K) in enumerate([(1, 128), (300, 1024), (2048, 4096)]):
         x = exact_sum_input(M, K, seed=31 * b + i)
         ref = o.nv_tensor_scale(o.rotated_amax(x, b))
-        assert gu.run_amax(F, plan, x) == ref, (b, M, K)
+        for kernel in kernels:
+            plan = F.fp4q_plan_create(o.NVFP4, 16, b, o.SCALE_NV_STATIC)
+            F.fp4q_plan_set_kernel(plan, kernel)
+            assert gu.run_amax(F, plan, x) == ref, (b, M, K, kernel)
         res = o.rotate_quantize(x, o.NVFP4, 16, b, o.SCALE_NV_DYNAMIC)
         for kernel in (1, 2) if b >= 16 else (1,):
             dyn = F.fp4q_plan_create(o.NVFP4, 16, b, o.SCALE_NV_DYNAMIC)
