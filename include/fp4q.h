@@ -185,7 +185,8 @@ fp4q_status fp4q_rotate_quantize_dump(fp4q_plan plan, const void* x_bf16, int64_
 
 /* NVFP4 per-tensor scale: s_g = fp32(max|y| / 2688) over the rotated X (1 for an all-zero
  * X), written to *tensor_scale_out (device fp32).  Uses the plan's block size; needs a
- * plan made with an NV rule. */
+ * plan made with an NV rule.  The pass runs on the kernel the plan's rotate + quantize calls
+ * would use (see fp4q_kernel), so max|y| is taken over the same fp32 sums. */
 fp4q_status fp4q_amax(fp4q_plan plan, const void* x_bf16, int64_t M, int64_t K,
                       float* tensor_scale_out, void* stream);
 
@@ -252,7 +253,8 @@ fp4q_status fp4q_gemm(int format, const void* a_codes, const void* a_scales, con
  * (FP4Q_NVFP4, 16, hadamard_block, FP4Q_SCALE_NV_DYNAMIC): x_bf16 device bf16 [M][K];
  * codes_out device uint8 [M][K/2]; scales_out device uint8 [M][K/16]; tensor_scale_out
  * device fp32, written with the s_g the call used.  The caller still owns and passes every
- * input and output.
+ * input and output.  Both passes run on the butterfly kernel, so the outputs are those of such
+ * a plan held to FP4Q_KERNEL_BUTTERFLY.
  *
  * Scratch: the per-CTA partial maxima live in a fixed array inside this library (4096 fp32
  * values, 16 KB), reserved on every GPU that loads the library until the process exits.
