@@ -305,50 +305,85 @@ __device__ __forceinline__ float abs_max(const float* v) {
   return m;
 }
 
-// Signal and error energy of one group of G rotated sums s, added to fp64 running sums: the
-// same scale byte and quotients as quantize_group (so the same codes), then sum v^2 and
-// sum (v - q)^2 in units of X^2.  A zero NV block scale zeroes every code: the error is then
-// the whole signal, y = s / sqrt(b) in fp64.
+// Error-pass sums of one lane.  For NVFP4 they are kept in fp32 within a super-tile, in units
+// that need no per-group scale: the signal as sum s^2 over the raw sums s (y = s / sqrt(b),
+// so y^2 = s^2 / b, and 1/b is a power of two), the error as sum (v - q)^2 E4M3(byte)^2
+// (X = E4M3(byte) s_g, so X^2 = E4M3(byte)^2 s_g^2); qe_sums_flush converts them to fp64 once
+// per super-tile.  The error of a group with a zero block scale (every code 0: the error is
+// the whole signal) goes to fp64 at once.  MXFP4, whose scales 2^(byte - 127) span more than
+// fp32's range, adds both energies per group in fp64.
+struct QeSums {
+  f32x2 s2;
+  float e_nv;
+  double sig, err;
+};
+
+__device__ __forceinline__ void qe_sums_init(QeSums& q) {
+  q.s2 = f2_pack(0.0f, 0.0f);
+  q.e_nv = 0.0f;
+  q.sig = q.err = 0.0;
+}
+
+template <int B>
+__device__ __forceinline__ void qe_sums_flush(QeSums& q, float s_g) {
+  constexpr double inv_b = 1.0 / B;
+  float a0, a1;
+  f2_unpack(q.s2, a0, a1);
+  q.sig = fma(static_cast<double>(a0 + a1), inv_b, q.sig);
+  const double sg = s_g;
+  q.err = fma(static_cast<double>(q.e_nv), sg * sg, q.err);
+  q.s2 = f2_pack(0.0f, 0.0f);
+  q.e_nv = 0.0f;
+}
+
+// One group of G rotated sums s: the same scale byte and quotients as quantize_group (so the
+// same codes), then its signal and error into the lane's sums.
 template <class Cfg, int G>
-__device__ __forceinline__ void group_energy_mma(const float (&s)[G], const float* nv_tab, float s_g, float nv_den,
-                                                 float nv_rden, double& sig, double& err) {
+__device__ __forceinline__ void group_energy_mma(const float (&s)[G], const float* nv_tab, float nv_den,
+                                                 float nv_rden, QeSums& q) {
   constexpr float c = Cfg::kC;
   f32x2 p[G / 2];
 #pragma unroll
   for (int k = 0; k < G / 2; ++k) p[k] = f2_pack(s[2 * k], s[2 * k + 1]);
   const float A = scale_by_inv_sqrt<Cfg::kBlock>(pairs_amax<G / 2>(p));
   float mult;
-  double X2;
   if constexpr (Cfg::kFmt == kMX) {
+    // both energies per group in fp64 (measured: the fp32 signal sum costs MXFP4 b = 128 more
+    // registers than it saves)
     const int byte = mx_scale_byte<Cfg::kRule>(A);
     mult = c * mx_inv_scale(byte);
-    X2 = mx_scale_sq(byte);
+    const f32x2 mm = f2_pack(mult, mult);
+    f32x2 v[G / 2];
+#pragma unroll
+    for (int k = 0; k < G / 2; ++k) v[k] = f2_mul(p[k], mm);
+    float gs, ge;
+    group_energies<G / 2>(v, gs, ge);
+    const double X2 = mx_scale_sq(byte);
+    q.sig = fma(static_cast<double>(gs), X2, q.sig);
+    q.err = fma(static_cast<double>(ge), X2, q.err);
   } else {
+#pragma unroll
+    for (int k = 0; k < G / 2; ++k) q.s2 = f2_fma(p[k], p[k], q.s2);
     const uint32_t byte = e4m3_encode(div_rn_markstein(A, nv_den, nv_rden));
     mult = nv_tab[byte];
     if (byte == 0u || mult == 0.0f) {
-      constexpr double c64 = inv_sqrt_block_f64(Cfg::kBlock);
-      double e2 = 0.0;
+      f32x2 g2 = f2_pack(0.0f, 0.0f);
 #pragma unroll
-      for (int k = 0; k < G; ++k) {
-        const double y = static_cast<double>(s[k]) * c64;
-        e2 = fma(y, y, e2);
-      }
-      sig += e2;
-      err += e2;
+      for (int k = 0; k < G / 2; ++k) g2 = f2_fma(p[k], p[k], g2);
+      float a0, a1;
+      f2_unpack(g2, a0, a1);
+      q.err = fma(static_cast<double>(a0 + a1), 1.0 / Cfg::kBlock, q.err);
       return;
     }
-    const double S = static_cast<double>(e4m3_decode(byte) * s_g);
-    X2 = S * S;
-  }
-  const f32x2 mm = f2_pack(mult, mult);
-  f32x2 v[G / 2];
+    const f32x2 mm = f2_pack(mult, mult);
+    f32x2 v[G / 2];
 #pragma unroll
-  for (int k = 0; k < G / 2; ++k) v[k] = f2_mul(p[k], mm);
-  float gs, ge;
-  group_energies<G / 2>(v, gs, ge);
-  sig = fma(static_cast<double>(gs), X2, sig);
-  err = fma(static_cast<double>(ge), X2, err);
+    for (int k = 0; k < G / 2; ++k) v[k] = f2_mul(p[k], mm);
+    float gs, ge;
+    group_energies<G / 2>(v, gs, ge);
+    const float dec = e4m3_decode(byte);
+    q.e_nv = fmaf(ge, dec * dec, q.e_nv);
+  }
 }
 
 // One lane's piece of a block: BW codes (BW / 8 code words) from element `off` of block `row`,
@@ -815,7 +850,9 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
     const float nv_rden = __frcp_rn(nv_den);
     constexpr int EC = Cfg::kEpiCols;                 // 16, 32 or 64 columns
     constexpr int NGW = EC / G;                        // groups per warp slice
-    double qe_sig = 0.0, qe_err = 0.0;                 // error pass: this lane's running energies
+    double qe_sig = 0.0, qe_err = 0.0;                 // error pass (MBS): this lane's running energies
+    QeSums qe;                                         // error pass (MXFP4, NVFP4): this lane's sums
+    qe_sums_init(qe);
     float amax_m = 0.0f;                               // amax pass: this lane's largest |sum|
     int64_t i = 0;
     for (int64_t t = blockIdx.x; t < n_super; t += gridDim.x, ++i) {
@@ -955,10 +992,11 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
               float gv[G];
 #pragma unroll
               for (int e = 0; e < G; ++e) gv[e] = v[pc * BW + q * G + e];
-              group_energy_mma<Cfg, G>(gv, nv_tab, s_g, nv_den, nv_rden, qe_sig, qe_err);
+              group_energy_mma<Cfg, G>(gv, nv_tab, nv_den, nv_rden, qe);
             }
           }
         }
+        qe_sums_flush<B>(qe, s_g);
         continue;
       }
 #pragma unroll
@@ -1027,6 +1065,8 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kCtasPerSm)
       // the CTA's energies (epilogue warps in order), then the last CTA to finish sums the
       // per-CTA pairs in CTA order: a fixed order for a fixed grid, so the result is deterministic
       constexpr int kEpiThreads = 32 * Cfg::kEpiWarps;
+      qe_sig += qe.sig;
+      qe_err += qe.err;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
         qe_sig += __shfl_xor_sync(0xFFFFFFFFu, qe_sig, o);
