@@ -7,7 +7,7 @@
 //
 // Work is cut into super-tiles of 128 TMEM columns: 128 / b row-tiles of 128 rows, 16384
 // elements, 32 KB of input.  CTAs are persistent (one or two per SM) and take super-tiles
-// round-robin.  Roles, per CTA of 2 + 8 or 2 + 16 warps:
+// round-robin.  Roles, per CTA of 2 + 8 + 2 or 2 + 16 + 8 warps:
 //   warp 0        producer: for b <= 32 one contiguous bulk copy per stage (left unswizzled,
 //                 see MmaConfig::kBulk), else TMA tensor loads (2-D map over the rows, swizzled
 //                 K-major layout), into a ring of shared-memory stages, completion on mbarriers;
@@ -17,7 +17,11 @@
 //   warps 2..     epilogue: warp w reads TMEM lanes 32 * (w % 4) .. + 31 (tcgen05.ld), one
 //                 column slice of the super-tile each, so each thread owns one row (one rotated
 //                 block, or a part of one) and does the amax, scale, E2M1 rounding, packing and
-//                 stores of it in its registers; it frees the buffer as soon as its slice is read.
+//                 stores of it in its registers; it frees the buffer as soon as its slice is read;
+//                 the error pass and the amax pass keep sums or maxima instead of storing;
+//   the last 2 or 8 warps   sign warps, for plans with per-channel signs only: they flip the
+//                 signs of each landed stage's elements in shared memory (XOR words from a table
+//                 staged once per CTA) before the MMA warp may read it.
 // All roles wait on the grid dependency (programmatic dependent launch) before touching global
 // memory, so the set-up overlaps the end of the kernel this one follows; before it the producer
 // only asks L2 to prefetch its first stages.
