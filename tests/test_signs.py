@@ -178,6 +178,40 @@ def test_tensor_core_sign_sources(F, combo, K):
     assert rotated_value_error(out["y"], res) <= 1e-5, (M, K)
 
 
+def every_byte_mask(K):
+    """Mask words whose 8-channel chunks take every byte value 0 .. 255 in turn (K a multiple
+    of 32): every pattern each kernel's sign expansion can meet."""
+    n = K // 8
+    return np.tile(np.arange(256, dtype=np.uint8), n // 256 + 1)[:n].view(np.uint32).copy()
+
+
+EVERY_BYTE_CASES = [((o.NVFP4, 16, 16, o.SCALE_NV_STATIC), 4096, 2), ((o.NVFP4, 16, 16, o.SCALE_NV_STATIC), 32768, 2),
+                    ((o.MXFP4, 32, 32, o.SCALE_FLOOR_OCP), 4096, 2), ((o.MXFP4, 32, 128, o.SCALE_FLOOR_OCP), 8192, 2),
+                    ((o.MXFP4, 32, 128, o.SCALE_FLOOR_OCP), 32768, 2), ((o.NVFP4, 16, 16, o.SCALE_NV_STATIC), 4096, 1),
+                    ((o.MXFP4, 32, 128, o.SCALE_FLOOR_OCP), 8192, 1)]
+
+
+@pytest.mark.parametrize("combo,K,kernel", EVERY_BYTE_CASES,
+                         ids=[f"{combo_id(c)}-K{K}-{'tc' if k == 2 else 'bf'}" for c, K, k in EVERY_BYTE_CASES])
+def test_every_mask_byte(F, combo, K, kernel):
+    """All 256 values of a chunk's eight sign bits, through each sign source of the tensor-core
+    kernel (expanded table, word table, mask bytes) and through the butterfly kernel."""
+    import gpu_util as gu
+    fmt, g, b, rule = combo
+    M = 16
+    mask = every_byte_mask(K)
+    plan = F.fp4q_plan_create(fmt, g, b, rule)
+    F.fp4q_plan_set_signs(plan, torch.from_numpy(mask.view(np.int32)).cuda(), K)
+    F.fp4q_plan_set_kernel(plan, kernel)
+    s = o.sign_vector(mask, K)
+    x = make_input(M, K, seed=4646 + b + K, adversarial=False)
+    s_g = o.nv_tensor_scale(o.rotated_amax(x, b, signs=s)) if rule == o.SCALE_NV_STATIC else None
+    res = o.rotate_quantize(x, fmt, g, b, rule, tensor_scale=s_g, signs=s)
+    out = gu.run_rotate_quantize(F, plan, x, tensor_scale=s_g, dump=True)
+    assert_parity(res, out["codes"], out["scales"], f"{combo_id(combo)} {M}x{K} every mask byte, kernel {kernel}")
+    assert rotated_value_error(out["y"], res) <= 1e-5, (M, K)
+
+
 @pytest.mark.parametrize("b,kernel", [(16, 1), (128, 1), (16, 2), (128, 2)],
                          ids=["b16-bf", "b128-bf", "b16-tc", "b128-tc"])
 def test_unstaged_mask_on_every_signed_path(F, b, kernel):
