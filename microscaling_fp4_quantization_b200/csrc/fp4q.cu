@@ -211,8 +211,9 @@ fp4q_status amax_grid(int b, int* n) {
 // butterfly kernel's 2 KB copies.  A plan held to the butterfly kernel keeps its amax pass
 // there too, so that its maxima come from the same fp32 sums.
 fp4q_status launch_amax(fp4q_plan p, const uint16_t* x, int64_t n_elems, int64_t K, cudaStream_t stream) {
-  const bool tc = p->block >= 16 && n_elems / p->block < kMmaMaxRows && p->kernel != FP4Q_KERNEL_BUTTERFLY &&
-                  (p->kernel == FP4Q_KERNEL_TENSOR_CORE || n_elems >= kMmaMinElems);
+  // (an empty tensor takes the butterfly kernel, whose fixed grid writes every slot)
+  const bool tc = n_elems > 0 && p->block >= 16 && n_elems / p->block < kMmaMaxRows &&
+                  p->kernel != FP4Q_KERNEL_BUTTERFLY && (p->kernel == FP4Q_KERNEL_TENSOR_CORE || n_elems >= kMmaMinElems);
   if (tc) {
     return with_block(p->block, [&]<int B>() -> fp4q_status {
       if constexpr (B >= 16)

@@ -180,3 +180,16 @@ def test_empty_input_is_a_no_op(F):
     F.fp4q_rotate_quantize(plan, 0, 16, 0, 0, 0, None)
     torch.cuda.synchronize()
     assert F.fp4q_device_status() == F.FP4Q_OK
+
+
+@pytest.mark.parametrize("kernel", [0, 1, 2])
+def test_amax_of_an_empty_tensor_is_one(F, kernel):
+    """s_g of an empty X is 1 (the all-zero rule), whichever kernel the plan names."""
+    import torch
+    plan = F.fp4q_plan_create(o.NVFP4, 16, 16, o.SCALE_NV_STATIC)
+    F.fp4q_plan_set_kernel(plan, kernel)
+    ts = torch.full((1,), -1.0, dtype=torch.float32, device="cuda")
+    F.fp4q_amax(plan, 0, 0, 4096, ts)
+    torch.cuda.synchronize()
+    assert F.fp4q_device_status() == F.FP4Q_OK
+    assert ts.item() == 1.0
